@@ -1,0 +1,100 @@
+// Row-wise pieces of the shared block (pre-norm layer): RMSNorm into the GEMM operand
+// type, RoPE (rotate-half, theta) splitting the fused q/k/v projection, and the SwiGLU
+// product. The pages (FlashLoop §1) name the looped block but not its layer; these are
+// the standard pre-norm decoder choices.
+#include "fl_internal.cuh"
+
+namespace fl {
+namespace {
+
+template <typename T>
+__global__ void __launch_bounds__(256) k_rmsnorm(const float* __restrict__ x,
+                                                 const float* __restrict__ gamma, float eps,
+                                                 T* __restrict__ out, int d) {
+  const int row = blockIdx.x;
+  const float* xr = x + (size_t)row * d;
+  float ss = 0.f;
+  for (int e = threadIdx.x; e < d; e += blockDim.x) ss = fmaf(xr[e], xr[e], ss);
+  __shared__ float red[8];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += red[i];
+  const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+  T* o = out + (size_t)row * d;
+  for (int e = threadIdx.x; e < d; e += blockDim.x) o[e] = from_f32<T>(xr[e] * inv * gamma[e]);
+}
+
+// qkv [M][3d] -> q, k (rotated) and v [M][H][hd]; angle = pos * theta^(-2i/hd) in fp64.
+__global__ void k_rope_split(const float* __restrict__ qkv, const int32_t* __restrict__ pos,
+                             int M, int H, int hd, float theta, float* __restrict__ q,
+                             float* __restrict__ k, float* __restrict__ v) {
+  const int half = hd / 2;
+  const size_t total = (size_t)M * H * half;
+  const int d = H * hd;
+  for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
+       id += (size_t)gridDim.x * blockDim.x) {
+    const int i = (int)(id % half);
+    const int h = (int)((id / half) % H);
+    const int m = (int)(id / ((size_t)half * H));
+    const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)hd);
+    double sn, cs;
+    sincos((double)pos[m] * inv_freq, &sn, &cs);
+    const float c = (float)cs, s = (float)sn;
+    const float* row = qkv + (size_t)m * 3 * d;
+    const size_t o = (size_t)m * d + (size_t)h * hd;
+    const float qa = row[h * hd + i], qb = row[h * hd + i + half];
+    const float ka = row[d + h * hd + i], kb = row[d + h * hd + i + half];
+    q[o + i] = qa * c - qb * s;
+    q[o + i + half] = qa * s + qb * c;
+    k[o + i] = ka * c - kb * s;
+    k[o + i + half] = ka * s + kb * c;
+    v[o + i] = row[2 * d + h * hd + i];
+    v[o + i + half] = row[2 * d + h * hd + i + half];
+  }
+}
+
+template <typename T>
+__global__ void k_swiglu(const float* __restrict__ gu, int M, int F, T* __restrict__ out) {
+  const size_t total = (size_t)M * F;
+  for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
+       id += (size_t)gridDim.x * blockDim.x) {
+    const size_t m = id / F, f = id % F;
+    const float g = gu[m * 2 * F + f], u = gu[m * 2 * F + F + f];
+    out[id] = from_f32<T>(g / (1.0f + expf(-g)) * u);
+  }
+}
+
+int grid_for(size_t n) {
+  size_t b = (n + 255) / 256;
+  return (int)(b > 148 * 32 ? 148 * 32 : (b == 0 ? 1 : b));
+}
+
+}  // namespace
+
+cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* out,
+                           fl_dtype dt, int M, int d, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (dt == FL_F32) k_rmsnorm<float><<<M, 256, 0, s>>>(x, gamma, eps, (float*)out, d);
+  else k_rmsnorm<__nv_bfloat16><<<M, 256, 0, s>>>(x, gamma, eps, (__nv_bfloat16*)out, d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H, int hd,
+                              float theta, float* q, float* k, float* v, cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  k_rope_split<<<grid_for((size_t)M * H * hd / 2), 256, 0, s>>>(qkv, pos, M, H, hd, theta, q, k, v);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu(const float* gu, int M, int F, void* out, fl_dtype dt,
+                          cudaStream_t s) {
+  if (M <= 0) return cudaSuccess;
+  if (dt == FL_F32) k_swiglu<float><<<grid_for((size_t)M * F), 256, 0, s>>>(gu, M, F, (float*)out);
+  else k_swiglu<__nv_bfloat16><<<grid_for((size_t)M * F), 256, 0, s>>>(gu, M, F, (__nv_bfloat16*)out);
+  return cudaGetLastError();
+}
+
+}  // namespace fl

@@ -1,0 +1,419 @@
+// The C interface (include/fl.h): host-side validation, workspace carving and the
+// launch sequence of each entry point. Nothing here allocates device memory.
+#include <mutex>
+#include <string.h>
+
+#include "fl_internal.cuh"
+
+__device__ int g_fl_status;  // first error recorded by a kernel on this device
+
+namespace fl {
+
+cudaError_t launch_gemm_simt(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
+                             int K, int ldc, GemmEpi epi, cudaStream_t s);
+cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N, int K,
+                           int ldc, GemmEpi epi, cudaStream_t s);
+bool gemm_tc_supported(int M, int N, int K);
+
+int* status_word() {
+  static int* cache[128] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fl_status) != cudaSuccess) return nullptr;
+    cache[dev] = static_cast<int*>(p);
+  }
+  return cache[dev];
+}
+
+cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
+                        int K, int ldc, GemmEpi epi, cudaStream_t s) {
+  if (dt == FL_BF16 && gemm_tc_supported(M, N, K))
+    return launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s);
+  return launch_gemm_simt(dt, A, W, C, M, N, K, ldc, epi, s);
+}
+
+}  // namespace fl
+
+using namespace fl;
+
+namespace {
+
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline fl_status cuda_st(cudaError_t e) { return e == cudaSuccess ? FL_OK : FL_ERR_CUDA; }
+#define FL_TRY(expr)                              \
+  do {                                            \
+    cudaError_t _e = (expr);                      \
+    if (_e != cudaSuccess) return FL_ERR_CUDA;    \
+  } while (0)
+#define FL_CHECK(cond, code) \
+  do {                       \
+    if (!(cond)) return (code); \
+  } while (0)
+
+bool valid_dt(fl_dtype dt) { return dt == FL_F32 || dt == FL_BF16; }
+bool valid_bits(int b) { return b == 0 || b == 2 || b == 4 || b == 8; }
+
+// Carves aligned sub-buffers out of a caller-provided workspace.
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += align_up(bytes);
+    return p;
+  }
+};
+
+fl_status check_kv(const fl_kv_desc* kv) {
+  FL_CHECK(kv, FL_ERR_INVALID_ARG);
+  FL_CHECK(kv->n_tok > 0 && kv->n_tok <= 65535, FL_ERR_SHAPE);
+  FL_CHECK(kv->n_heads > 0, FL_ERR_SHAPE);
+  FL_CHECK(kv->head_dim == 64 || kv->head_dim == 128, FL_ERR_UNSUPPORTED);
+  FL_CHECK(kv->group == 32 || kv->group == 64, FL_ERR_UNSUPPORTED);
+  FL_CHECK(kv->head_dim % kv->group == 0, FL_ERR_SHAPE);
+  FL_CHECK(kv->base_bits == 0 || kv->base_bits == 8, FL_ERR_UNSUPPORTED);
+  FL_CHECK(kv->n_loops >= 1 && kv->n_loops <= FL_MAX_LOOPS, FL_ERR_SHAPE);
+  FL_CHECK(kv->slot, FL_ERR_INVALID_ARG);
+  for (int r = 2; r <= kv->n_loops; ++r) FL_CHECK(valid_bits(kv->res_bits[r]), FL_ERR_UNSUPPORTED);
+  return FL_OK;
+}
+
+fl_status check_model(const fl_model* m) {
+  FL_CHECK(m && m->layers, FL_ERR_INVALID_ARG);
+  FL_CHECK(valid_dt(m->dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(m->n_tok > 0 && m->n_tok <= 65535 && m->n_layers > 0, FL_ERR_SHAPE);
+  FL_CHECK(m->head_dim == 64 || m->head_dim == 128, FL_ERR_UNSUPPORTED);
+  FL_CHECK(m->n_heads > 0 && m->d_model == m->n_heads * m->head_dim, FL_ERR_SHAPE);
+  FL_CHECK(m->d_ffn > 0 && m->d_ffn % 8 == 0 && m->d_model % 8 == 0, FL_ERR_SHAPE);
+  for (int l = 0; l < m->n_layers; ++l) {
+    const fl_layer_weights& w = m->layers[l];
+    FL_CHECK(w.w_qkv && w.w_o && w.w_gate_up && w.w_down && w.g_attn && w.g_ffn,
+             FL_ERR_INVALID_ARG);
+  }
+  return FL_OK;
+}
+
+size_t block_ws(const fl_model* m, int n) {
+  const size_t d = m->d_model, F = m->d_ffn, e = dt_size(m->dt);
+  const size_t qkv_path = align_up(n * d * e) + align_up(n * 3 * d * 4);
+  const size_t ffn_path = align_up(n * d * e) + align_up(n * 2 * F * 4) + align_up(n * F * e);
+  return qkv_path > ffn_path ? qkv_path : ffn_path;
+}
+
+fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int32_t* pos,
+                  float* q, float* k, float* v, void* ws, cudaStream_t s) {
+  const fl_layer_weights& w = m->layers[layer];
+  const int d = m->d_model;
+  Carver c(ws);
+  void* a = c.take((size_t)n * d * dt_size(m->dt));
+  float* qkv = (float*)c.take((size_t)n * 3 * d * 4);
+  FL_TRY(launch_rmsnorm(x, w.g_attn, m->rms_eps, a, m->dt, n, d, s));
+  FL_TRY(launch_gemm(m->dt, a, w.w_qkv, qkv, n, 3 * d, d, 3 * d, EPI_STORE, s));
+  FL_TRY(launch_rope_split(qkv, pos, n, m->n_heads, m->head_dim, m->rope_theta, q, k, v, s));
+  return FL_OK;
+}
+
+fl_status run_out_ffn(const fl_model* m, int layer, float* x, int n, const void* attn, void* ws,
+                      cudaStream_t s) {
+  const fl_layer_weights& w = m->layers[layer];
+  const int d = m->d_model, F = m->d_ffn;
+  Carver c(ws);
+  void* a = c.take((size_t)n * d * dt_size(m->dt));
+  float* gu = (float*)c.take((size_t)n * 2 * F * 4);
+  void* mid = c.take((size_t)n * F * dt_size(m->dt));
+  FL_TRY(launch_gemm(m->dt, attn, w.w_o, x, n, d, d, d, EPI_ADD, s));
+  FL_TRY(launch_rmsnorm(x, w.g_ffn, m->rms_eps, a, m->dt, n, d, s));
+  FL_TRY(launch_gemm(m->dt, a, w.w_gate_up, gu, n, 2 * F, d, 2 * F, EPI_STORE, s));
+  FL_TRY(launch_swiglu(gu, n, F, mid, m->dt, s));
+  FL_TRY(launch_gemm(m->dt, mid, w.w_down, x, n, d, F, d, EPI_ADD, s));
+  return FL_OK;
+}
+
+fl_status check_attn(const fl_attn_args* a) {
+  FL_CHECK(a && a->q && a->q_tok && a->out, FL_ERR_INVALID_ARG);
+  fl_status st = check_kv(a->kv);
+  if (st != FL_OK) return st;
+  FL_CHECK(valid_dt(a->q_dt) && valid_dt(a->out_dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(a->n_q >= 0, FL_ERR_SHAPE);
+  FL_CHECK(a->loop >= 1 && a->loop <= a->kv->n_loops, FL_ERR_SHAPE);
+  if (a->sel) {
+    FL_CHECK(a->mass && a->unsel, FL_ERR_INVALID_ARG);
+    FL_CHECK(a->sel_stride >= 1 && a->stat_rows > 0, FL_ERR_SHAPE);
+    FL_CHECK(a->sel_stride <= 8192, FL_ERR_UNSUPPORTED);
+  }
+  if (a->sel_out) {
+    FL_CHECK(a->mass_out && a->unsel_out, FL_ERR_INVALID_ARG);
+    FL_CHECK(a->k_next >= 0 && a->out_stride >= a->k_next + 1, FL_ERR_SHAPE);
+    FL_CHECK(a->stat_rows > 0, FL_ERR_SHAPE);
+    FL_CHECK(a->stat_kind == FL_STAT_PV || a->stat_kind == FL_STAT_P, FL_ERR_INVALID_ARG);
+    FL_CHECK(a->stat_kind == FL_STAT_P || a->kv->vnorm, FL_ERR_INVALID_ARG);
+    if (a->sel) FL_CHECK(a->out_stride <= a->sel_stride || a->sel_out != a->sel, FL_ERR_SHAPE);
+  }
+  return FL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fl_status_str(fl_status s) {
+  switch (s) {
+    case FL_OK: return "ok";
+    case FL_ERR_INVALID_ARG: return "invalid argument";
+    case FL_ERR_SHAPE: return "bad shape";
+    case FL_ERR_UNSUPPORTED: return "unsupported dtype, bit width or group size";
+    case FL_ERR_CUDA: return "CUDA error";
+    case FL_ERR_TIMEOUT: return "device wait timed out";
+    case FL_ERR_RANGE: return "index out of range or fp16 overflow";
+    case FL_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* fl_version(void) { return "0.1.0"; }
+
+fl_status fl_check_device_status(void* stream) {
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return FL_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_fl_status, sizeof(int)) != cudaSuccess) return FL_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_fl_status, &zero, sizeof(int)) != cudaSuccess) return FL_ERR_CUDA;
+  return (fl_status)v;
+}
+
+size_t fl_select_active_workspace_bytes(int32_t n_rows) {
+  return n_rows > 0 ? align_up((size_t)n_rows * 4) : 0;
+}
+
+fl_status fl_select_active(const void* h_cur, const void* h_prev, fl_dtype dt, int32_t n_rows,
+                           int32_t d, const int32_t* row_tok, int32_t k, int32_t* out_tok,
+                           int32_t* out_pos, float* out_delta, void* ws, size_t ws_bytes,
+                           void* stream) {
+  FL_CHECK(h_cur && h_prev && out_tok, FL_ERR_INVALID_ARG);
+  FL_CHECK(valid_dt(dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(n_rows >= 1 && n_rows <= (1 << 24) && d >= 1, FL_ERR_SHAPE);
+  FL_CHECK(d % (dt == FL_BF16 ? 8 : 4) == 0, FL_ERR_SHAPE);
+  FL_CHECK(k >= 0 && k <= n_rows, FL_ERR_SHAPE);
+  FL_CHECK(((uintptr_t)h_cur % 16 == 0) && ((uintptr_t)h_prev % 16 == 0), FL_ERR_INVALID_ARG);
+  float* delta = out_delta;
+  if (!delta) {
+    FL_CHECK(ws && ws_bytes >= fl_select_active_workspace_bytes(n_rows), FL_ERR_WORKSPACE);
+    delta = static_cast<float*>(ws);
+  }
+  cudaStream_t s = S(stream);
+  FL_TRY(launch_row_delta(h_cur, h_prev, dt, n_rows, d, delta, s));
+  FL_TRY(launch_topk_rows(delta, n_rows, k, row_tok, out_tok, out_pos, status_word(), s));
+  return FL_OK;
+}
+
+fl_status fl_gather_scatter(fl_gs_op op, const void* src, void* dst, const int32_t* idx,
+                            int32_t n_idx, int32_t n_full, int32_t row_elems, fl_dtype dt,
+                            void* stream) {
+  FL_CHECK(op == FL_GATHER || op == FL_SCATTER, FL_ERR_INVALID_ARG);
+  FL_CHECK(valid_dt(dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(n_idx >= 0 && n_full >= 0 && row_elems >= 1, FL_ERR_SHAPE);
+  if (n_idx == 0) return FL_OK;
+  FL_CHECK(src && dst && idx, FL_ERR_INVALID_ARG);
+  return cuda_st(launch_gather_scatter(op, src, dst, idx, n_idx, n_full,
+                                       (size_t)row_elems * dt_size(dt), status_word(), S(stream)));
+}
+
+fl_status fl_kv_residual_quant(const fl_kv_desc* kv, int32_t loop, const void* k_new,
+                               const void* v_new, fl_dtype dt, const int32_t* act_tok,
+                               int32_t n_act, void* stream) {
+  fl_status st = check_kv(kv);
+  if (st != FL_OK) return st;
+  FL_CHECK(k_new && v_new, FL_ERR_INVALID_ARG);
+  FL_CHECK(valid_dt(dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(loop >= 1 && loop <= kv->n_loops, FL_ERR_SHAPE);
+  if (loop == 1) {
+    FL_CHECK(act_tok == nullptr && n_act == kv->n_tok, FL_ERR_SHAPE);
+  } else {
+    FL_CHECK(n_act >= 0 && n_act <= kv->n_tok, FL_ERR_SHAPE);
+    FL_CHECK(n_act == 0 || act_tok, FL_ERR_INVALID_ARG);
+  }
+  const int bits = loop == 1 ? kv->base_bits : kv->res_bits[loop];
+  FL_CHECK(kv->codes[0][loop] && kv->codes[1][loop], FL_ERR_INVALID_ARG);
+  if (bits != 0) FL_CHECK(kv->sz[0][loop] && kv->sz[1][loop], FL_ERR_INVALID_ARG);
+  for (int r = 2; r < loop; ++r) {
+    FL_CHECK(kv->codes[0][r] && kv->codes[1][r], FL_ERR_INVALID_ARG);
+    if (kv->res_bits[r] != 0) FL_CHECK(kv->sz[0][r] && kv->sz[1][r], FL_ERR_INVALID_ARG);
+  }
+  if (loop >= 2) FL_CHECK(kv->codes[0][1] && kv->codes[1][1], FL_ERR_INVALID_ARG);
+  return cuda_st(launch_kv_quant(*kv, loop, k_new, v_new, dt, act_tok, n_act, status_word(),
+                                 S(stream)));
+}
+
+size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a) {
+  return a ? attention_ws_bytes(*a) : 0;
+}
+
+fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream) {
+  fl_status st = check_attn(a);
+  if (st != FL_OK) return st;
+  if (a->n_q == 0) return FL_OK;
+  return cuda_st(launch_attention(*a, status_word(), S(stream)));
+}
+
+size_t fl_block_workspace_bytes(const fl_model* m, int32_t n_rows) {
+  if (!m || n_rows <= 0) return 0;
+  return block_ws(m, n_rows);
+}
+
+fl_status fl_block_qkv(const fl_model* m, int32_t layer, const float* x, int32_t n_rows,
+                       const int32_t* pos, float* q, float* k, float* v, void* ws,
+                       size_t ws_bytes, void* stream) {
+  fl_status st = check_model(m);
+  if (st != FL_OK) return st;
+  FL_CHECK(layer >= 0 && layer < m->n_layers && n_rows >= 0, FL_ERR_SHAPE);
+  if (n_rows == 0) return FL_OK;
+  FL_CHECK(x && pos && q && k && v, FL_ERR_INVALID_ARG);
+  FL_CHECK(ws && ws_bytes >= block_ws(m, n_rows), FL_ERR_WORKSPACE);
+  return run_qkv(m, layer, x, n_rows, pos, q, k, v, ws, S(stream));
+}
+
+fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n_rows,
+                           const void* attn, void* ws, size_t ws_bytes, void* stream) {
+  fl_status st = check_model(m);
+  if (st != FL_OK) return st;
+  FL_CHECK(layer >= 0 && layer < m->n_layers && n_rows >= 0, FL_ERR_SHAPE);
+  if (n_rows == 0) return FL_OK;
+  FL_CHECK(x && attn, FL_ERR_INVALID_ARG);
+  FL_CHECK(ws && ws_bytes >= block_ws(m, n_rows), FL_ERR_WORKSPACE);
+  return run_out_ffn(m, layer, x, n_rows, attn, ws, S(stream));
+}
+
+// ---------------------------------------------------------------- loop step
+static size_t loop_ws_layout(const fl_model* m, Carver* c, int32_t** iota, float** delta,
+                             float** q, float** k, float** v, void** attn, void** blk) {
+  const size_t N = m->n_tok, d = m->d_model;
+  *iota = (int32_t*)c->take(N * 4);
+  *delta = (float*)c->take(N * 4);
+  *q = (float*)c->take(N * d * 4);
+  *k = (float*)c->take(N * d * 4);
+  *v = (float*)c->take(N * d * 4);
+  *attn = c->take(N * d * dt_size(m->dt));
+  *blk = c->take(block_ws(m, (int)N));
+  return c->off;
+}
+
+size_t fl_loop_step_workspace_bytes(const fl_model* m, const fl_schedule* s) {
+  (void)s;
+  if (!m || m->n_tok <= 0) return 0;
+  Carver c(nullptr);
+  int32_t* i; float *dl, *q, *k, *v; void *a, *b;
+  return loop_ws_layout(m, &c, &i, &dl, &q, &k, &v, &a, &b);
+}
+
+fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* sc, int32_t loop,
+                       void* stream) {
+  fl_status rc = check_model(m);
+  if (rc != FL_OK) return rc;
+  FL_CHECK(st && sc && st->h && st->x_cur && st->x_prev && st->kv, FL_ERR_INVALID_ARG);
+  FL_CHECK(sc->n_loops >= 1 && sc->n_loops <= FL_MAX_LOOPS, FL_ERR_SHAPE);
+  FL_CHECK(loop >= 1 && loop <= sc->n_loops, FL_ERR_SHAPE);
+  FL_CHECK(sc->first_sparse >= 2, FL_ERR_SHAPE);
+  const int N = m->n_tok, d = m->d_model, L = m->n_layers;
+  const int R = sc->n_loops;
+  // schedule consistency
+  int prev_k = N;
+  for (int r = 2; r <= R; ++r) {
+    const int kr = sc->n_active[r];
+    FL_CHECK(kr >= 0 && kr <= prev_k, FL_ERR_SHAPE);
+    if (r < sc->first_sparse) FL_CHECK(kr == N, FL_ERR_SHAPE);
+    prev_k = kr;
+    FL_CHECK(sc->col_k[r] >= 0 && sc->col_k[r] + 1 <= (sc->col_k[r] ? st->sel_stride : 1 << 30),
+             FL_ERR_SHAPE);
+    if (sc->col_k[r] > 0 && r > 2 && sc->col_k[r - 1] > 0)
+      FL_CHECK(sc->col_k[r] <= sc->col_k[r - 1], FL_ERR_SHAPE);
+  }
+  FL_CHECK(st->ws && st->ws_bytes >= fl_loop_step_workspace_bytes(m, sc), FL_ERR_WORKSPACE);
+  const bool next_sparse = loop + 1 <= R && sc->col_k[loop + 1] > 0;
+  const bool this_sparse = loop >= 2 && sc->col_k[loop] > 0;
+  if (next_sparse || this_sparse) {
+    FL_CHECK(st->sel && st->mass && st->unsel, FL_ERR_INVALID_ARG);
+    for (int l = 0; l < L; ++l) FL_CHECK(st->sel[l] && st->mass[l] && st->unsel[l], FL_ERR_INVALID_ARG);
+  }
+  for (int l = 0; l < L; ++l) {
+    rc = check_kv(&st->kv[l]);
+    if (rc != FL_OK) return rc;
+    FL_CHECK(st->kv[l].n_tok == N && st->kv[l].n_heads == m->n_heads &&
+             st->kv[l].head_dim == m->head_dim && st->kv[l].n_loops >= R, FL_ERR_SHAPE);
+  }
+  if (loop >= 2) FL_CHECK(st->act[loop] && st->act_pos, FL_ERR_INVALID_ARG);
+
+  cudaStream_t s = S(stream);
+  int* sw = status_word();
+  Carver c(st->ws);
+  int32_t* iota; float *delta, *q, *k, *v; void *attn, *blk;
+  loop_ws_layout(m, &c, &iota, &delta, &q, &k, &v, &attn, &blk);
+  if (st->delta) delta = st->delta;
+  FL_TRY(launch_iota(iota, N, s));
+
+  float* X;
+  int M;
+  const int32_t* act;
+  const size_t row_bytes = (size_t)d * 4;
+  if (loop == 1) {
+    FL_TRY(cudaMemcpyAsync(st->x_prev, st->h, (size_t)N * row_bytes, cudaMemcpyDeviceToDevice, s));
+    X = st->h;
+    M = N;
+    act = iota;
+  } else {
+    M = sc->n_active[loop];
+    int32_t* a_out = st->act[loop];
+    if (loop < sc->first_sparse) {
+      FL_TRY(launch_iota(a_out, N, s));
+      FL_TRY(launch_iota(st->act_pos, N, s));
+    } else {
+      const float* cur;
+      const float* prv = st->x_prev;
+      int rows;
+      const int32_t* row_tok;
+      if (loop == 2) {
+        cur = st->h; rows = N; row_tok = nullptr;
+      } else {
+        cur = st->x_cur; rows = sc->n_active[loop - 1]; row_tok = st->act[loop - 1];
+      }
+      FL_TRY(launch_row_delta(cur, prv, FL_F32, rows, d, delta, s));
+      FL_TRY(launch_topk_rows(delta, rows, M, row_tok, a_out, st->act_pos, sw, s));
+    }
+    act = a_out;
+    FL_TRY(launch_gather_scatter(FL_GATHER, st->h, st->x_prev, act, M, N, row_bytes, sw, s));
+    FL_TRY(cudaMemcpyAsync(st->x_cur, st->x_prev, (size_t)M * row_bytes, cudaMemcpyDeviceToDevice, s));
+    X = st->x_cur;
+  }
+  for (int l = 0; l < L; ++l) {
+    rc = run_qkv(m, l, X, M, act, q, k, v, blk, s);
+    if (rc != FL_OK) return rc;
+    FL_TRY(launch_kv_quant(st->kv[l], loop, k, v, FL_F32, loop == 1 ? nullptr : act, M, sw, s));
+    fl_attn_args a;
+    memset(&a, 0, sizeof(a));
+    a.q = q; a.q_dt = FL_F32; a.n_q = M; a.q_tok = act;
+    a.kv = &st->kv[l]; a.loop = loop; a.col_bias = m->col_bias;
+    a.stat_rows = N; a.sel_stride = st->sel_stride;
+    if (this_sparse) {
+      a.sel = st->sel[l]; a.mass = st->mass[l]; a.unsel = st->unsel[l];
+    }
+    if (next_sparse) {
+      a.k_next = sc->col_k[loop + 1];
+      a.sel_out = st->sel[l]; a.mass_out = st->mass[l]; a.unsel_out = st->unsel[l];
+      a.out_stride = st->sel_stride;
+      a.stat_kind = sc->stat_kind;
+    }
+    a.out = attn; a.out_dt = m->dt;
+    FL_TRY(launch_attention(a, sw, s));
+    rc = run_out_ffn(m, l, X, M, attn, blk, s);
+    if (rc != FL_OK) return rc;
+  }
+  if (loop >= 2)
+    FL_TRY(launch_gather_scatter(FL_SCATTER, st->x_cur, st->h, act, M, N, row_bytes, sw, s));
+  return FL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,142 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "../../include/fl.h"
+
+namespace fl {
+
+// ---------------------------------------------------------------- status word
+// One int per device (a __device__ variable lives once per device context). Kernels
+// receive its address and record the first error with an atomic compare-and-swap.
+int* status_word();   // device address for the current device, nullptr on failure
+
+__device__ __forceinline__ void record_error(int* st, int code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+// ---------------------------------------------------------------- KV store view
+// By-value copy of fl_kv_desc for kernels (loops up to FL_MAX_LOOPS).
+struct KvView {
+  int n_tok, H, hd, g, base_bits, n_loops;
+  int res_bits[FL_MAX_LOOPS + 1];
+  const uint8_t* codes[2][FL_MAX_LOOPS + 1];
+  const uint16_t* sz[2][FL_MAX_LOOPS + 1];
+  const int32_t* slot;
+};
+
+inline KvView make_view(const fl_kv_desc& d) {
+  KvView v;
+  v.n_tok = d.n_tok; v.H = d.n_heads; v.hd = d.head_dim; v.g = d.group;
+  v.base_bits = d.base_bits; v.n_loops = d.n_loops;
+  for (int r = 0; r <= FL_MAX_LOOPS; ++r) {
+    v.res_bits[r] = d.res_bits[r];
+    for (int kv = 0; kv < 2; ++kv) { v.codes[kv][r] = d.codes[kv][r]; v.sz[kv][r] = d.sz[kv][r]; }
+  }
+  v.slot = d.slot;
+  return v;
+}
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+
+// Decode N consecutive elements [e0, e0+N) of one stored row (row `row` of loop
+// r's arrays, head h). The N elements lie in one quantisation group. Codes of b
+// bits sit little-endian, low bits first. Returns deq = fmaf(code, s, z) or the raw
+// binary32 values when bits == 0.
+template <int N>
+__device__ __forceinline__ void decode_run(const KvView& kv, int which, int r, int bits,
+                                           int row, int h, int e0, float* out) {
+  const int hd = kv.hd;
+  if (bits == 0) {
+    const float* p = reinterpret_cast<const float*>(kv.codes[which][r]) +
+                     ((size_t)row * kv.H + h) * hd + e0;
+#pragma unroll
+    for (int i = 0; i < N; ++i) out[i] = p[i];
+    return;
+  }
+  const size_t rowbytes = (size_t)hd * bits / 8;
+  const uint8_t* cp = kv.codes[which][r] + ((size_t)row * kv.H + h) * rowbytes;
+  const uint32_t szw = reinterpret_cast<const uint32_t*>(kv.sz[which][r])
+      [((size_t)row * kv.H + h) * (hd / kv.g) + e0 / kv.g];
+  const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
+  const float z = half_bits_to_float((uint16_t)(szw >> 16));
+  const int mask = (1 << bits) - 1;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const int bit = (e0 + i) * bits;
+    const int code = (cp[bit >> 3] >> (bit & 7)) & mask;
+    out[i] = __fmaf_rn((float)code, s, z);
+  }
+}
+
+// K^ or V^ of token t at loop `upto` for elements [e0, e0+N): base, then every loop
+// 2..upto whose slot table lists t, added in order (a raw loop replaces the value).
+template <int N>
+__device__ __forceinline__ void reconstruct(const KvView& kv, int which, int upto, int t,
+                                            int h, int e0, float* acc) {
+  decode_run<N>(kv, which, 1, kv.base_bits, t, h, e0, acc);
+  for (int r = 2; r <= upto; ++r) {
+    const int row = kv.slot[(size_t)r * kv.n_tok + t];
+    if (row < 0) continue;
+    float d[N];
+    const int bits = kv.res_bits[r];
+    decode_run<N>(kv, which, r, bits, row, h, e0, d);
+    if (bits == 0) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = d[i];
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = __fadd_rn(acc[i], d[i]);
+    }
+  }
+}
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+inline size_t dt_size(fl_dtype dt) { return dt == FL_BF16 ? 2 : 4; }
+inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- internal launches
+// All return cudaSuccess or the launch error. Arguments are validated by callers.
+cudaError_t launch_row_delta(const void* cur, const void* prev, fl_dtype dt, int n_rows,
+                             int d, float* delta, cudaStream_t s);
+cudaError_t launch_topk_rows(const float* delta, int n, int k, const int32_t* row_tok,
+                             int32_t* out_tok, int32_t* out_pos, int* st, cudaStream_t s);
+cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const int32_t* idx,
+                                  int n_idx, int n_full, size_t row_bytes, int* st,
+                                  cudaStream_t s);
+cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
+                            const void* v_new, fl_dtype dt, const int32_t* act_tok, int n_act,
+                            int* st, cudaStream_t s);
+cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s);
+size_t attention_ws_bytes(const fl_attn_args& a);
+
+// C[M x N] (binary32, leading dim ldc) = or += A[M x K] . W[N x K]^T
+enum GemmEpi { EPI_STORE = 0, EPI_ADD = 1 };
+cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
+                        int K, int ldc, GemmEpi epi, cudaStream_t s);
+cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* out,
+                           fl_dtype dt, int M, int d, cudaStream_t s);
+cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H, int hd,
+                              float theta, float* q, float* k, float* v, cudaStream_t s);
+cudaError_t launch_swiglu(const float* gu, int M, int F, void* out, fl_dtype dt,
+                          cudaStream_t s);
+cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s);
+cudaError_t launch_fill_i32(int32_t* p, int32_t v, size_t n, cudaStream_t s);
+
+}  // namespace fl

@@ -1,0 +1,75 @@
+// Row gather / scatter between the full hidden state and compact active-row buffers
+// (FlashLoop §4.4: selected tokens are gathered into compact buffers so the
+// projections stay regular GEMMs; §4.1: results return to their rows and inactive
+// rows keep their state). One CTA per row, 16-byte vector copies when the row size and
+// both base addresses allow it, element copies otherwise.
+#include "fl_internal.cuh"
+
+namespace fl {
+namespace {
+
+template <typename V>
+__global__ void __launch_bounds__(256) k_gather_scatter(int op, const uint8_t* __restrict__ src,
+                                                        uint8_t* __restrict__ dst,
+                                                        const int32_t* __restrict__ idx,
+                                                        int n_full, size_t row_bytes, int* st) {
+  const int i = blockIdx.x;
+  const int j = idx[i];
+  if (j < 0 || j >= n_full) {
+    if (threadIdx.x == 0) record_error(st, FL_ERR_RANGE);
+    return;
+  }
+  const size_t s_row = (op == FL_GATHER) ? (size_t)j : (size_t)i;
+  const size_t d_row = (op == FL_GATHER) ? (size_t)i : (size_t)j;
+  const V* s = reinterpret_cast<const V*>(src + s_row * row_bytes);
+  V* d = reinterpret_cast<V*>(dst + d_row * row_bytes);
+  const size_t n = row_bytes / sizeof(V);
+  for (size_t e = threadIdx.x; e < n; e += blockDim.x) d[e] = s[e];
+}
+
+__global__ void k_fill_i32(int32_t* p, int32_t v, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+__global__ void k_iota(int32_t* p, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    p[i] = i;
+}
+
+}  // namespace
+
+cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const int32_t* idx,
+                                  int n_idx, int n_full, size_t row_bytes, int* st,
+                                  cudaStream_t s) {
+  if (n_idx <= 0) return cudaSuccess;
+  const bool v16 = row_bytes % 16 == 0 && ((uintptr_t)src % 16 == 0) && ((uintptr_t)dst % 16 == 0);
+  const bool v4 = row_bytes % 4 == 0 && ((uintptr_t)src % 4 == 0) && ((uintptr_t)dst % 4 == 0);
+  if (v16)
+    k_gather_scatter<uint4><<<n_idx, 256, 0, s>>>(op, (const uint8_t*)src, (uint8_t*)dst, idx,
+                                                  n_full, row_bytes, st);
+  else if (v4)
+    k_gather_scatter<uint32_t><<<n_idx, 256, 0, s>>>(op, (const uint8_t*)src, (uint8_t*)dst,
+                                                     idx, n_full, row_bytes, st);
+  else
+    k_gather_scatter<uint16_t><<<n_idx, 256, 0, s>>>(op, (const uint8_t*)src, (uint8_t*)dst,
+                                                     idx, n_full, row_bytes, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_i32(int32_t* p, int32_t v, size_t n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  k_fill_i32<<<blocks, 256, 0, s>>>(p, v, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
+  k_iota<<<blocks, 256, 0, s>>>(p, n);
+  return cudaGetLastError();
+}
+
+}  // namespace fl

@@ -1,0 +1,165 @@
+// Cross-loop KV residual quantisation (FlashLoop §3.3, §4.3; Appendix E
+// "Quantization Setting": asymmetric group-wise min/max quantisation, the same
+// scheme for the base state and the residuals).
+//
+// One warp per (row, head, K|V). Lane l holds the hd/32 consecutive elements
+// [l*hd/32, (l+1)*hd/32); a quantisation group of g elements is g/(hd/32) adjacent
+// lanes, reduced with xor shuffles. Every step is an IEEE binary32/binary16 operation
+// with the stated rounding, so the codes are bit-exact against any implementation of
+// the same definition:
+//   z = fp16_RD(min), s = fp16_RU(f32_RU(f32_RU(max - z) / (2^b - 1))),
+//   code = s == 0 ? 0 : clamp(rint(f32_RN(f32_RN(x - z) / s)), 0, 2^b - 1),
+//   deq = fmaf(code, s, z).
+// Loop r >= 2 first rebuilds K^_{r-1} of the row (base + chain) and quantises the
+// residual x = fl32(k - K^_{r-1}). Codes are OR-combined across the lanes that share a
+// 32-bit word and stored little-endian, low bits first.
+#include "fl_internal.cuh"
+
+namespace fl {
+namespace {
+
+struct QuantOut {
+  uint8_t* codes[2];
+  uint16_t* sz[2];
+  int32_t* slot_row;  // slot[loop][*] (loop >= 2) or nullptr
+  float* vnorm;       // [n_tok][H] or nullptr
+};
+
+template <int EPL, typename T>
+__global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int loop,
+                                                  const T* __restrict__ k_new,
+                                                  const T* __restrict__ v_new,
+                                                  const int32_t* __restrict__ act_tok,
+                                                  int n_act, int* st) {
+  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int H = kv.H, hd = kv.hd, g = kv.g;
+  if (gw >= n_act * H * 2) return;
+  const int which = gw % 2;
+  const int h = (gw / 2) % H;
+  const int i = gw / (2 * H);
+  const int t = act_tok ? act_tok[i] : i;
+  if (t < 0 || t >= kv.n_tok) {
+    if (lane == 0) record_error(st, FL_ERR_RANGE);
+    return;
+  }
+  const int e0 = lane * EPL;
+  const T* src = (which == 0 ? k_new : v_new) + ((size_t)i * H + h) * hd + e0;
+  float xin[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) xin[j] = to_f32<T>(src[j]);
+
+  const int bits = loop == 1 ? kv.base_bits : kv.res_bits[loop];
+  float prev[EPL];
+  float x[EPL];
+  if (loop >= 2) {
+    reconstruct<EPL>(kv, which, loop - 1, t, h, e0, prev);
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) x[j] = bits == 0 ? xin[j] : __fsub_rn(xin[j], prev[j]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) x[j] = xin[j];
+  }
+  const int row = loop == 1 ? t : i;
+  float hat[EPL];
+  if (bits == 0) {
+    float* dst = reinterpret_cast<float*>(out.codes[which]) + ((size_t)row * H + h) * hd + e0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { dst[j] = xin[j]; hat[j] = xin[j]; }
+  } else {
+    const int LPG = g / EPL;  // lanes per group
+    float mn = x[0], mx = x[0];
+#pragma unroll
+    for (int j = 1; j < EPL; ++j) { mn = fminf(mn, x[j]); mx = fmaxf(mx, x[j]); }
+    for (int o = 1; o < LPG; o <<= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const __half zh = __float2half_rd(mn);
+    const float zf = __half2float(zh);
+    const float qmax = (float)((1 << bits) - 1);
+    const float t1 = __fsub_ru(mx, zf);
+    const float t2 = __fdiv_ru(t1, qmax);
+    const __half sh = __float2half_ru(t2);
+    const float sf = __half2float(sh);
+    const bool bad = isinf(zf) || isinf(sf) || isnan(zf) || isnan(sf);
+    if (bad && (lane % LPG) == 0) record_error(st, FL_ERR_RANGE);
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      int code = 0;
+      if (!bad && sf != 0.f) {
+        const float w = __fdiv_rn(__fsub_rn(x[j], zf), sf);
+        code = (int)fminf(fmaxf(rintf(w), 0.f), qmax);
+      }
+      const float deq = __fmaf_rn((float)code, sf, zf);
+      hat[j] = loop == 1 ? deq : __fadd_rn(prev[j], deq);
+      word |= (uint32_t)code << (j * bits);
+    }
+    // combine the lanes that share one 32-bit output word
+    const int wbits = EPL * bits;
+    const int LPW = 32 / wbits;
+    word <<= (lane % LPW) * wbits;
+    for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+    const size_t rowbytes = (size_t)hd * bits / 8;
+    if (lane % LPW == 0) {
+      uint32_t* cw = reinterpret_cast<uint32_t*>(out.codes[which] + ((size_t)row * H + h) * rowbytes);
+      cw[lane / LPW] = word;
+    }
+    if (lane % LPG == 0) {
+      uint32_t* szw = reinterpret_cast<uint32_t*>(out.sz[which]);
+      const uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+      szw[((size_t)row * H + h) * (hd / g) + e0 / g] = pair;
+    }
+  }
+  if (which == 1 && out.vnorm) {
+    float ss = 0.f;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) ss = fmaf(hat[j], hat[j], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) out.vnorm[(size_t)t * H + h] = sqrtf(ss);
+  }
+  if (loop >= 2 && which == 0 && h == 0 && lane == 0 && out.slot_row) out.slot_row[t] = i;
+}
+
+template <int EPL>
+cudaError_t launch_epl(const KvView& v, const QuantOut& o, int loop, const void* k,
+                       const void* vv, fl_dtype dt, const int32_t* act, int n_act, int* st,
+                       cudaStream_t s) {
+  const size_t warps = (size_t)n_act * v.H * 2;
+  const int blocks = (int)((warps * 32 + 255) / 256);
+  if (dt == FL_F32)
+    k_kv_quant<EPL, float><<<blocks, 256, 0, s>>>(v, o, loop, (const float*)k,
+                                                  (const float*)vv, act, n_act, st);
+  else
+    k_kv_quant<EPL, __nv_bfloat16><<<blocks, 256, 0, s>>>(
+        v, o, loop, (const __nv_bfloat16*)k, (const __nv_bfloat16*)vv, act, n_act, st);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
+                            const void* v_new, fl_dtype dt, const int32_t* act_tok, int n_act,
+                            int* st, cudaStream_t s) {
+  if (n_act <= 0) return cudaSuccess;
+  KvView v = make_view(kv);
+  QuantOut o;
+  for (int w = 0; w < 2; ++w) { o.codes[w] = kv.codes[w][loop]; o.sz[w] = kv.sz[w][loop]; }
+  o.slot_row = nullptr;
+  o.vnorm = kv.vnorm;
+  cudaError_t e;
+  if (loop >= 2) {
+    o.slot_row = kv.slot + (size_t)loop * kv.n_tok;
+    e = launch_fill_i32(o.slot_row, -1, (size_t)kv.n_tok, s);
+    if (e != cudaSuccess) return e;
+  } else if (kv.slot) {
+    e = launch_iota(kv.slot + kv.n_tok, kv.n_tok, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (kv.head_dim == 128) return launch_epl<4>(v, o, loop, k_new, v_new, dt, act_tok, n_act, st, s);
+  return launch_epl<2>(v, o, loop, k_new, v_new, dt, act_tok, n_act, st, s);
+}
+
+}  // namespace fl

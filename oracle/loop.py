@@ -32,7 +32,8 @@ def run(layers, h0, sched, n_heads, head_dim, bias=None, eps=1e-6, theta=10000.0
     """Run loops 1..R. ``layers`` is a list of weight dicts (see ``block``).
 
     ``select_prev`` optionally maps a loop r to the array used in place of
-    h_{r-2}[A_{r-1}] when that loop ranks tokens (a synthetic previous state).
+    h_{r-2}[A_{r-1}] when that loop ranks tokens (a synthetic previous state), or to
+    a function of the current rows h_{r-1}[A_{r-1}] returning it.
     Returns a dict with per-loop hidden states, active sets, deltas, the per-layer
     KV stores and the statistics after every loop."""
     h0 = np.asarray(h0, np.float64)
@@ -61,7 +62,8 @@ def run(layers, h0, sched, n_heads, head_dim, bias=None, eps=1e-6, theta=10000.0
             cand = out["act"][r - 1]
             hp = out["h"][r - 2][cand]
             if select_prev is not None and r in select_prev:
-                hp = np.asarray(select_prev[r], np.float64)
+                sp = select_prev[r]
+                hp = np.asarray(sp(h_prev[cand]) if callable(sp) else sp, np.float64)
             kr = select.active_count(sched["tok_frac"][r], N, len(cand))
             act, _, delta = select.select_active(h_prev[cand], hp, cand, kr)
             out["delta"][r] = delta

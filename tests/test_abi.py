@@ -1,0 +1,105 @@
+"""The C-ABI library on the CPU: it loads without a GPU, exports every entry point that
+include/fl.h declares, its structs have the layout the C compiler gives them (checked
+against gcc), and host validation rejects bad arguments before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fl.h")
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(fl_[a-z_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    from cross_loop_sparse_step_b200 import fl
+    names = _declared()
+    assert len(names) >= 14
+    out = subprocess.run(["nm", "-D", "--defined-only", fl.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (fl_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        getattr(fl.lib_handle(), n)
+
+
+_LAYOUT_C = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "fl.h"
+#define F(T, m) printf(#T "." #m " %zu\n", offsetof(T, m));
+int main(void) {
+  printf("fl_kv_desc %zu\n", sizeof(fl_kv_desc));
+  F(fl_kv_desc, res_bits) F(fl_kv_desc, codes) F(fl_kv_desc, sz) F(fl_kv_desc, slot) F(fl_kv_desc, vnorm)
+  printf("fl_attn_args %zu\n", sizeof(fl_attn_args));
+  F(fl_attn_args, q_tok) F(fl_attn_args, kv) F(fl_attn_args, sel) F(fl_attn_args, stat_rows)
+  F(fl_attn_args, q_row) F(fl_attn_args, k_next) F(fl_attn_args, out_stride) F(fl_attn_args, out)
+  F(fl_attn_args, ws_bytes)
+  printf("fl_layer_weights %zu\n", sizeof(fl_layer_weights));
+  printf("fl_model %zu\n", sizeof(fl_model));
+  F(fl_model, rms_eps) F(fl_model, layers) F(fl_model, col_bias)
+  printf("fl_schedule %zu\n", sizeof(fl_schedule));
+  F(fl_schedule, n_active) F(fl_schedule, col_k) F(fl_schedule, stat_kind)
+  printf("fl_loop_state %zu\n", sizeof(fl_loop_state));
+  F(fl_loop_state, act) F(fl_loop_state, act_pos) F(fl_loop_state, kv) F(fl_loop_state, sel_stride)
+  F(fl_loop_state, ws) F(fl_loop_state, ws_bytes)
+  return 0;
+}
+"""
+
+
+def test_struct_layouts_match_c():
+    from cross_loop_sparse_step_b200 import fl
+    with tempfile.TemporaryDirectory() as d:
+        src = os.path.join(d, "layout.c")
+        exe = os.path.join(d, "layout")
+        open(src, "w").write(_LAYOUT_C)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), src, "-o", exe], check=True)
+        lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
+    c = dict(l.rsplit(" ", 1) for l in lines if l.strip())
+    py = {"fl_kv_desc": fl.KvDesc, "fl_attn_args": fl.AttnArgs, "fl_layer_weights": fl.LayerWeights,
+          "fl_model": fl.Model, "fl_schedule": fl.Schedule, "fl_loop_state": fl.LoopState}
+    for key, val in c.items():
+        if "." in key:
+            s, m = key.split(".")
+            assert getattr(py[s], m).offset == int(val), key
+        else:
+            assert ctypes.sizeof(py[key]) == int(val), key
+
+
+def test_host_validation_without_gpu():
+    from cross_loop_sparse_step_b200 import fl
+    lib = fl.lib_handle()
+    assert fl.status_str(0) == "ok"
+    assert fl.version().count(".") == 2
+    # null inputs, bad dtype, k out of range: rejected before any CUDA call
+    assert fl._select(None, None, 0, 10, 8, None, 3, None, None, None, None, 0, None) == 1
+    p = ctypes.c_void_p(16)
+    assert fl._select(p, p, 7, 10, 8, None, 3, p, None, None, None, 0, None) == 3
+    assert fl._select(p, p, 0, 10, 8, None, 11, p, None, None, None, 0, None) == 2
+    assert fl._select(p, p, 0, 10, 6, None, 3, p, None, None, None, 0, None) == 2  # d % 4
+    assert fl._select(p, p, 0, 10, 8, None, 3, p, None, None, None, 0, None) == 7  # no workspace
+    assert fl._gs(5, p, p, p, 1, 1, 1, 0, None) == 1
+    assert fl._gs(0, p, p, p, 0, 1, 1, 0, None) == 0    # nothing to do
+    kv = fl.KvDesc()
+    kv.n_tok, kv.n_heads, kv.head_dim, kv.group, kv.base_bits, kv.n_loops = 8, 1, 96, 32, 8, 2
+    kv.slot = 16
+    assert fl._quant(ctypes.byref(kv), 1, p, p, 0, None, 8, None) == 3   # head_dim 96
+    kv.head_dim = 64
+    kv.res_bits[2] = 3
+    assert fl._quant(ctypes.byref(kv), 1, p, p, 0, None, 8, None) == 3   # 3-bit residual
+    kv.res_bits[2] = 4
+    assert fl._quant(ctypes.byref(kv), 1, p, p, 0, p, 8, None) == 2      # act_tok at loop 1
+    assert fl._quant(ctypes.byref(kv), 3, p, p, 0, p, 8, None) == 2      # loop > n_loops
+    assert fl._quant(ctypes.byref(kv), 1, p, p, 0, None, 8, None) == 1   # no code buffers
+    a = fl.AttnArgs()
+    assert fl._attn(ctypes.byref(a), None) == 1

@@ -1,0 +1,478 @@
+#!/usr/bin/env python
+"""Loop-step throughput of the FlashLoop lazy loop step on B200.
+
+Workload (default): the Ouro-1.4B-shaped 4K prefill - 4096 tokens, d_model 2048,
+16 x 128 heads, SwiGLU FFN 5632, 24 shared layers, R = 4 loops, bf16 GEMM operands,
+20% active tokens per sparse loop, 82 carried columns per query plus the sink,
+int8 base + 4-bit residual KV (group 32), a +4 logit bias on 2% of the columns and
+the sink, heavy-tailed (Pareto 1.5) hidden-state changes. Loop 1 (dense, every
+token, the producer of the carried statistics) runs once, untimed; one timed step
+is loops 2..R through fl_loop_step: selection, gather, 24 layers of the block on the
+active rows (QKV + RoPE, residual KV quantisation, sparse attention, O projection,
+FFN), scatter. value = N * (R - 1) / step time: loop-step tokens/s.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: one process per GPU (torchrun); every rank runs an independent replica of
+the workload (the method's prefill loop step has no cross-GPU exchange), time is the
+max over ranks, value the sum of tokens over the max time ("weak" scaling).
+"""
+import argparse
+import ctypes
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "loop-step tokens/s at R loops + % of HBM/tensor roofline; KV bytes/token"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="ouro-1.4b-shape-prefill-4k")
+    ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_uuid):
+        self.uuid = gpu_uuid
+        self.proc = None
+        self.path = os.path.join("/tmp", f"fl_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "200"]
+            if self.uuid:
+                cmd += ["-i", self.uuid]
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        power = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------- workload
+def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
+    N, d, H, hd, F = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn"))
+    L = n_layers or cfg["n_layers"]
+    R = cfg["n_loops"]
+    dev = "cuda"
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+
+    def w(*shape):
+        return (torch.randn(*shape, generator=gen, device=dev) * 0.02).to(torch.bfloat16)
+    layers = [{"w_qkv": w(3 * d, d), "w_o": w(d, d), "w_gate_up": w(2 * F, d), "w_down": w(d, F),
+               "g_attn": torch.ones(d, device=dev), "g_ffn": torch.ones(d, device=dev)}
+              for _ in range(L)]
+    g = synth.rng(seed)
+    bias = torch.from_numpy(synth.col_bias(g, N, cfg["bias_frac"], cfg["bias_value"])).to(dev)
+    n_active = configs.active_counts(cfg)
+    model = fl.LoopModel(layers, N, H, hd, col_bias=bias)
+    res = {r: cfg["res_bits"][r] for r in range(2, R + 1)}
+    stores = [fl.KVStore(N, H, hd, cfg["group"], cfg["base_bits"], res, R, n_active)
+              for _ in range(L)]
+    col_k = {r: cfg["col_k"][r] for r in range(2, R + 1)}
+    sched = fl.make_schedule(R, cfg["first_sparse"], n_active, col_k)
+    run = fl.LoopRunner(model, sched, n_active, stores, max(col_k.values()) + 1)
+    run.h.copy_(torch.from_numpy(synth.embeddings(g, N, d)).to(dev))
+    run.step(1)
+    cur, prev, _ = synth.pareto_delta_pair(g, N, d, 2)
+    run.x_prev.copy_(run.h - torch.from_numpy((cur - prev).astype(np.float32)).to(dev))
+    st = fl.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"loop 1 reported {fl.status_str(st)}")
+    snap = (run.h.clone(), run.x_prev.clone())
+    return dict(run=run, stores=stores, model=model, layers=layers, n_active=n_active, snap=snap,
+                L=L, R=R, N=N, d=d, H=H, hd=hd, F=F, col_k=col_k, res=res)
+
+
+def step_loops(W):
+    for r in range(2, W["R"] + 1):
+        W["run"].step(r)
+
+
+def restore(W):
+    W["run"].h.copy_(W["snap"][0])
+    W["run"].x_prev.copy_(W["snap"][1])
+
+
+def gemm_flops_per_step(W):
+    d, F, L = W["d"], W["F"], W["L"]
+    per_row = 2 * (3 * d * d + d * d + 2 * F * d + F * d)
+    return sum(W["n_active"][r] * per_row * L for r in range(2, W["R"] + 1))
+
+
+def attention_bytes_per_launch(W, torch):
+    """Algorithmic bytes of one sparse-attention launch (one layer of one loop), from
+    the carried column sets: q (fp32), S, m, u read; o (bf16), S', m', u' written;
+    and the compressed KV of the distinct columns each head reads (base K and V plus
+    the residual rows of every loop up to r in which the column was active)."""
+    H, hd, N = W["H"], W["hd"], W["N"]
+    g = W["stores"][0].g
+    out = {}
+    for r in range(2, W["R"] + 1):
+        act = W["run"].act[r][: W["n_active"][r]].long()
+        nq = act.numel()
+        k1 = W["col_k"][r] + 1
+        sel = W["run"].sel[0][:, act].cpu().numpy().view(np.uint16)
+        slot = W["stores"][0].slot.cpu().numpy()
+        kv = 0
+        for h in range(H):
+            cols = np.unique(sel[h][sel[h] != 0xFFFF]).astype(np.int64)
+            kv += len(cols) * 2 * (hd + hd // g * 4)   # base codes + (s, z) for K and V
+            for rr in range(2, r + 1):
+                b = W["res"][rr]
+                nrow = int((slot[rr][cols] >= 0).sum())
+                kv += nrow * 2 * (hd * b // 8 + hd // g * 4)
+        fixed = nq * H * hd * 4 + 2 * (H * nq * k1 * 2 + H * nq * 4 + H * nq * hd * 4) + nq * H * hd * 2
+        flops = 4 * hd * int((sel != 0xFFFF).sum())
+        out[r] = (fixed + kv, flops)
+    return out
+
+
+def kv_bytes(W):
+    tot = sum(s.nbytes(r) for s in W["stores"] for r in range(1, W["R"] + 1))
+    per_tok_layer = tot / (W["N"] * W["L"])
+    dense = W["R"] * 2 * W["d"] * 2
+    return per_tok_layer, dense
+
+
+# ---------------------------------------------------------------- CPU baseline (oracle)
+def oracle_sample(cfg, n_layers=1, rows=256, seed=1):
+    """Times the oracle on a bounded sample of the loop-2 step: the token ranking over
+    all N rows, then for `n_layers` layers the block, residual quantisation and sparse
+    attention of `rows` active rows. Returns seconds extrapolated to one full sparse
+    loop (k_r rows x L layers), the measured seconds and the sample description."""
+    from cross_loop_sparse_step_b200 import configs, synth
+    from oracle import attention as oatt
+    from oracle import block as oblk
+    from oracle import kvstore as okv
+    from oracle import select as osel
+    N, d, H, hd, F, L = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn",
+                                          "n_layers"))
+    k_act = configs.active_counts(cfg)[2]
+    kcol = cfg["col_k"][2]
+    g = synth.rng(seed)
+    cur, prev, _ = synth.pareto_delta_pair(g, N, d, 2)
+    layers = synth.model_weights(g, n_layers, d, F, bf16=True)
+    bias = synth.col_bias(g, N, cfg["bias_frac"], cfg["bias_value"])
+    stores = []
+    for _ in range(n_layers):
+        st = okv.LayerKV(N, H, hd, cfg["group"], cfg["base_bits"], cfg["res_bits"], cfg["n_loops"])
+        st.write_base(synth.kv_values(g, N, H, hd), synth.kv_values(g, N, H, hd))
+        stores.append(st)
+    # carried statistics of the sampled queries: the sink, biased columns, then random
+    t0 = time.perf_counter()
+    act, _, _ = osel.select_active(cur, prev, None, k_act)
+    t_select = time.perf_counter() - t0
+    rs = synth.rng(seed + 1)
+    q_rows = np.sort(rs.choice(act, size=min(rows, len(act)), replace=False)).astype(np.int32)
+    X = synth.embeddings(g, len(q_rows), d).astype(np.float64)
+    S = np.full((H, N, kcol + 1), oatt.SENTINEL, np.uint16)
+    for t in q_rows:
+        for h in range(H):
+            n = min(kcol, int(t)) + 1
+            c = np.sort(np.concatenate([[0], rs.choice(np.arange(1, t + 1), n - 1, replace=False)])) \
+                if t > 0 else np.array([0])
+            S[h, t, :n] = c
+    m = np.full((H, N), 0.9)
+    u = np.zeros((H, N, hd))
+    t0 = time.perf_counter()
+    for li in range(n_layers):
+        q, k, v = oblk.qkv(X, q_rows, layers[li], H, hd)
+        stores[li].write_residual(2, q_rows, k.astype(np.float32), v.astype(np.float32))
+        Kh, Vh = stores[li].hat[2]
+        o = oatt.sparse_attention(q, q_rows, q_rows, Kh, Vh, S, m, u, bias)
+        X = oblk.out_ffn(X, o.reshape(len(q_rows), d), layers[li])
+    t_layers = time.perf_counter() - t0
+    per_loop = t_select + t_layers / n_layers * L * (k_act / len(q_rows))
+    desc = (f"loop-2 step sample: token ranking over all {N} rows, then {n_layers} layer(s) x "
+            f"{len(q_rows)} active rows (of {k_act}) x {H} heads; extrapolated x{L} layers, "
+            f"x{k_act}/{len(q_rows)} rows")
+    return per_loop, t_select + t_layers, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from cross_loop_sparse_step_b200 import configs
+    cfg = configs.CONFIGS[args.config]
+    R = cfg["n_loops"]
+    times = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        per_loop, _, desc = oracle_sample(cfg, n_layers=2, rows=512, seed=1 + i)
+        if i >= args.warmup:
+            times.append(per_loop)
+    per_loop = float(np.mean(times))
+    value = cfg["n_tok"] / per_loop
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": per_loop * (R - 1) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg["name"], "n_tok": cfg["n_tok"], "layers": cfg["n_layers"],
+                   "loops": R},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- main
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    import torch
+    import torch.distributed as dist
+    from cross_loop_sparse_step_b200 import configs, fl, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    cfg = configs.CONFIGS[args.config]
+    W = build_workload(cfg, fl, torch, synth, configs, seed=rank, n_layers=args.layers)
+    R, N = W["R"], W["N"]
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        restore(W)
+        step_loops(W)
+    torch.cuda.synchronize()
+    st = fl.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"warm-up reported {fl.status_str(st)}")
+
+    # per-kernel events for the roofline (GEMMs and attention inside the timed steps)
+    n_gemm = 4 * W["L"] * (R - 1) * args.steps
+    n_attn = W["L"] * (R - 1) * args.steps
+    ev = {}
+    lib = fl.lib_handle()
+    lib.fl_set_timing_events.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+    lib.fl_timing_recorded.restype = ctypes.c_int32
+    lib.fl_launch_count.restype = ctypes.c_int64
+    for kind, n in ((0, n_gemm), (1, n_attn)):
+        b = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for x in b + e:
+            x.record(stream)   # materialise the handles
+        arr_b = (ctypes.c_void_p * n)(*[x.cuda_event for x in b])
+        arr_e = (ctypes.c_void_p * n)(*[x.cuda_event for x in e])
+        ev[kind] = (b, e, arr_b, arr_e)
+        lib.fl_set_timing_events(kind, arr_b, arr_e, n)
+    torch.cuda.synchronize()
+
+    gpu = torch.cuda.get_device_properties(local)
+    uuid = getattr(gpu, "uuid", None)
+    clocks = ClockSampler(f"GPU-{uuid}" if uuid else None)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    launches0 = lib.fl_launch_count()
+    for i in range(args.steps):
+        restore(W)
+        starts[i].record(stream)
+        step_loops(W)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    launches = lib.fl_launch_count() - launches0
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    st = fl.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"timed steps reported {fl.status_str(st)}")
+    for kind in (0, 1):
+        lib.fl_set_timing_events(kind, None, None, 0)
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    t_rank = sum(step_ms) / 1e3
+    if world > 1:
+        t = torch.tensor([t_rank], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    else:
+        t_max = t_rank
+    tokens = N * (R - 1) * args.steps * world
+    value = tokens / t_max
+
+    # roofline of the dominant kernel (the projection GEMMs) and of the attention
+    pk, pk_kind = peaks()
+    b, e, _, _ = ev[0]
+    gemm_ms = [x.elapsed_time(y) for x, y in zip(b, e)]
+    gemm_s = sum(gemm_ms) / 1e3
+    gemm_tflops = gemm_flops_per_step(W) * args.steps / gemm_s / 1e12
+    peak_t = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    b, e, _, _ = ev[1]
+    attn_ms = [x.elapsed_time(y) for x, y in zip(b, e)]
+    abytes = attention_bytes_per_launch(W, torch)
+    per_loop_launch = W["L"] * args.steps
+    attn_bytes_total = sum(abytes[r][0] for r in abytes) * per_loop_launch
+    attn_s = sum(attn_ms) / 1e3
+    attn_gbs = attn_bytes_total / attn_s / 1e9
+    peak_h = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    step_total_ms = sum(step_ms)
+    kvb, dense = kv_bytes(W)
+
+    e2e = None
+    if not args.no_e2e:
+        h_host = W["snap"][0].cpu().pin_memory()
+        x_host = W["snap"][1].cpu().pin_memory()
+        out_host = torch.empty_like(h_host).pin_memory()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            W["run"].h.copy_(h_host, non_blocking=True)
+            W["run"].x_prev.copy_(x_host, non_blocking=True)
+            step_loops(W)
+            out_host.copy_(W["run"].h, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = e0.elapsed_time(e1) / 1e3
+        if world > 1:
+            t = torch.tensor([te], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            te = float(t.item())
+        e2e = {"value": tokens / te, "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h_host.numel() * 4 + x_host.numel() * 4),
+               "d2h_bytes_per_step": int(out_host.numel() * 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        per_loop, measured, desc = oracle_sample(cfg, n_layers=8, rows=512)
+        cpu = {"value": N / per_loop, "unit": "tokens/s", "cores": blas_threads(),
+               "kind": "oracle", "sample": desc, "measured_s": round(measured, 2)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg["name"], "n_tok": N, "d_model": W["d"],
+                       "heads": f"{W['H']}x{W['hd']}", "d_ffn": W["F"], "layers": W["L"],
+                       "loops": R, "timed_loops": list(range(2, R + 1)),
+                       "active_tokens": W["n_active"][2], "col_k": cfg["col_k"][2],
+                       "res_bits": cfg["res_bits"][2], "group": cfg["group"],
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (2.47 GB of bf16 weights per loop step)"},
+            "roofline": {"bound": "tensor", "kernel": "k_gemm_tc (projection GEMMs)",
+                         "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": gemm_tflops / peak_t, "traffic": None,
+                         "peak_source": f"{pk_kind} bf16 sustained",
+                         "share_of_step": gemm_s * 1e3 / step_total_ms},
+            "attention_roofline": {"bound": "hbm", "kernel": "k_attention (sparse, carried mass)",
+                                   "achieved": attn_gbs, "peak": peak_h, "unit": "GB/s",
+                                   "frac": attn_gbs / peak_h,
+                                   "bytes_per_launch": {str(r): abytes[r][0] for r in abytes},
+                                   "avg_launch_us": attn_s / len(attn_ms) * 1e6,
+                                   "share_of_step": attn_s * 1e3 / step_total_ms},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "kv_bytes_per_token_per_layer": kvb,
+            "kv_dense_bytes_per_token_per_layer": dense,
+            "kv_reduction": dense / kvb,
+            "step_ms": [round(x, 3) for x in step_ms],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -329,6 +329,7 @@ cudaError_t launch_t(const AttnParams& P, int max_cols, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   kern<<<P.n_q * P.H, NT, sm, s>>>(P, max_cols);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -79,6 +79,7 @@ cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* 
   if (M <= 0) return cudaSuccess;
   if (dt == FL_F32) k_rmsnorm<float><<<M, 256, 0, s>>>(x, gamma, eps, (float*)out, d);
   else k_rmsnorm<__nv_bfloat16><<<M, 256, 0, s>>>(x, gamma, eps, (__nv_bfloat16*)out, d);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -86,6 +87,7 @@ cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H
                               float theta, float* q, float* k, float* v, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   k_rope_split<<<grid_for((size_t)M * H * hd / 2), 256, 0, s>>>(qkv, pos, M, H, hd, theta, q, k, v);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -94,6 +96,7 @@ cudaError_t launch_swiglu(const float* gu, int M, int F, void* out, fl_dtype dt,
   if (M <= 0) return cudaSuccess;
   if (dt == FL_F32) k_swiglu<float><<<grid_for((size_t)M * F), 256, 0, s>>>(gu, M, F, (float*)out);
   else k_swiglu<__nv_bfloat16><<<grid_for((size_t)M * F), 256, 0, s>>>(gu, M, F, (__nv_bfloat16*)out);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -1,6 +1,8 @@
 // The C interface (include/fl.h): host-side validation, workspace carving and the
 // launch sequence of each entry point. Nothing here allocates device memory.
+#include <atomic>
 #include <mutex>
+#include <vector>
 #include <string.h>
 
 #include "fl_internal.cuh"
@@ -29,11 +31,42 @@ int* status_word() {
   return cache[dev];
 }
 
+// ---------------------------------------------------------------- launch accounting
+static std::atomic<long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+struct TimingHook {
+  std::vector<cudaEvent_t> begin, end;
+  int next = 0;
+};
+static TimingHook g_hooks[TIMED_KINDS];
+
+void timing_begin(int kind, cudaStream_t s) {
+  TimingHook& h = g_hooks[kind];
+  if (h.next < (int)h.begin.size()) cudaEventRecord(h.begin[h.next], s);
+}
+void timing_end(int kind, cudaStream_t s) {
+  TimingHook& h = g_hooks[kind];
+  if (h.next < (int)h.end.size()) cudaEventRecord(h.end[h.next++], s);
+}
+
 cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
                         int K, int ldc, GemmEpi epi, cudaStream_t s) {
+  timing_begin(TIMED_GEMM, s);
+  cudaError_t e;
   if (dt == FL_BF16 && gemm_tc_supported(M, N, K))
-    return launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s);
-  return launch_gemm_simt(dt, A, W, C, M, N, K, ldc, epi, s);
+    e = launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s);
+  else
+    e = launch_gemm_simt(dt, A, W, C, M, N, K, ldc, epi, s);
+  timing_end(TIMED_GEMM, s);
+  return e;
+}
+
+cudaError_t launch_attention_timed(const fl_attn_args& a, int* st, cudaStream_t s) {
+  timing_begin(TIMED_ATTN, s);
+  cudaError_t e = launch_attention(a, st, s);
+  timing_end(TIMED_ATTN, s);
+  return e;
 }
 
 }  // namespace fl
@@ -177,6 +210,25 @@ const char* fl_status_str(fl_status s) {
 
 const char* fl_version(void) { return "0.1.0"; }
 
+int64_t fl_launch_count(void) { return (int64_t)g_launches.load(); }
+
+fl_status fl_set_timing_events(int32_t kind, void* const* begin, void* const* end, int32_t n) {
+  FL_CHECK(kind >= 0 && kind < TIMED_KINDS && n >= 0, FL_ERR_INVALID_ARG);
+  FL_CHECK(n == 0 || (begin && end), FL_ERR_INVALID_ARG);
+  TimingHook& h = g_hooks[kind];
+  h.begin.clear(); h.end.clear(); h.next = 0;
+  for (int i = 0; i < n; ++i) {
+    h.begin.push_back(reinterpret_cast<cudaEvent_t>(begin[i]));
+    h.end.push_back(reinterpret_cast<cudaEvent_t>(end[i]));
+  }
+  return FL_OK;
+}
+
+int32_t fl_timing_recorded(int32_t kind) {
+  if (kind < 0 || kind >= TIMED_KINDS) return -1;
+  return g_hooks[kind].next;
+}
+
 fl_status fl_check_device_status(void* stream) {
   if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return FL_ERR_CUDA;
   int v = 0;
@@ -257,7 +309,7 @@ fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream) {
   fl_status st = check_attn(a);
   if (st != FL_OK) return st;
   if (a->n_q == 0) return FL_OK;
-  return cuda_st(launch_attention(*a, status_word(), S(stream)));
+  return cuda_st(launch_attention_timed(*a, status_word(), S(stream)));
 }
 
 size_t fl_block_workspace_bytes(const fl_model* m, int32_t n_rows) {
@@ -407,7 +459,7 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
       a.stat_kind = sc->stat_kind;
     }
     a.out = attn; a.out_dt = m->dt;
-    FL_TRY(launch_attention(a, sw, s));
+    FL_TRY(launch_attention_timed(a, sw, s));
     rc = run_out_ffn(m, l, X, M, attn, blk, s);
     if (rc != FL_OK) return rc;
   }

@@ -19,6 +19,14 @@ __device__ __forceinline__ void record_error(int* st, int code) {
   if (st) atomicCAS(st, 0, code);
 }
 
+// ---------------------------------------------------------------- launch accounting
+// Every kernel launch of the library bumps a process-wide counter (read through
+// fl_launch_count); GEMM and attention launches can be bracketed by caller events.
+void count_launch();
+enum TimedKind { TIMED_GEMM = 0, TIMED_ATTN = 1, TIMED_KINDS = 2 };
+void timing_begin(int kind, cudaStream_t s);
+void timing_end(int kind, cudaStream_t s);
+
 // ---------------------------------------------------------------- KV store view
 // By-value copy of fl_kv_desc for kernels (loops up to FL_MAX_LOOPS).
 struct KvView {

@@ -55,6 +55,7 @@ cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const
   else
     k_gather_scatter<uint16_t><<<n_idx, 256, 0, s>>>(op, (const uint8_t*)src, (uint8_t*)dst,
                                                      idx, n_full, row_bytes, st);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -62,6 +63,7 @@ cudaError_t launch_fill_i32(int32_t* p, int32_t v, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
   k_fill_i32<<<blocks, 256, 0, s>>>(p, v, n);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -69,6 +71,7 @@ cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   const int blocks = (n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096;
   k_iota<<<blocks, 256, 0, s>>>(p, n);
+  count_launch();
   return cudaGetLastError();
 }
 

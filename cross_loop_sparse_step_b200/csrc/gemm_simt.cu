@@ -78,6 +78,7 @@ cudaError_t launch_gemm_simt(fl_dtype dt, const void* A, const void* W, float* C
     k_gemm_simt<__nv_bfloat16><<<grid, 256, 0, s>>>((const __nv_bfloat16*)A,
                                                     (const __nv_bfloat16*)W, C, M, N, K, ldc,
                                                     (int)epi);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -1,10 +1,230 @@
-// Tensor-core GEMM (tcgen05 + TMEM + TMA) for the bf16 model path.
+// Tensor-core GEMM for the bf16 path (FlashLoop §4.4: the gathered active rows keep
+// the projections regular GEMMs): C (=|+=) A . W^T, A [M x K] bf16 activations,
+// W [N x K] bf16 linear-layer weights, fp32 accumulation in tensor memory.
+//
+// One 128 x BN output tile per CTA, 6 warps:
+//   warp 0     TMA producer: A and W tiles (64 K-columns, 128-byte swizzle) into a
+//              STAGES-deep shared-memory ring, completion counted on mbarriers;
+//   warp 1     allocates TMEM and issues tcgen05.mma (M 128, N BN, K 16) from one
+//              thread; tcgen05.commit frees each ring slot and finally signals the
+//              epilogue;
+//   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (= tile rows), binary32
+//              store or accumulate into C.
+// Rows beyond M are zero-filled by TMA and not stored. Every mbarrier wait is bounded
+// in time; a wait that runs out records FL_ERR_TIMEOUT and the CTA drains its copies
+// in flight, frees TMEM and returns.
+#include <mutex>
+#include <unordered_map>
+
 #include "fl_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace fl {
-bool gemm_tc_supported(int M, int N, int K) { (void)M; (void)N; (void)K; return false; }
-cudaError_t launch_gemm_tc(const void*, const void*, float*, int, int, int, int, GemmEpi,
-                           cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+using namespace sm100;
+
+constexpr int BM = 128, BK = 64;
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+              float* __restrict__ C, int M, int N, int K, int ldc, int epi, int* st) {
+  constexpr uint32_t A_BYTES = BM * BK * 2;
+  constexpr uint32_t B_BYTES = BN * BK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], acc_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  volatile int* abort = &abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int nk = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    mbar_init(&acc_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) { prefetch_tmap(&tma_a); prefetch_tmap(&tma_b); }
+  if (warp == 1) tmem_alloc(&tmem_slot, BN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES, i = kb / STAGES;
+        if (i > 0 && !mbar_wait(&empty_bar[s], (i - 1) & 1, abort)) break;
+        uint8_t* a_dst = smem + s * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+        tma_load_2d(a_dst, &tma_a, &full_bar[s], kb * BK, m0);
+        tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, n0);
+        issued = kb + 1;
+      }
+      if (*abort) {  // drain the copies still in flight before shared memory is released
+        const uint64_t t0 = globaltimer();
+        for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb) {
+          const int s = kb % STAGES;
+          while (!mbar_try_wait(&full_bar[s], (kb / STAGES) & 1))
+            if (globaltimer() - t0 > kWaitLimitNs) break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % STAGES, i = kb / STAGES;
+        if (!mbar_wait(&full_bar[s], i & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+        const uint32_t b_base = a_base + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          mma_bf16(tmem, desc_sw128_kmajor(a_base + kk * 32), desc_sw128_kmajor(b_base + kk * 32),
+                   idesc, (kb | kk) != 0 ? 1u : 0u);
+        }
+        mma_commit(&empty_bar[s]);
+      }
+      mma_commit(&acc_bar);
+    }
+  } else {
+    const int ew = warp & 3;  // TMEM lanes [32 ew, 32 ew + 32) belong to this warp
+    const int row = m0 + ew * 32 + lane;
+    // wait for the accumulator (time-bounded only: MMAs already issued must finish
+    // before TMEM is freed, even after an abort elsewhere)
+    bool ok = mbar_try_wait(&acc_bar, 0);
+    if (!ok) {
+      const uint64_t t0 = globaltimer();
+      while (!(ok = mbar_try_wait(&acc_bar, 0)))
+        if (globaltimer() - t0 > kWaitLimitNs) { *abort = 1; break; }
+    }
+    tc_fence_after();
+    if (ok && !*abort) {
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(c * 32), v);
+        if (row < M) {
+          float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c * 32);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 x = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            if (epi == EPI_ADD) {
+              const float4 y = dst[j];
+              x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+            }
+            dst[j] = x;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+  if (threadIdx.x == 0 && abort_flag) record_error(st, FL_ERR_TIMEOUT);
 }
+
+// ---------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct MapKey {
+  const void* p; int rows, cols, box_rows;
+  bool operator==(const MapKey& o) const {
+    return p == o.p && rows == o.rows && cols == o.cols && box_rows == o.box_rows;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    return std::hash<const void*>()(k.p) ^ ((size_t)k.rows << 20) ^ ((size_t)k.cols << 40) ^
+           (size_t)k.box_rows;
+  }
+};
+
+// Row-major bf16 [rows x cols] matrix, boxes of 64 columns x box_rows rows, 128B swizzle.
+bool get_map(const void* p, int rows, int cols, int box_rows, CUtensorMap* out) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  const MapKey key{p, rows, cols, box_rows};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) { *out = it->second; return true; }
+  }
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(p), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() > 4096) cache.clear();
+  cache[key] = m;
+  *out = m;
+  return true;
+}
+
+template <int BN, int STAGES>
+cudaError_t launch_bn(const void* A, const void* W, float* C, int M, int N, int K, int ldc,
+                      GemmEpi epi, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  if (!get_map(A, M, K, BM, &ma) || !get_map(W, N, K, BN, &mb)) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
+  auto kern = k_gemm_tc<BN, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(N / BN, (M + BM - 1) / BM);
+  kern<<<grid, 192, smem, s>>>(ma, mb, C, M, N, K, ldc, (int)epi, status_word());
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(int M, int N, int K) {
+  return M >= 1 && K >= BK && K % BK == 0 && N % 128 == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N, int K, int ldc,
+                           GemmEpi epi, cudaStream_t s) {
+  if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)C % 16 || ldc % 4)
+    return cudaErrorInvalidValue;
+  return launch_bn<128, 6>(A, W, C, M, N, K, ldc, epi, s);
+}
+
 }  // namespace fl

@@ -135,6 +135,7 @@ cudaError_t launch_epl(const KvView& v, const QuantOut& o, int loop, const void*
   else
     k_kv_quant<EPL, __nv_bfloat16><<<blocks, 256, 0, s>>>(
         v, o, loop, (const __nv_bfloat16*)k, (const __nv_bfloat16*)vv, act, n_act, st);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -175,6 +175,7 @@ cudaError_t launch_row_delta(const void* cur, const void* prev, fl_dtype dt, int
   else
     k_row_delta<__nv_bfloat16><<<blocks, threads, 0, s>>>(
         (const __nv_bfloat16*)cur, (const __nv_bfloat16*)prev, n_rows, d, delta);
+  count_launch();
   return cudaGetLastError();
 }
 
@@ -183,6 +184,7 @@ cudaError_t launch_topk_rows(const float* delta, int n, int k, const int32_t* ro
   (void)st;
   if (k <= 0) return cudaSuccess;
   k_topk_rows<<<1, TK_THREADS, 0, s>>>(delta, n, k, row_tok, out_tok, out_pos);
+  count_launch();
   return cudaGetLastError();
 }
 

@@ -58,6 +58,17 @@ const char* fl_status_str(fl_status s);
 /* Library version, "major.minor.patch". */
 const char* fl_version(void);
 
+/* Number of kernel launches the library has issued in this process. */
+int64_t fl_launch_count(void);
+
+/* Measurement hook. With n > 0 the library records the caller's events begin[i] and
+ * end[i] (each a cudaEvent_t passed as void*) on the launch stream around its next n
+ * launches of one kind (0: the projection GEMMs, 1: the attention kernel);
+ * fl_timing_recorded(kind) says how many pairs were recorded. n = 0 turns it off.
+ * Not thread-safe: set it from the thread that issues the work. */
+fl_status fl_set_timing_events(int32_t kind, void* const* begin, void* const* end, int32_t n);
+int32_t fl_timing_recorded(int32_t kind);
+
 /* Synchronises `stream`, returns the first error a kernel recorded on the current
  * device since the last call (FL_OK if none) and clears it. */
 fl_status fl_check_device_status(void* stream);

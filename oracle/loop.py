@@ -28,12 +28,13 @@ from . import attention, block, kvstore, select
 
 
 def run(layers, h0, sched, n_heads, head_dim, bias=None, eps=1e-6, theta=10000.0,
-        select_prev=None):
+        select_prev=None, bf16_ops=False):
     """Run loops 1..R. ``layers`` is a list of weight dicts (see ``block``).
 
     ``select_prev`` optionally maps a loop r to the array used in place of
     h_{r-2}[A_{r-1}] when that loop ranks tokens (a synthetic previous state), or to
-    a function of the current rows h_{r-1}[A_{r-1}] returning it.
+    a function of the current rows h_{r-1}[A_{r-1}] returning it. ``bf16_ops``: the
+    GEMM operands are bfloat16 tensors (bf16 workloads).
     Returns a dict with per-loop hidden states, active sets, deltas, the per-layer
     KV stores and the statistics after every loop."""
     h0 = np.asarray(h0, np.float64)
@@ -72,7 +73,7 @@ def run(layers, h0, sched, n_heads, head_dim, bias=None, eps=1e-6, theta=10000.0
         kn = next_k(r)
         new_stats = [None] * L
         for li, layer in enumerate(layers):
-            q, k, v = block.qkv(X, act, layer, n_heads, head_dim, eps, theta)
+            q, k, v = block.qkv(X, act, layer, n_heads, head_dim, eps, theta, bf16_ops)
             if r == 1:
                 stores[li].write_base(k.astype(np.float32), v.astype(np.float32))
             else:
@@ -98,7 +99,7 @@ def run(layers, h0, sched, n_heads, head_dim, bias=None, eps=1e-6, theta=10000.0
                 new_stats[li] = (S_full, m_full, u_full)
             else:
                 o = res
-            X = block.out_ffn(X, o.reshape(len(act), d), layer, eps)
+            X = block.out_ffn(X, o.reshape(len(act), d), layer, eps, bf16_ops)
         stats = new_stats
         out["stats"][r] = stats
         h = h_prev.copy()

@@ -337,6 +337,10 @@ BLOCK_CASES = [
     (77, 256, 2, 128, 512, "f32"),
     (820, 2048, 16, 128, 5632, "bf16"),
     (131, 2048, 16, 128, 5632, "bf16"),
+    (1, 256, 2, 128, 512, "bf16"),       # a single row: one ragged 128-row tile
+    (128, 256, 2, 128, 512, "bf16"),     # exactly one tile
+    (129, 256, 2, 128, 512, "bf16"),     # one row into the next tile
+    (4096, 2048, 16, 128, 5632, "bf16"), # every token (loop 1)
 ]
 
 

@@ -147,7 +147,8 @@ def test_4k_shape_two_layers_two_loops():
                    col_k={2: cfg["col_k"][2]}, base_bits=8, res_bits=res, group=cfg["group"])
     # the oracle's own loop 1, then its loop 2 ranking with the same synthetic change
     want = oloop.run(layers, h0, sched_o, H, hd, bias,
-                     select_prev={2: lambda rows: rows - delta.astype(np.float64)})
+                     select_prev={2: lambda rows: rows - delta.astype(np.float64)},
+                     bf16_ops=True)
     assert_close(h1_gpu, want["h"][1], what="h_1")
     assert np.array_equal(host(run.act[2]), want["act"][2])
     h2 = host(run.h)

@@ -102,3 +102,29 @@ def test_rmsnorm_constant_row():
 def test_silu_closed_form():
     assert block.silu(np.array(0.0)) == 0.0
     assert abs(block.silu(np.array(1.0)) - 1 / (1 + np.exp(-1))) < 1e-16
+
+
+def test_bf16_operand_rounding():
+    """bf16 operand rounding: representable values unchanged, ties to even, and the
+    same as torch's float32 -> bfloat16 conversion (a library routine)."""
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -3.5, 0.0])
+    y = block.bf16(x)
+    assert y[0] == 1.0 and y[4] == -3.5 and y[5] == 0.0
+    assert y[1] == 1.0            # exact tie 1 + 2^-8 rounds to even (1.0)
+    assert y[2] == 1.0 + 2 ** -6  # tie 1 + 3*2^-8 rounds to even (1 + 2^-6)
+    assert y[3] == 1.0            # below half an ulp
+    g = np.random.Generator(np.random.PCG64(24))
+    z = g.normal(size=1000) * 10
+    want = torch.tensor(z, dtype=torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(block.bf16(z.astype(np.float32).astype(np.float64)), want)
+
+
+def test_bf16_operands_change_only_by_rounding():
+    g = synth.rng(25)
+    n, d, H, hd, Fd = 12, 64, 4, 16, 96
+    layer = synth.layer_weights(g, d, Fd, std=0.2, bf16=True)
+    X = synth.embeddings(g, n, d).astype(np.float64)
+    a = block.qkv(X, np.arange(n), layer, H, hd)
+    b = block.qkv(X, np.arange(n), layer, H, hd, bf16_ops=True)
+    for u, v in zip(a, b):
+        assert 0 < np.max(np.abs(u - v)) < 2e-2

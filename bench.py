@@ -116,6 +116,20 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
+# ---------------------------------------------------------------- multi-rank aggregation
+def aggregate(t_rank, units_rank, dist=None, device="cpu"):
+    """Whole-job throughput over replicas: every rank's units divided by the slowest
+    rank's time (max over ranks). Returns (value, t_max, units_total)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return units_rank / t_rank, t_rank, units_rank
+    t = torch.tensor([t_rank], dtype=torch.float64, device=device)
+    u = torch.tensor([units_rank], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(u.item()) / float(t.item()), float(t.item()), float(u.item())
+
+
 # ---------------------------------------------------------------- workload
 def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
     N, d, H, hd, F = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn"))
@@ -376,14 +390,8 @@ def main():
         lib.fl_set_timing_events(kind, None, None, 0)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     t_rank = sum(step_ms) / 1e3
-    if world > 1:
-        t = torch.tensor([t_rank], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
-    else:
-        t_max = t_rank
-    tokens = N * (R - 1) * args.steps * world
-    value = tokens / t_max
+    value, t_max, tokens = aggregate(t_rank, N * (R - 1) * args.steps,
+                                     dist if world > 1 else None, device="cuda")
 
     # roofline of the dominant kernel (the projection GEMMs) and of the attention
     pk, pk_kind = peaks()
@@ -420,11 +428,9 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         te = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            t = torch.tensor([te], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            te = float(t.item())
-        e2e = {"value": tokens / te, "unit": "tokens/s",
+        v_e2e, _, _ = aggregate(te, N * (R - 1) * args.steps, dist if world > 1 else None,
+                                device="cuda")
+        e2e = {"value": v_e2e, "unit": "tokens/s",
                "h2d_bytes_per_step": int(h_host.numel() * 4 + x_host.numel() * 4),
                "d2h_bytes_per_step": int(out_host.numel() * 4)}
 

@@ -17,24 +17,6 @@
 namespace fl {
 namespace {
 
-struct AttnParams {
-  const void* q; int q_bf16;
-  const int32_t* q_tok;
-  int n_q, H, hd;
-  float scale;
-  KvView kv;
-  int loop;
-  const float* bias;
-  const uint16_t* sel; const float* mass; const float* unsel;
-  int stat_rows, sel_stride;
-  const int32_t* q_row;
-  int k_next;
-  uint16_t* sel_out; float* mass_out; float* unsel_out;
-  int out_stride, stat_kind;
-  const float* vnorm;
-  void* out; int out_bf16;
-  int* st;
-};
 
 template <int NT>
 __device__ __forceinline__ float block_reduce(float v, bool is_max, float* red) {
@@ -326,8 +308,15 @@ cudaError_t launch_t(const AttnParams& P, int max_cols, cudaStream_t s) {
   const size_t sm = smem_bytes(NT, P.hd, max_cols, P.sel != nullptr);
   if (sm > 227 * 1024) return cudaErrorInvalidValue;
   auto kern = k_attention<NT, EPL>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
+  static int attr_bytes[128] = {0};   // per device: the largest size allowed so far
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if ((int)sm > attr_bytes[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    attr_bytes[dev] = (int)sm;
+  }
   kern<<<P.n_q * P.H, NT, sm, s>>>(P, max_cols);
   count_launch();
   return cudaGetLastError();
@@ -353,6 +342,7 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   P.out_stride = a.out_stride; P.stat_kind = a.stat_kind; P.vnorm = a.kv->vnorm;
   P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
   const bool sparse = a.sel != nullptr;
+  if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);
   const int max_cols = sparse ? a.sel_stride : a.kv->n_tok;
   if (sparse) {
     if (P.hd == 128) return launch_t<128, 16>(P, max_cols, s);

@@ -16,6 +16,9 @@ cudaError_t launch_gemm_simt(fl_dtype dt, const void* A, const void* W, float* C
 cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N, int K,
                            int ldc, GemmEpi epi, cudaStream_t s);
 bool gemm_tc_supported(int M, int N, int K);
+bool gemm_swiglu_supported(int M, int F, int K);
+cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int F, int K,
+                               cudaStream_t s);
 
 int* status_word() {
   static int* cache[128] = {nullptr};
@@ -161,8 +164,15 @@ fl_status run_out_ffn(const fl_model* m, int layer, float* x, int n, const void*
   void* mid = c.take((size_t)n * F * dt_size(m->dt));
   FL_TRY(launch_gemm(m->dt, attn, w.w_o, x, n, d, d, d, EPI_ADD, s));
   FL_TRY(launch_rmsnorm(x, w.g_ffn, m->rms_eps, a, m->dt, n, d, s));
-  FL_TRY(launch_gemm(m->dt, a, w.w_gate_up, gu, n, 2 * F, d, 2 * F, EPI_STORE, s));
-  FL_TRY(launch_swiglu(gu, n, F, mid, m->dt, s));
+  if (m->dt == FL_BF16 && gemm_swiglu_supported(n, F, d)) {
+    timing_begin(TIMED_GEMM, s);
+    cudaError_t e = launch_gemm_swiglu(a, w.w_gate_up, mid, n, F, d, s);
+    timing_end(TIMED_GEMM, s);
+    FL_TRY(e);
+  } else {
+    FL_TRY(launch_gemm(m->dt, a, w.w_gate_up, gu, n, 2 * F, d, 2 * F, EPI_STORE, s));
+    FL_TRY(launch_swiglu(gu, n, F, mid, m->dt, s));
+  }
   FL_TRY(launch_gemm(m->dt, mid, w.w_down, x, n, d, F, d, EPI_ADD, s));
   return FL_OK;
 }

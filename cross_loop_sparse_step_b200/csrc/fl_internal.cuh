@@ -105,6 +105,29 @@ __device__ __forceinline__ void reconstruct(const KvView& kv, int which, int upt
   }
 }
 
+// Arguments of the attention kernels (a by-value copy of fl_attn_args plus the store view).
+struct AttnParams {
+  const void* q; int q_bf16;
+  const int32_t* q_tok;
+  int n_q, H, hd;
+  float scale;
+  KvView kv;
+  int loop;
+  const float* bias;
+  const uint16_t* sel; const float* mass; const float* unsel;
+  int stat_rows, sel_stride;
+  const int32_t* q_row;
+  int k_next;
+  uint16_t* sel_out; float* mass_out; float* unsel_out;
+  int out_stride, stat_kind;
+  const float* vnorm;
+  void* out; int out_bf16;
+  int* st;
+};
+
+bool sparse_fast_eligible(const AttnParams& P);
+cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s);
+
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {

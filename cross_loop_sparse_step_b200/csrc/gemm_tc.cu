@@ -26,10 +26,17 @@ using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
 
-template <int BN, int STAGES>
+// EPI_STORE / EPI_ADD: C[M x N] fp32 (=|+=) A . W^T, tile columns n0 = 128 * blockIdx.x.
+// EPI_SWIGLU: W = [gate; up] with `half` rows each; a tile holds 64 gate rows and the
+// matching 64 up rows (two TMA boxes), and the epilogue writes silu(g) * u as bf16 into
+// Y [M x half] at columns 64 * blockIdx.x.
+constexpr int EPI_SWIGLU = 2;
+
+template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-              float* __restrict__ C, int M, int N, int K, int ldc, int epi, int* st) {
+              float* __restrict__ C, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int ldc,
+              int half, int* st) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -67,7 +74,13 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* a_dst = smem + s * STAGE_BYTES;
         mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
         tma_load_2d(a_dst, &tma_a, &full_bar[s], kb * BK, m0);
-        tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, n0);
+        if constexpr (EPI == EPI_SWIGLU) {
+          const int f0 = blockIdx.x * (BN / 2);
+          tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, f0);
+          tma_load_2d(a_dst + A_BYTES + B_BYTES / 2, &tma_b, &full_bar[s], kb * BK, half + f0);
+        } else {
+          tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, n0);
+        }
         issued = kb + 1;
       }
       if (*abort) {  // drain the copies still in flight before shared memory is released
@@ -109,7 +122,31 @@ __global__ void __launch_bounds__(192, 1)
         if (globaltimer() - t0 > kWaitLimitNs) { *abort = 1; break; }
     }
     tc_fence_after();
-    if (ok && !*abort) {
+    if (EPI == EPI_SWIGLU && ok && !*abort) {
+      const int f0 = blockIdx.x * (BN / 2);
+#pragma unroll 1
+      for (int c = 0; c < BN / 64; ++c) {
+        float g[32], u[32];
+        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(c * 32), g);
+        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(BN / 2 + c * 32), u);
+        if (row < M) {
+          uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * half + f0 + c * 32);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int e = 8 * j + 2 * q;
+              const float y0 = g[e] / (1.0f + expf(-g[e])) * u[e];
+              const float y1 = g[e + 1] / (1.0f + expf(-g[e + 1])) * u[e + 1];
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+              w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    } else if (EPI != EPI_SWIGLU && ok && !*abort) {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         float v[32];
@@ -119,7 +156,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             float4 x = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            if (epi == EPI_ADD) {
+            if (EPI == EPI_ADD) {
               const float4 y = dst[j];
               x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
             }
@@ -199,17 +236,26 @@ bool get_map(const void* p, int rows, int cols, int box_rows, CUtensorMap* out) 
   return true;
 }
 
-template <int BN, int STAGES>
-cudaError_t launch_bn(const void* A, const void* W, float* C, int M, int N, int K, int ldc,
-                      GemmEpi epi, cudaStream_t s) {
+template <int BN, int STAGES, int EPI>
+cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, int M, int N,
+                      int K, int ldc, cudaStream_t s) {
   CUtensorMap ma, mb;
-  if (!get_map(A, M, K, BM, &ma) || !get_map(W, N, K, BN, &mb)) return cudaErrorInvalidValue;
+  const int box_b = EPI == EPI_SWIGLU ? BN / 2 : BN;
+  if (!get_map(A, M, K, BM, &ma) || !get_map(W, N, K, box_b, &mb)) return cudaErrorInvalidValue;
   const size_t smem = (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
-  auto kern = k_gemm_tc<BN, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(N / BN, (M + BM - 1) / BM);
-  kern<<<grid, 192, smem, s>>>(ma, mb, C, M, N, K, ldc, (int)epi, status_word());
+  auto kern = k_gemm_tc<BN, STAGES, EPI>;
+  static bool attr_set[128] = {false};   // per device; set on the first (uncaptured) call
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int tiles_n = EPI == EPI_SWIGLU ? (N / 2) / (BN / 2) : N / BN;
+  dim3 grid(tiles_n, (M + BM - 1) / BM);
+  kern<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, status_word());
   count_launch();
   return cudaGetLastError();
 }
@@ -224,7 +270,21 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N,
                            GemmEpi epi, cudaStream_t s) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)C % 16 || ldc % 4)
     return cudaErrorInvalidValue;
-  return launch_bn<128, 6>(A, W, C, M, N, K, ldc, epi, s);
+  if (epi == EPI_ADD) return launch_bn<128, 6, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s);
+  return launch_bn<128, 6, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s);
+}
+
+bool gemm_swiglu_supported(int M, int F, int K) {
+  return gemm_tc_supported(M, 2 * F, K) && F % 64 == 0;
+}
+
+// Y[M x F] bf16 = silu(A . W_gate^T) * (A . W_up^T), W = [gate; up] of [2F x K].
+cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int F, int K,
+                               cudaStream_t s) {
+  if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)Y % 16 || F % 64)
+    return cudaErrorInvalidValue;
+  return launch_bn<128, 6, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
+                                       2 * F, K, 0, s);
 }
 
 }  // namespace fl

@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="launch each step's kernels eagerly instead of replaying a CUDA graph")
     return ap.parse_args()
 
 
@@ -343,51 +345,92 @@ def main():
     if st != 0:
         raise RuntimeError(f"warm-up reported {fl.status_str(st)}")
 
-    # per-kernel events for the roofline (GEMMs and attention inside the timed steps)
-    n_gemm = 4 * W["L"] * (R - 1) * args.steps
-    n_attn = W["L"] * (R - 1) * args.steps
-    ev = {}
+    # per-kernel events for the roofline: the library records them around every GEMM
+    # (kind 0) and attention (kind 1) launch of a step
     lib = fl.lib_handle()
-    lib.fl_set_timing_events.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+    lib.fl_set_timing_events.argtypes = [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_int32]
     lib.fl_timing_recorded.restype = ctypes.c_int32
     lib.fl_launch_count.restype = ctypes.c_int64
-    for kind, n in ((0, n_gemm), (1, n_attn)):
+    per_step = {0: 4 * W["L"] * (R - 1), 1: W["L"] * (R - 1)}
+    reps = 1 if args.graph else args.steps
+    ev = {}
+    for kind in (0, 1):
+        n = per_step[kind] * reps
         b = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         e = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
         for x in b + e:
             x.record(stream)   # materialise the handles
-        arr_b = (ctypes.c_void_p * n)(*[x.cuda_event for x in b])
-        arr_e = (ctypes.c_void_p * n)(*[x.cuda_event for x in e])
-        ev[kind] = (b, e, arr_b, arr_e)
-        lib.fl_set_timing_events(kind, arr_b, arr_e, n)
+        ev[kind] = (b, e, (ctypes.c_void_p * n)(*[x.cuda_event for x in b]),
+                    (ctypes.c_void_p * n)(*[x.cuda_event for x in e]))
     torch.cuda.synchronize()
+
+    def arm_hooks():
+        for kind in (0, 1):
+            lib.fl_set_timing_events(kind, ev[kind][2], ev[kind][3], len(ev[kind][0]))
+
+    def disarm_hooks():
+        for kind in (0, 1):
+            lib.fl_set_timing_events(kind, None, None, 0)
+
+    graph = None
+    kernels_per_step = None
+    if args.graph:
+        restore(W)
+        torch.cuda.synchronize()
+        arm_hooks()
+        c0 = lib.fl_launch_count()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step_loops(W)
+        kernels_per_step = lib.fl_launch_count() - c0
+        disarm_hooks()
+        for _ in range(2):
+            restore(W)
+            graph.replay()
+        torch.cuda.synchronize()
+        st = fl.check_device_status()
+        if st != 0:
+            raise RuntimeError(f"graph warm-up reported {fl.status_str(st)}")
 
     gpu = torch.cuda.get_device_properties(local)
     uuid = getattr(gpu, "uuid", None)
     clocks = ClockSampler(f"GPU-{uuid}" if uuid else None)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    kern_ms = {0: [], 1: []}
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
     launches0 = lib.fl_launch_count()
+    if not args.graph:
+        arm_hooks()
     for i in range(args.steps):
         restore(W)
         starts[i].record(stream)
-        step_loops(W)
+        if graph is not None:
+            graph.replay()
+        else:
+            step_loops(W)
         ends[i].record(stream)
+        if graph is not None:   # the graph re-records one step's kernel events per replay
+            ends[i].synchronize()
+            for kind in (0, 1):
+                kern_ms[kind] += [x.elapsed_time(y) for x, y in zip(ev[kind][0], ev[kind][1])]
     torch.cuda.synchronize()
-    launches = lib.fl_launch_count() - launches0
+    if not args.graph:
+        disarm_hooks()
+        for kind in (0, 1):
+            kern_ms[kind] = [x.elapsed_time(y) for x, y in zip(ev[kind][0], ev[kind][1])]
+    launches = (lib.fl_launch_count() - launches0) if graph is None else kernels_per_step * args.steps
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
     st = fl.check_device_status()
     if st != 0:
         raise RuntimeError(f"timed steps reported {fl.status_str(st)}")
-    for kind in (0, 1):
-        lib.fl_set_timing_events(kind, None, None, 0)
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     t_rank = sum(step_ms) / 1e3
     value, t_max, tokens = aggregate(t_rank, N * (R - 1) * args.steps,
@@ -395,13 +438,10 @@ def main():
 
     # roofline of the dominant kernel (the projection GEMMs) and of the attention
     pk, pk_kind = peaks()
-    b, e, _, _ = ev[0]
-    gemm_ms = [x.elapsed_time(y) for x, y in zip(b, e)]
-    gemm_s = sum(gemm_ms) / 1e3
+    gemm_s = sum(kern_ms[0]) / 1e3
     gemm_tflops = gemm_flops_per_step(W) * args.steps / gemm_s / 1e12
     peak_t = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    b, e, _, _ = ev[1]
-    attn_ms = [x.elapsed_time(y) for x, y in zip(b, e)]
+    attn_ms = kern_ms[1]
     abytes = attention_bytes_per_launch(W, torch)
     per_loop_launch = W["L"] * args.steps
     attn_bytes_total = sum(abytes[r][0] for r in abytes) * per_loop_launch
@@ -423,7 +463,10 @@ def main():
         for _ in range(args.steps):
             W["run"].h.copy_(h_host, non_blocking=True)
             W["run"].x_prev.copy_(x_host, non_blocking=True)
-            step_loops(W)
+            if graph is not None:
+                graph.replay()
+            else:
+                step_loops(W)
             out_host.copy_(W["run"].h, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -467,6 +510,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": int(launches),
+            "launch_mode": "cuda-graph replay" if graph is not None else "eager",
             "clocks": clk,
             "kv_bytes_per_token_per_layer": kvb,
             "kv_dense_bytes_per_token_per_layer": dense,

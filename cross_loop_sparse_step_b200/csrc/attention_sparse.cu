@@ -4,16 +4,16 @@
 // K/V of the selected columns are gathered, here straight from the quantised store).
 //
 // Used when the store is quantised throughout (int8 base, 2/4/8-bit residuals).
-//   K pass, one lane per column: the lane streams the column's 128-byte base code row,
-//     its (scale, offset) pairs and the residual rows of every loop that rewrote it,
-//     with independent 16-byte loads, and forms q . K^ group by group as
-//     s * (q . codes) + z * sum(q) - the dequantisation folded into the dot product.
+//   Four lanes per column, eight columns in flight per warp; each lane owns a quarter
+//   of the head slice (one quantisation group at head_dim 128) and keeps its part of q
+//   in registers.
+//   K pass: every stored row of the column's chain (base, then each loop that rewrote
+//     it) contributes s * (q . codes) + z * sum(q) - dequantisation folded into the dot.
 //   softmax over the column set, p~ = m * softmax (m = cached mass).
 //   optional budget shrink: warp radix select over the binary32 bits of p~ * ||V^||
 //     (ties to the smaller column), ballot-ordered so the kept set stays ascending.
-//   V pass, lanes split head_dim: each column's rows are read coalesced, V^ is rebuilt
-//     in the store's order (base, then each residual added in binary32) and
-//     accumulated into o and, for dropped columns, into the next loop's u'.
+//   V pass: o += (p~ s) codes + p~ z over the chain's rows, and for dropped columns the
+//     same into the next loop's u'; the eight column groups are reduced by shuffles.
 #include <float.h>
 
 #include "fl_internal.cuh"
@@ -43,62 +43,65 @@ __device__ __forceinline__ float nib_f(uint32_t w, int i, int bits) {
   return __uint_as_float(0x4B000000u | c) - 8388608.0f;
 }
 
-// sum_e q[e] * deq[e] over one stored row of HD elements: per group g of `gs` elements,
-// s_g * (q_g . codes_g) + z_g * qsum_g. `bits` in {2, 4, 8}.
-template <int HD>
-__device__ __forceinline__ float row_dot(const uint8_t* codes, const uint32_t* sz, int bits,
-                                         int gs, const float* q, const float* qsum) {
-  float acc = 0.f;
-  const int ngroups = HD / gs;
-  const int wpg = gs * bits / 32;  // 32-bit code words per group
-  for (int gi = 0; gi < ngroups; ++gi) {
-    const uint32_t pair = sz[gi];
-    const float s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
-    const float z = half_bits_to_float((uint16_t)(pair >> 16));
-    const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes) + gi * wpg;
-    const float* qg = q + gi * gs;
-    float d = 0.f;
-    if (bits == 8) {
-      for (int k4 = 0; k4 < wpg; k4 += 4) {
-        const uint4 u = *reinterpret_cast<const uint4*>(cw + k4);
-        const uint32_t ww[4] = {u.x, u.y, u.z, u.w};
+// Codes [e0, e0 + EL) of one stored row (b bits, little-endian) as floats.
+template <int EL>
+__device__ __forceinline__ void load_codes(const uint8_t* row, int bits, int e0, float* c) {
+  if (bits == 8) {
+    const uint4* p = reinterpret_cast<const uint4*>(row + e0);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float4 qq = *reinterpret_cast<const float4*>(qg + (k4 + j) * 4);
-          d = fmaf(qq.x, byte_f(ww[j], 0), d);
-          d = fmaf(qq.y, byte_f(ww[j], 1), d);
-          d = fmaf(qq.z, byte_f(ww[j], 2), d);
-          d = fmaf(qq.w, byte_f(ww[j], 3), d);
-        }
-      }
-    } else {
-      const int per = 32 / bits;  // codes per word
-      for (int k = 0; k < wpg; ++k) {
-        const uint32_t wv = cw[k];
-        const float* qw = qg + k * per;
-        for (int j = 0; j < per; ++j) d = fmaf(qw[j], nib_f(wv, j, bits), d);
-      }
+    for (int k = 0; k < EL / 16; ++k) {
+      const uint4 u = p[k];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[16 * k + 4 * j + i] = byte_f(w[j], i);
     }
-    acc = fmaf(s, d, acc);
-    acc = fmaf(z, qsum[gi], acc);
+  } else if (bits == 4) {
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + e0 / 2);
+#pragma unroll
+    for (int k = 0; k < EL / 8; ++k) {
+      const uint32_t w = p[k];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[8 * k + i] = nib_f(w, i, 4);
+    }
+  } else {  // 2 bits
+    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + e0 / 4);
+#pragma unroll
+    for (int k = 0; k < EL / 16; ++k) {
+      const uint32_t w = p[k];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) c[16 * k + i] = nib_f(w, i, 2);
+    }
   }
-  return acc;
 }
 
-template <int HD>
+__device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s, float* z) {
+  const uint32_t pair = reinterpret_cast<const uint32_t*>(sz)[idx];
+  *s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
+  *z = half_bits_to_float((uint16_t)(pair >> 16));
+}
+
+// Four lanes per column: lane part l4 = lane % 4 owns elements [l4 * EL, (l4 + 1) * EL) of
+// the head slice, EL = HD / 4 (32 at HD 128), which lie in one quantisation group.
+// SHRINK: the call may shrink the budget (k_next below the carried set size), so the
+// dropped columns' contribution is accumulated too.
+template <int HD, bool SHRINK>
 __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__ AttnParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
-  constexpr int EPL = HD / 32;
+  constexpr int EL = HD / 4;
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * NW + w;
   if (gw >= P.n_q * P.H) return;  // whole warp leaves; no CTA-wide barrier below
   const int qi = gw / P.H, h = gw % P.H;
   const int H = P.H, n_tok = P.kv.n_tok, gs = P.kv.g, stride = P.sel_stride;
   const KvView& kv = P.kv;
+  const int l4 = lane & 3, cg = lane >> 2;   // part of the column, column group (0..7)
+  const int e0 = l4 * EL;
+  const int gidx = e0 / gs;                  // quantisation group of this lane's part
+  const int ngrp = HD / gs;
 
   uint8_t* base = smem + (size_t)w * warp_smem(HD, stride);
-  float* qs = reinterpret_cast<float*>(base);
-  float* qsum = qs + HD;
   float* p = reinterpret_cast<float*>(base + align16((size_t)HD * 4 + 16));
   uint16_t* cols = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p) + align16((size_t)stride * 4));
   uint8_t* mark = reinterpret_cast<uint8_t*>(cols) + align16((size_t)stride * 2);
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
   }
   const bool want_stats = P.sel_out != nullptr;
 
-  // ---- carried column set, cached mass, query slice
+  // ---- carried column set, cached mass, this lane's part of the query
   const uint16_t* srow_p = P.sel + ((size_t)h * P.stat_rows + srow) * stride;
   int n_cols = 0;
   for (int i0 = 0; i0 < stride; i0 += 32) {
@@ -122,53 +125,70 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     n_cols += __popc(__ballot_sync(0xffffffffu, c != FL_SENTINEL));
   }
   const float m_in = P.mass[(size_t)h * P.stat_rows + srow];
-  const int e0 = lane * EPL;
+  float qv[EL];
+  float qsum = 0.f;
   {
     const size_t off = ((size_t)qi * H + h) * HD + e0;
-    float part = 0.f;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const float v = P.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(P.q)[off + j])
-                               : reinterpret_cast<const float*>(P.q)[off + j];
-      qs[e0 + j] = v;
-      part += v;
+    for (int j = 0; j < EL; ++j) {
+      qv[j] = P.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(P.q)[off + j])
+                       : reinterpret_cast<const float*>(P.q)[off + j];
+      qsum += qv[j];
     }
-    const int lpg = gs / EPL;  // lanes per quantisation group
-    for (int o = 1; o < lpg; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane % lpg == 0) qsum[e0 / gs] = part;
   }
   __syncwarp();
 
-  // ---- K pass: one lane per column
+  // ---- K pass: 8 columns in flight, q . K^ = sum over parts of s (q . codes) + z sum(q)
   float lmax = -FLT_MAX;
-  const size_t krow = (size_t)HD;                 // base code bytes per (token, head)
-  for (int idx = lane; idx < n_cols; idx += 32) {
-    const int c = cols[idx];
-    float sc;
-    if (c > t || c >= n_tok) {
-      record_error(P.st, FL_ERR_RANGE);
-      sc = -INFINITY;
-    } else {
+  for (int i0 = 0; i0 < n_cols; i0 += 8) {
+    const int idx = i0 + cg;
+    float part = 0.f;
+    int c = -1;
+    bool valid = idx < n_cols;
+    if (valid) {
+      c = cols[idx];
+      valid = c <= t && c < n_tok;
+    }
+    if (valid) {
       const size_t bh = (size_t)c * H + h;
-      float acc = row_dot<HD>(kv.codes[0][1] + bh * krow,
-                              reinterpret_cast<const uint32_t*>(kv.sz[0][1]) + bh * (HD / gs), 8, gs,
-                              qs, qsum);
+      float cf[EL], sb, zb;
+      load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb, &zb);
+      load_codes<EL>(kv.codes[0][1] + bh * HD, 8, e0, cf);
+      float d = 0.f;
+#pragma unroll
+      for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
+      part = fmaf(sb, d, zb * qsum);
       for (int r = 2; r <= P.loop; ++r) {
         const int row = kv.slot[(size_t)r * n_tok + c];
         if (row < 0) continue;
         const int b = kv.res_bits[r];
         const size_t rh = (size_t)row * H + h;
-        acc += row_dot<HD>(kv.codes[0][r] + rh * (HD * b / 8),
-                           reinterpret_cast<const uint32_t*>(kv.sz[0][r]) + rh * (HD / gs), b, gs,
-                           qs, qsum);
+        float sr, zr;
+        load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr, &zr);
+        load_codes<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
+        float dr = 0.f;
+#pragma unroll
+        for (int j = 0; j < EL; ++j) dr = fmaf(qv[j], cf[j], dr);
+        part += fmaf(sr, dr, zr * qsum);
       }
-      sc = acc * P.scale + (P.bias ? P.bias[c] : 0.f);
     }
-    p[idx] = sc;
-    lmax = fmaxf(lmax, sc);
+    part += __shfl_xor_sync(0xffffffffu, part, 1);
+    part += __shfl_xor_sync(0xffffffffu, part, 2);
+    if (idx < n_cols && l4 == 0) {
+      float sc;
+      if (!valid) {
+        record_error(P.st, FL_ERR_RANGE);
+        sc = -INFINITY;
+      } else {
+        sc = part * P.scale + (P.bias ? P.bias[c] : 0.f);
+      }
+      p[idx] = sc;
+      lmax = fmaxf(lmax, sc);
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  __syncwarp();
   float lsum = 0.f;
   for (int idx = lane; idx < n_cols; idx += 32) {
     const float e = expf(p[idx] - lmax);
@@ -182,7 +202,7 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
   __syncwarp();
 
   // ---- budget shrink: keep the sink and the top-k_next columns by p~ * ||V^||
-  const bool prune = want_stats && (n_cols - 1 > P.k_next);
+  const bool prune = SHRINK && want_stats && (n_cols - 1 > P.k_next);
   if (prune) {
     uint32_t prefix = 0, pmask = 0, need = (uint32_t)P.k_next;
     for (int shift = 24; shift >= 0; shift -= 8) {
@@ -233,67 +253,78 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     __syncwarp();
   }
 
-  // ---- V pass: lanes split head_dim
-  float o[EPL], ua[EPL];
+  // ---- V pass: o part += (w s) codes + w z, per stored row of the column's chain
+  float o[EL], ua[EL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
-  const int grp = e0 / gs;
-  const uint32_t* vsz1 = reinterpret_cast<const uint32_t*>(kv.sz[1][1]);
-  for (int idx = 0; idx < n_cols; ++idx) {
+  for (int j = 0; j < EL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
+  float oz = 0.f, uz = 0.f;   // the offsets' share, added to every element at the end
+  for (int i0 = 0; i0 < n_cols; i0 += 8) {
+    const int idx = i0 + cg;
+    if (idx >= n_cols) continue;
     const int c = cols[idx];
     const float wgt = p[idx];
-    if (c > t || c >= n_tok || wgt == 0.f) continue;  // uniform across the warp
+    if (c > t || c >= n_tok || wgt == 0.f) continue;
+    const bool drop = prune && !mark[idx];
     const size_t bh = (size_t)c * H + h;
-    float v[EPL];
-    {
-      const uint32_t pair = vsz1[bh * (HD / gs) + grp];
-      const float s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
-      const float z = half_bits_to_float((uint16_t)(pair >> 16));
-      const uint8_t* cp = kv.codes[1][1] + bh * HD + e0;
-      uint32_t word;
-      if (EPL == 4) word = *reinterpret_cast<const uint32_t*>(cp);
-      else word = *reinterpret_cast<const uint16_t*>(cp);
+    float cf[EL], s, z;
+    load_sz(kv.sz[1][1], bh * ngrp + gidx, &s, &z);
+    load_codes<EL>(kv.codes[1][1] + bh * HD, 8, e0, cf);
+    float ws = wgt * s;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) v[j] = __fmaf_rn(byte_f(word, j), s, z);
+    for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+    oz = fmaf(wgt, z, oz);
+    if (SHRINK && drop) {
+#pragma unroll
+      for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+      uz = fmaf(wgt, z, uz);
     }
     for (int r = 2; r <= P.loop; ++r) {
       const int row = kv.slot[(size_t)r * n_tok + c];
       if (row < 0) continue;
       const int b = kv.res_bits[r];
       const size_t rh = (size_t)row * H + h;
-      const uint32_t pair = reinterpret_cast<const uint32_t*>(kv.sz[1][r])[rh * (HD / gs) + grp];
-      const float s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
-      const float z = half_bits_to_float((uint16_t)(pair >> 16));
-      const uint8_t* rp = kv.codes[1][r] + rh * (HD * b / 8);
-      const int bit0 = e0 * b;
+      load_sz(kv.sz[1][r], rh * ngrp + gidx, &s, &z);
+      load_codes<EL>(kv.codes[1][r] + rh * (HD * b / 8), b, e0, cf);
+      ws = wgt * s;
 #pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int bit = bit0 + j * b;
-        const int code = (rp[bit >> 3] >> (bit & 7)) & ((1 << b) - 1);
-        v[j] = __fadd_rn(v[j], __fmaf_rn((float)code, s, z));
+      for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+      oz = fmaf(wgt, z, oz);
+      if (SHRINK && drop) {
+#pragma unroll
+        for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+        uz = fmaf(wgt, z, uz);
       }
     }
-    const bool drop = prune && !mark[idx];
+  }
+  // reduce the 8 column groups (lanes with the same part differ in bits 2..4)
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      o[j] = fmaf(wgt, v[j], o[j]);
-      if (drop) ua[j] = fmaf(wgt, v[j], ua[j]);
+  for (int j = 0; j < EL; ++j) {
+    o[j] += oz;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) o[j] += __shfl_xor_sync(0xffffffffu, o[j], off);
+    if (SHRINK) {
+      ua[j] += uz;
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) ua[j] += __shfl_xor_sync(0xffffffffu, ua[j], off);
     }
   }
 
-  // ---- outputs
-  const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD;
-  const size_t ob = ((size_t)qi * H + h) * HD + e0;
-  float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD : nullptr;
+  // ---- outputs (lanes 0..3 hold the four parts)
+  if (cg == 0) {
+    const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD + e0;
+    const size_t ob = ((size_t)qi * H + h) * HD + e0;
+    float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + e0 : nullptr;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const float ui = u_in[e0 + j];
-    const float val = ui + o[j];
-    if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(val);
-    else reinterpret_cast<float*>(P.out)[ob + j] = val;
-    if (want_stats) u_out[e0 + j] = prune ? ui + ua[j] : ui;
+    for (int j = 0; j < EL; ++j) {
+      const float ui = u_in[j];
+      const float val = ui + o[j];
+      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(P.out)[ob + j] = val;
+      if (want_stats) u_out[j] = prune ? ui + ua[j] : ui;
+    }
   }
   if (!want_stats) return;
+  __syncwarp();
   uint16_t* so = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
   float lm = 0.f;
   int written = 0;
@@ -330,12 +361,14 @@ cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s) {
   const size_t sm = (size_t)NW * warp_smem(P.hd, P.sel_stride);
   const int warps = P.n_q * P.H;
   const int blocks = (warps + NW - 1) / NW;
-  auto kern = P.hd == 128 ? k_attn_sparse<128> : k_attn_sparse<64>;
-  static int attr_bytes[2][128] = {{0}};
+  const bool shrink = P.sel_out != nullptr && P.k_next + 1 < P.sel_stride;
+  auto kern = P.hd == 128 ? (shrink ? k_attn_sparse<128, true> : k_attn_sparse<128, false>)
+                          : (shrink ? k_attn_sparse<64, true> : k_attn_sparse<64, false>);
+  static int attr_bytes[4][128] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  int& have = attr_bytes[P.hd == 128 ? 1 : 0][dev];
+  int& have = attr_bytes[(P.hd == 128 ? 2 : 0) + (shrink ? 1 : 0)][dev];
   if ((int)sm > have) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;

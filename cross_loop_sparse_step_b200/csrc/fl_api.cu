@@ -44,13 +44,21 @@ struct TimingHook {
 };
 static TimingHook g_hooks[TIMED_KINDS];
 
+// Under stream capture the events become external event-record nodes of the graph, so
+// every replay records them again.
+static void record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive) cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else cudaEventRecord(e, s);
+}
 void timing_begin(int kind, cudaStream_t s) {
   TimingHook& h = g_hooks[kind];
-  if (h.next < (int)h.begin.size()) cudaEventRecord(h.begin[h.next], s);
+  if (h.next < (int)h.begin.size()) record_event(h.begin[h.next], s);
 }
 void timing_end(int kind, cudaStream_t s) {
   TimingHook& h = g_hooks[kind];
-  if (h.next < (int)h.end.size()) cudaEventRecord(h.end[h.next++], s);
+  if (h.next < (int)h.end.size()) record_event(h.end[h.next++], s);
 }
 
 cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,

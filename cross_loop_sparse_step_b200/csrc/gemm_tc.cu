@@ -2,14 +2,15 @@
 // the projections regular GEMMs): C (=|+=) A . W^T, A [M x K] bf16 activations,
 // W [N x K] bf16 linear-layer weights, fp32 accumulation in tensor memory.
 //
-// One 128 x BN output tile per CTA, 6 warps:
+// Persistent CTAs (one per SM) over 128 x BN output tiles, 6 warps:
 //   warp 0     TMA producer: A and W tiles (64 K-columns, 128-byte swizzle) into a
 //              STAGES-deep shared-memory ring, completion counted on mbarriers;
-//   warp 1     allocates TMEM and issues tcgen05.mma (M 128, N BN, K 16) from one
-//              thread; tcgen05.commit frees each ring slot and finally signals the
-//              epilogue;
+//   warp 1     allocates TMEM (two accumulators of BN columns) and issues
+//              tcgen05.mma (M 128, N BN, K 16) from one thread; tcgen05.commit frees
+//              each ring slot and signals the epilogue when a tile is complete;
 //   warps 2-5  epilogue: tcgen05.ld of their 32 TMEM lanes (= tile rows), binary32
-//              store or accumulate into C.
+//              store or accumulate into C (or the SwiGLU product in bf16), then hand
+//              the accumulator back to the MMA warp.
 // Rows beyond M are zero-filled by TMA and not stored. Every mbarrier wait is bounded
 // in time; a wait that runs out records FL_ERR_TIMEOUT and the CTA drains its copies
 // in flight, frees TMEM and returns.
@@ -26,12 +27,15 @@ using namespace sm100;
 
 constexpr int BM = 128, BK = 64;
 
-// EPI_STORE / EPI_ADD: C[M x N] fp32 (=|+=) A . W^T, tile columns n0 = 128 * blockIdx.x.
-// EPI_SWIGLU: W = [gate; up] with `half` rows each; a tile holds 64 gate rows and the
-// matching 64 up rows (two TMA boxes), and the epilogue writes silu(g) * u as bf16 into
-// Y [M x half] at columns 64 * blockIdx.x.
+// EPI_STORE / EPI_ADD: C[M x N] fp32 (=|+=) A . W^T, tiles of 128 x BN.
+// EPI_SWIGLU: W = [gate; up] with `half` rows each; a tile holds BN/2 gate rows and the
+// matching BN/2 up rows (two TMA boxes), and the epilogue writes silu(g) * u as bf16 into
+// Y [M x half].
 constexpr int EPI_SWIGLU = 2;
 
+// Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+// (M-tile fastest, so the CTAs running together share each weight tile through L2).
+// Two TMEM accumulators: the epilogue drains tile i while the MMA warp fills tile i+1.
 template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
@@ -40,26 +44,31 @@ __global__ void __launch_bounds__(192, 1)
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], acc_bar;
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES];
+  __shared__ uint64_t accf_bar[2], acce_bar[2], final_bar;
   __shared__ uint32_t tmem_slot;
   __shared__ int abort_flag;
   volatile int* abort = &abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int nk = K / BK;
+  const int m_tiles = (M + BM - 1) / BM;
+  const int n_tiles = EPI == EPI_SWIGLU ? half / (BN / 2) : N / BN;
+  const int tiles = m_tiles * n_tiles;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-    mbar_init(&acc_bar, 1);
+    for (int a = 0; a < 2; ++a) { mbar_init(&accf_bar[a], 1); mbar_init(&acce_bar[a], 4); }
+    mbar_init(&final_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) { prefetch_tmap(&tma_a); prefetch_tmap(&tma_b); }
-  if (warp == 1) tmem_alloc(&tmem_slot, BN);
+  if (warp == 1) tmem_alloc(&tmem_slot, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -67,27 +76,29 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES, i = kb / STAGES;
-        if (i > 0 && !mbar_wait(&empty_bar[s], (i - 1) & 1, abort)) break;
-        uint8_t* a_dst = smem + s * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
-        tma_load_2d(a_dst, &tma_a, &full_bar[s], kb * BK, m0);
-        if constexpr (EPI == EPI_SWIGLU) {
-          const int f0 = blockIdx.x * (BN / 2);
-          tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, f0);
-          tma_load_2d(a_dst + A_BYTES + B_BYTES / 2, &tma_b, &full_bar[s], kb * BK, half + f0);
-        } else {
-          tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, n0);
+      int g = 0;  // k-blocks issued over all tiles
+      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
+        const int m0 = (tile % m_tiles) * BM;
+        const int nt = tile / m_tiles;
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = g % STAGES, i = g / STAGES;
+          if (i > 0 && !mbar_wait(&empty_bar[s], (i - 1) & 1, abort)) break;
+          uint8_t* a_dst = smem + s * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[s], STAGE_BYTES);
+          tma_load_2d(a_dst, &tma_a, &full_bar[s], kb * BK, m0);
+          if constexpr (EPI == EPI_SWIGLU) {
+            const int f0 = nt * (BN / 2);
+            tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, f0);
+            tma_load_2d(a_dst + A_BYTES + B_BYTES / 2, &tma_b, &full_bar[s], kb * BK, half + f0);
+          } else {
+            tma_load_2d(a_dst + A_BYTES, &tma_b, &full_bar[s], kb * BK, nt * BN);
+          }
         }
-        issued = kb + 1;
       }
       if (*abort) {  // drain the copies still in flight before shared memory is released
         const uint64_t t0 = globaltimer();
-        for (int kb = issued > STAGES ? issued - STAGES : 0; kb < issued; ++kb) {
-          const int s = kb % STAGES;
-          while (!mbar_try_wait(&full_bar[s], (kb / STAGES) & 1))
+        for (int x = g > STAGES ? g - STAGES : 0; x < g; ++x) {
+          while (!mbar_try_wait(&full_bar[x % STAGES], (x / STAGES) & 1))
             if (globaltimer() - t0 > kWaitLimitNs) break;
         }
       }
@@ -95,82 +106,101 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % STAGES, i = kb / STAGES;
-        if (!mbar_wait(&full_bar[s], i & 1, abort)) break;
+      int g = 0, lt = 0;
+      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x, ++lt) {
+        const int a = lt & 1, j = lt >> 1;
+        if (lt >= 2 && !mbar_wait(&acce_bar[a], (j - 1) & 1, abort)) break;
         tc_fence_after();
-        const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
-        const uint32_t b_base = a_base + A_BYTES;
+        const uint32_t d_tmem = tmem + (uint32_t)(a * BN);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = g % STAGES, i = g / STAGES;
+          if (!mbar_wait(&full_bar[s], i & 1, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + s * STAGE_BYTES);
+          const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          mma_bf16(tmem, desc_sw128_kmajor(a_base + kk * 32), desc_sw128_kmajor(b_base + kk * 32),
-                   idesc, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            mma_bf16(d_tmem, desc_sw128_kmajor(a_base + kk * 32),
+                     desc_sw128_kmajor(b_base + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty_bar[s]);
         }
-        mma_commit(&empty_bar[s]);
+        if (!ok) break;
+        mma_commit(&accf_bar[a]);
       }
-      mma_commit(&acc_bar);
+      mma_commit(&final_bar);  // arrives once every MMA issued above has completed
     }
   } else {
     const int ew = warp & 3;  // TMEM lanes [32 ew, 32 ew + 32) belong to this warp
-    const int row = m0 + ew * 32 + lane;
-    // wait for the accumulator (time-bounded only: MMAs already issued must finish
-    // before TMEM is freed, even after an abort elsewhere)
-    bool ok = mbar_try_wait(&acc_bar, 0);
-    if (!ok) {
-      const uint64_t t0 = globaltimer();
-      while (!(ok = mbar_try_wait(&acc_bar, 0)))
-        if (globaltimer() - t0 > kWaitLimitNs) { *abort = 1; break; }
-    }
-    tc_fence_after();
-    if (EPI == EPI_SWIGLU && ok && !*abort) {
-      const int f0 = blockIdx.x * (BN / 2);
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+      const int a = lt & 1, j = lt >> 1;
+      if (!mbar_wait(&accf_bar[a], j & 1, abort)) break;
+      tc_fence_after();
+      const int row = (tile % m_tiles) * BM + ew * 32 + lane;
+      const int nt = tile / m_tiles;
+      const uint32_t t_base = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(a * BN);
+      if constexpr (EPI == EPI_SWIGLU) {
+        const int f0 = nt * (BN / 2);
 #pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
-        float g[32], u[32];
-        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(c * 32), g);
-        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(BN / 2 + c * 32), u);
-        if (row < M) {
-          uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * half + f0 + c * 32);
+        for (int c = 0; c < BN / 64; ++c) {
+          float gv[32], uv[32];
+          tmem_ld32(t_base + (uint32_t)(c * 32), gv);
+          tmem_ld32(t_base + (uint32_t)(BN / 2 + c * 32), uv);
+          if (row < M) {
+            uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * half + f0 + c * 32);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t w[4];
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t wv[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int e = 8 * j + 2 * q;
-              const float y0 = g[e] / (1.0f + expf(-g[e])) * u[e];
-              const float y1 = g[e + 1] / (1.0f + expf(-g[e + 1])) * u[e + 1];
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
-              w[q] = *reinterpret_cast<const uint32_t*>(&b2);
+              for (int q = 0; q < 4; ++q) {
+                const int e = 8 * q4 + 2 * q;
+                const float y0 = gv[e] / (1.0f + expf(-gv[e])) * uv[e];
+                const float y1 = gv[e + 1] / (1.0f + expf(-gv[e + 1])) * uv[e + 1];
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                wv[q] = *reinterpret_cast<const uint32_t*>(&b2);
+              }
+              dst[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
             }
-            dst[j] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      } else {
+        const int n0 = nt * BN;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(t_base + (uint32_t)(c * 32), v);
+          if (row < M) {
+            float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c * 32);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float4 x = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+              if (EPI == EPI_ADD) {
+                const float4 y = dst[q];
+                x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
+              }
+              dst[q] = x;
+            }
           }
         }
       }
-    } else if (EPI != EPI_SWIGLU && ok && !*abort) {
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(c * 32), v);
-        if (row < M) {
-          float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c * 32);
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float4 x = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-            if (EPI == EPI_ADD) {
-              const float4 y = dst[j];
-              x.x += y.x; x.y += y.y; x.z += y.z; x.w += y.w;
-            }
-            dst[j] = x;
-          }
-        }
-      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce_bar[a]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    if (lane == 0) {  // every issued MMA must finish before TMEM is released
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&final_bar, 0))
+        if (globaltimer() - t0 > kWaitLimitNs) { abort_flag = 1; break; }
+    }
+    __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, TMEM_COLS);
   }
   if (threadIdx.x == 0 && abort_flag) record_error(st, FL_ERR_TIMEOUT);
 }
@@ -254,7 +284,10 @@ cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, 
     attr_set[dev] = true;
   }
   const int tiles_n = EPI == EPI_SWIGLU ? (N / 2) / (BN / 2) : N / BN;
-  dim3 grid(tiles_n, (M + BM - 1) / BM);
+  const int tiles = tiles_n * ((M + BM - 1) / BM);
+  static int sms[128] = {0};
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  const int grid = tiles < sms[dev] ? tiles : sms[dev];
   kern<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, status_word());
   count_launch();
   return cudaGetLastError();

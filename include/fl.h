@@ -65,7 +65,8 @@ int64_t fl_launch_count(void);
  * end[i] (each a cudaEvent_t passed as void*) on the launch stream around its next n
  * launches of one kind (0: the projection GEMMs, 1: the attention kernel);
  * fl_timing_recorded(kind) says how many pairs were recorded. n = 0 turns it off.
- * Not thread-safe: set it from the thread that issues the work. */
+ * During stream capture the records become external event-record nodes of the graph
+ * (recorded again at every replay). Not thread-safe: set it from the issuing thread. */
 fl_status fl_set_timing_events(int32_t kind, void* const* begin, void* const* end, int32_t n);
 int32_t fl_timing_recorded(int32_t kind);
 

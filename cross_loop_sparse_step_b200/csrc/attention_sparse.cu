@@ -113,7 +113,11 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     if (lane == 0) record_error(P.st, FL_ERR_RANGE);
     return;
   }
-  const bool want_stats = P.sel_out != nullptr;
+  // statistics for the next loop; nothing to write when they are updated in place and
+  // the budget does not shrink (S' = S, m' = m, u' = u)
+  const bool want_stats = P.sel_out != nullptr &&
+      !(P.sel_out == P.sel && P.mass_out == P.mass && P.unsel_out == P.unsel &&
+        P.out_stride == P.sel_stride && P.k_next + 1 >= P.sel_stride);
 
   // ---- carried column set, cached mass, this lane's part of the query
   const uint16_t* srow_p = P.sel + ((size_t)h * P.stat_rows + srow) * stride;

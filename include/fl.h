@@ -95,6 +95,25 @@ fl_status fl_select_active(const void* h_cur, const void* h_prev, fl_dtype dt,
                            int32_t* out_tok, int32_t* out_pos, float* out_delta,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* Allocation-free variant of fl_select_active, for callers that cannot allocate
+ * device memory at all - for instance code embedded in a host runtime that owns every
+ * device byte and hands a plugin only its input and output buffers, or a deployment
+ * that plans a fixed memory budget up front and forbids allocations afterwards.
+ * (The paper has no counterpart: this is a packaging choice of the library.)
+ * Same computation and outputs as fl_select_active (out_delta not offered); the
+ * normalized changes go to a fixed scratch array of FL_SELECT_NOALLOC_MAX_ROWS floats
+ * (256 KiB) built into the library, which every GPU that loads the library holds until
+ * the process exits. n_rows above that maximum returns FL_ERR_SHAPE without launching.
+ * The first call on a device looks up the scratch array's device address (with that
+ * device current) and caches it: make that first call before any stream capture.
+ * Every call on a device shares the one scratch array, so calls whose work overlaps on
+ * the GPU (other streams or host threads) race; the caller must serialise them. No
+ * scratch content has to survive between calls. Calls no allocator of any kind. */
+#define FL_SELECT_NOALLOC_MAX_ROWS 65536
+fl_status fl_select_active_noalloc(const void* h_cur, const void* h_prev, fl_dtype dt,
+                                   int32_t n_rows, int32_t d, const int32_t* row_tok,
+                                   int32_t k, int32_t* out_tok, int32_t* out_pos, void* stream);
+
 /* ------------------------------------------------------------------------- *
  * Row gather / scatter into compact buffers (§4.4: selected tokens are gathered
  * into compact, GEMM-friendly buffers; §4.1: results go back to their rows).

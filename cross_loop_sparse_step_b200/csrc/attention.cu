@@ -343,6 +343,7 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
   const bool sparse = a.sel != nullptr;
   if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);
+  if (!sparse && dense_fast_eligible(P)) return launch_attn_dense_fast(P, s);
   const int max_cols = sparse ? a.sel_stride : a.kv->n_tok;
   if (sparse) {
     if (P.hd == 128) return launch_t<128, 16>(P, max_cols, s);

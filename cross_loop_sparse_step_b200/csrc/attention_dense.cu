@@ -1,0 +1,287 @@
+// Dense causal attention of loop 1 and the column statistics it hands to loop 2
+// (FlashLoop §4.2: the sparse loops rank columns with statistics of the previous loop;
+// the dense loop is where they are produced). One warp per (query, head).
+//
+// Four lanes per column (a lane owns a quarter of the head slice, one quantisation group
+// at head_dim 128), sixteen columns in flight per warp (two per lane group per step):
+//   K pass   s_j = (sum over parts of s (q . codes) + z sum(q)) / sqrt(hd) + b_j for
+//            j = 0..t, kept in shared memory;
+//   softmax  p_j;
+//   select   (when statistics are asked for and t > k) top-k of c_j = p_j ||V^_j||
+//            (or p_j) over j = 1..t by a warp radix select on the binary32 bits, equal
+//            values to the smaller column; the sink is always kept;
+//   V pass   o = sum p V^, and the dropped columns' share u' = sum_{j not kept} p V^;
+//            m' = sum_kept p; the kept columns are written ascending.
+// Used for loop 1 over an 8-bit base; other cases take the general kernel.
+#include <float.h>
+
+#include "fl_internal.cuh"
+
+namespace fl {
+namespace {
+
+__host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~size_t(15); }
+
+// Per-warp shared memory: p [n_tok] f32 | mark [n_tok] u8 | hist [256] i32.
+__host__ __device__ inline size_t dense_warp_smem(int n_tok) {
+  return a16((size_t)n_tok * 4) + a16((size_t)n_tok) + 256 * 4;
+}
+
+__device__ __forceinline__ float byte_to_f(uint32_t w, int i) {
+  const uint32_t sel = (uint32_t)i | (4u << 4) | (4u << 8) | (7u << 12);
+  return __uint_as_float(__byte_perm(w, 0x4B000000u, sel)) - 8388608.0f;
+}
+
+// 8-bit codes [e0, e0 + EL) of one base row as floats, and the row's (s, z) for them.
+template <int EL>
+__device__ __forceinline__ void base_part(const KvView& kv, int which, size_t bh, int e0,
+                                          int gidx, int ngrp, float* c, float* s, float* z) {
+  const uint32_t pair = reinterpret_cast<const uint32_t*>(kv.sz[which][1])[bh * ngrp + gidx];
+  *s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
+  *z = half_bits_to_float((uint16_t)(pair >> 16));
+  const uint4* p = reinterpret_cast<const uint4*>(kv.codes[which][1] + bh * (size_t)(EL * 4) + e0);
+#pragma unroll
+  for (int k = 0; k < EL / 16; ++k) {
+    const uint4 u = p[k];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[16 * k + 4 * j + i] = byte_to_f(w[j], i);
+  }
+}
+
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ AttnParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  constexpr int EL = HD / 4;
+  const int nw = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * nw + w;
+  if (gw >= P.n_q * P.H) return;  // whole warp leaves; no CTA-wide barrier below
+  const int qi = gw / P.H, h = gw % P.H;
+  const int H = P.H, n_tok = P.kv.n_tok, gs = P.kv.g;
+  const KvView& kv = P.kv;
+  const int l4 = lane & 3, cg = lane >> 2;
+  const int e0 = l4 * EL, gidx = e0 / gs, ngrp = HD / gs;
+
+  uint8_t* base = smem + (size_t)w * dense_warp_smem(n_tok);
+  float* p = reinterpret_cast<float*>(base);
+  uint8_t* mark = base + a16((size_t)n_tok * 4);
+  int* hist = reinterpret_cast<int*>(mark + a16((size_t)n_tok));
+
+  const int t = P.q_tok[qi];
+  const int srow = P.q_row ? P.q_row[qi] : t;
+  const bool want_stats = P.sel_out != nullptr;
+  if (t < 0 || t >= n_tok || (want_stats && (srow < 0 || srow >= P.stat_rows))) {
+    if (lane == 0) record_error(P.st, FL_ERR_RANGE);
+    return;
+  }
+  const int n_cols = t + 1;
+  float qv[EL];
+  float qsum = 0.f;
+  {
+    const size_t off = ((size_t)qi * H + h) * HD + e0;
+#pragma unroll
+    for (int j = 0; j < EL; ++j) {
+      qv[j] = P.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(P.q)[off + j])
+                       : reinterpret_cast<const float*>(P.q)[off + j];
+      qsum += qv[j];
+    }
+  }
+
+  // ---- K pass
+  float lmax = -FLT_MAX;
+  for (int i0 = 0; i0 < n_cols; i0 += 16) {
+    float part[2] = {0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = i0 + 8 * u + cg;
+      if (c < n_cols) {
+        float cf[EL], s, z;
+        base_part<EL>(kv, 0, (size_t)c * H + h, e0, gidx, ngrp, cf, &s, &z);
+        float d = 0.f;
+#pragma unroll
+        for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
+        part[u] = fmaf(s, d, z * qsum);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float v = part[u];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      const int c = i0 + 8 * u + cg;
+      if (c < n_cols && l4 == 0) {
+        const float sc = v * P.scale + (P.bias ? P.bias[c] : 0.f);
+        p[c] = sc;
+        lmax = fmaxf(lmax, sc);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
+  __syncwarp();
+  float lsum = 0.f;
+  for (int c = lane; c < n_cols; c += 32) {
+    const float e = expf(p[c] - lmax);
+    p[c] = e;
+    lsum += e;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  const float inv = 1.0f / lsum;
+  for (int c = lane; c < n_cols; c += 32) p[c] *= inv;
+  __syncwarp();
+
+  // ---- statistics: keep the sink and the top-k of c over columns 1..t
+  const bool prune = want_stats && (n_cols - 1 > P.k_next);
+  if (prune) {
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)P.k_next;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int i = lane; i < 256; i += 32) hist[i] = 0;
+      __syncwarp();
+      for (int c = 1 + lane; c < n_cols; c += 32) {
+        float cv = p[c];
+        if (P.stat_kind == FL_STAT_PV) cv *= P.vnorm[(size_t)c * H + h];
+        const uint32_t b = __float_as_uint(cv);
+        if ((b & pmask) == prefix) atomicAdd(&hist[(b >> shift) & 255u], 1);
+      }
+      __syncwarp();
+      uint32_t dg = 0, above = 0;
+      if (lane == 0) {
+        int d = 255;
+        for (; d > 0; --d) {
+          if (above + (uint32_t)hist[d] >= need) break;
+          above += (uint32_t)hist[d];
+        }
+        dg = (uint32_t)d;
+      }
+      dg = __shfl_sync(0xffffffffu, dg, 0);
+      above = __shfl_sync(0xffffffffu, above, 0);
+      prefix |= dg << shift;
+      need -= above;
+      pmask |= 255u << shift;
+      __syncwarp();
+    }
+    if (lane == 0) mark[0] = 1;
+    int eq_seen = 0;
+    for (int b0 = 1; b0 < n_cols; b0 += 32) {
+      const int c = b0 + lane;
+      const bool valid = c < n_cols;
+      uint32_t b = 0;
+      if (valid) {
+        float cv = p[c];
+        if (P.stat_kind == FL_STAT_PV) cv *= P.vnorm[(size_t)c * H + h];
+        b = __float_as_uint(cv);
+      }
+      const bool is_eq = valid && b == prefix;
+      const uint32_t bal = __ballot_sync(0xffffffffu, is_eq);
+      const int rank = eq_seen + __popc(bal & ((1u << lane) - 1u));
+      if (valid) mark[c] = (b > prefix || (is_eq && (uint32_t)rank < need)) ? 1 : 0;
+      eq_seen += __popc(bal);
+    }
+    __syncwarp();
+  }
+
+  // ---- V pass
+  float o[EL], ua[EL];
+#pragma unroll
+  for (int j = 0; j < EL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
+  float oz = 0.f, uz = 0.f;
+  for (int i0 = 0; i0 < n_cols; i0 += 16) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int c = i0 + 8 * u + cg;
+      if (c >= n_cols) continue;
+      const float wgt = p[c];
+      float cf[EL], s, z;
+      base_part<EL>(kv, 1, (size_t)c * H + h, e0, gidx, ngrp, cf, &s, &z);
+      const float ws = wgt * s;
+#pragma unroll
+      for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+      oz = fmaf(wgt, z, oz);
+      if (prune && !mark[c]) {
+#pragma unroll
+        for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+        uz = fmaf(wgt, z, uz);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < EL; ++j) {
+    o[j] += oz;
+    ua[j] += uz;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      o[j] += __shfl_xor_sync(0xffffffffu, o[j], off);
+      ua[j] += __shfl_xor_sync(0xffffffffu, ua[j], off);
+    }
+  }
+  if (cg == 0) {
+    const size_t ob = ((size_t)qi * H + h) * HD + e0;
+#pragma unroll
+    for (int j = 0; j < EL; ++j) {
+      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(o[j]);
+      else reinterpret_cast<float*>(P.out)[ob + j] = o[j];
+    }
+    if (want_stats) {
+      float* u_out = P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + e0;
+#pragma unroll
+      for (int j = 0; j < EL; ++j) u_out[j] = prune ? ua[j] : 0.f;
+    }
+  }
+  if (!want_stats) return;
+  __syncwarp();
+  uint16_t* so = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
+  float lm = 0.f;
+  int written = 0;
+  for (int b0 = 0; b0 < n_cols; b0 += 32) {
+    const int c = b0 + lane;
+    const bool keep = c < n_cols && (!prune || mark[c]);
+    if (keep) lm += p[c];
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    const int pos = written + __popc(bal & ((1u << lane) - 1u));
+    if (keep && pos < P.out_stride) so[pos] = (uint16_t)c;
+    written += __popc(bal);
+  }
+  for (int i = written + lane; i < P.out_stride; i += 32) so[i] = (uint16_t)FL_SENTINEL;
+#pragma unroll
+  for (int o2 = 16; o2 > 0; o2 >>= 1) lm += __shfl_xor_sync(0xffffffffu, lm, o2);
+  if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = lm;
+}
+
+}  // namespace
+
+bool dense_fast_eligible(const AttnParams& P) {
+  if (P.sel != nullptr || P.loop != 1) return false;
+  if (P.hd != 128 && P.hd != 64) return false;
+  if (P.kv.base_bits != 8 || (P.kv.g != 32 && P.kv.g != 64)) return false;
+  if (P.sel_out && P.stat_kind == FL_STAT_PV && !P.vnorm) return false;
+  return dense_warp_smem(P.kv.n_tok) <= 200 * 1024;
+}
+
+cudaError_t launch_attn_dense_fast(const AttnParams& P, cudaStream_t s) {
+  const size_t per = dense_warp_smem(P.kv.n_tok);
+  int nw = (int)((200 * 1024) / per);
+  nw = nw < 1 ? 1 : (nw > 4 ? 4 : nw);
+  const size_t sm = (size_t)nw * per;
+  const int warps = P.n_q * P.H;
+  const int blocks = (warps + nw - 1) / nw;
+  auto kern = P.hd == 128 ? k_attn_dense<128> : k_attn_dense<64>;
+  static int attr_bytes[2][128] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  int& have = attr_bytes[P.hd == 128 ? 1 : 0][dev];
+  if ((int)sm > have) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    have = (int)sm;
+  }
+  kern<<<blocks, nw * 32, sm, s>>>(P);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace fl

@@ -25,11 +25,11 @@ constexpr int NW = 4;  // warps per CTA
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
-// Per-warp shared memory: q [HD] | qsum [4] | p [stride] | cols [stride] u16 |
-// mark [stride] u8 | hist [256] i32.
+// Per-warp shared memory: (reserved) [HD + 4] f32 | p [stride] f32 | cols [stride] u16 |
+// mark [stride] u8 | hist [256] i32 | list_idx [stride] u16 | list_row [stride] i32.
 __host__ __device__ inline size_t warp_smem(int hd, int stride) {
   return align16((size_t)hd * 4 + 16) + align16((size_t)stride * 4) + align16((size_t)stride * 2) +
-         align16((size_t)stride) + 256 * 4;
+         align16((size_t)stride) + 256 * 4 + align16((size_t)stride * 2) + align16((size_t)stride * 4);
 }
 
 __device__ __forceinline__ float byte_f(uint32_t w, int i) {
@@ -142,8 +142,34 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
   }
   __syncwarp();
 
-  // ---- K pass: 8 columns in flight, q . K^ = sum over parts of s (q . codes) + z sum(q)
-  float lmax = -FLT_MAX;
+  // Work is split so every lane stays busy: a base pass over all columns, then one pass
+  // per loop r = 2..loop over the compacted list of columns that loop rewrote.
+  uint16_t* list_idx = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(hist) + 256 * 4);
+  int32_t* list_row = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(list_idx) + align16((size_t)stride * 2));
+  // compacts {idx : slot[r][cols[idx]] >= 0} into list_idx / list_row; returns its length
+  auto build_list = [&](int r) -> int {
+    int n = 0;
+    const int32_t* srow_r = kv.slot + (size_t)r * n_tok;
+    for (int b0 = 0; b0 < n_cols; b0 += 32) {
+      const int idx = b0 + lane;
+      int row = -1;
+      if (idx < n_cols) {
+        const int c = cols[idx];
+        if (c <= t && c < n_tok) row = srow_r[c];
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, row >= 0);
+      if (row >= 0) {
+        const int pos = n + __popc(bal & ((1u << lane) - 1u));
+        list_idx[pos] = (uint16_t)idx;
+        list_row[pos] = row;
+      }
+      n += __popc(bal);
+    }
+    __syncwarp();
+    return n;
+  };
+
+  // ---- K base pass: 8 columns in flight, score part = s (q . codes) + z sum(q)
   for (int i0 = 0; i0 < n_cols; i0 += 8) {
     const int idx = i0 + cg;
     float part = 0.f;
@@ -153,7 +179,9 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
       c = cols[idx];
       valid = c <= t && c < n_tok;
     }
+    float bias_c = 0.f;
     if (valid) {
+      if (P.bias && l4 == 0) bias_c = P.bias[c];
       const size_t bh = (size_t)c * H + h;
       float cf[EL], sb, zb;
       load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb, &zb);
@@ -162,34 +190,45 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
 #pragma unroll
       for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
       part = fmaf(sb, d, zb * qsum);
-      for (int r = 2; r <= P.loop; ++r) {
-        const int row = kv.slot[(size_t)r * n_tok + c];
-        if (row < 0) continue;
-        const int b = kv.res_bits[r];
-        const size_t rh = (size_t)row * H + h;
-        float sr, zr;
-        load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr, &zr);
-        load_codes<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
-        float dr = 0.f;
-#pragma unroll
-        for (int j = 0; j < EL; ++j) dr = fmaf(qv[j], cf[j], dr);
-        part += fmaf(sr, dr, zr * qsum);
-      }
     }
     part += __shfl_xor_sync(0xffffffffu, part, 1);
     part += __shfl_xor_sync(0xffffffffu, part, 2);
     if (idx < n_cols && l4 == 0) {
-      float sc;
       if (!valid) {
         record_error(P.st, FL_ERR_RANGE);
-        sc = -INFINITY;
+        p[idx] = -INFINITY;
       } else {
-        sc = part * P.scale + (P.bias ? P.bias[c] : 0.f);
+        p[idx] = part * P.scale + bias_c;
       }
-      p[idx] = sc;
-      lmax = fmaxf(lmax, sc);
     }
   }
+  __syncwarp();
+  // ---- K residual passes
+  for (int r = 2; r <= P.loop; ++r) {
+    const int n_r = build_list(r);
+    const int b = kv.res_bits[r];
+    const float sc = P.scale;
+    for (int i0 = 0; i0 < n_r; i0 += 8) {
+      const int li = i0 + cg;
+      float part = 0.f;
+      if (li < n_r) {
+        const size_t rh = (size_t)list_row[li] * H + h;
+        float cf[EL], sr, zr;
+        load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr, &zr);
+        load_codes<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
+        float d = 0.f;
+#pragma unroll
+        for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
+        part = fmaf(sr, d, zr * qsum);
+      }
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (li < n_r && l4 == 0) p[list_idx[li]] += part * sc;
+    }
+    __syncwarp();
+  }
+  float lmax = -FLT_MAX;
+  for (int idx = lane; idx < n_cols; idx += 32) lmax = fmaxf(lmax, p[idx]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lmax = fmaxf(lmax, __shfl_xor_sync(0xffffffffu, lmax, o));
   __syncwarp();
@@ -257,7 +296,7 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     __syncwarp();
   }
 
-  // ---- V pass: o part += (w s) codes + w z, per stored row of the column's chain
+  // ---- V passes: o part += (w s) codes + w z for every stored row of the chain
   float o[EL], ua[EL];
 #pragma unroll
   for (int j = 0; j < EL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
@@ -266,34 +305,39 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     const int idx = i0 + cg;
     if (idx >= n_cols) continue;
     const int c = cols[idx];
+    if (c > t || c >= n_tok) continue;
     const float wgt = p[idx];
-    if (c > t || c >= n_tok || wgt == 0.f) continue;
-    const bool drop = prune && !mark[idx];
     const size_t bh = (size_t)c * H + h;
     float cf[EL], s, z;
     load_sz(kv.sz[1][1], bh * ngrp + gidx, &s, &z);
     load_codes<EL>(kv.codes[1][1] + bh * HD, 8, e0, cf);
-    float ws = wgt * s;
+    const float ws = wgt * s;
 #pragma unroll
     for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
     oz = fmaf(wgt, z, oz);
-    if (SHRINK && drop) {
+    if (SHRINK && prune && !mark[idx]) {
 #pragma unroll
       for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
       uz = fmaf(wgt, z, uz);
     }
-    for (int r = 2; r <= P.loop; ++r) {
-      const int row = kv.slot[(size_t)r * n_tok + c];
-      if (row < 0) continue;
-      const int b = kv.res_bits[r];
-      const size_t rh = (size_t)row * H + h;
+  }
+  for (int r = 2; r <= P.loop; ++r) {
+    const int n_r = build_list(r);
+    const int b = kv.res_bits[r];
+    for (int i0 = 0; i0 < n_r; i0 += 8) {
+      const int li = i0 + cg;
+      if (li >= n_r) continue;
+      const int idx = list_idx[li];
+      const float wgt = p[idx];
+      const size_t rh = (size_t)list_row[li] * H + h;
+      float cf[EL], s, z;
       load_sz(kv.sz[1][r], rh * ngrp + gidx, &s, &z);
       load_codes<EL>(kv.codes[1][r] + rh * (HD * b / 8), b, e0, cf);
-      ws = wgt * s;
+      const float ws = wgt * s;
 #pragma unroll
       for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
       oz = fmaf(wgt, z, oz);
-      if (SHRINK && drop) {
+      if (SHRINK && prune && !mark[idx]) {
 #pragma unroll
         for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
         uz = fmaf(wgt, z, uz);

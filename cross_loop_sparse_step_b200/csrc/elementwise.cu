@@ -56,6 +56,21 @@ __global__ void k_rope_split(const float* __restrict__ qkv, const int32_t* __res
   }
 }
 
+// tab[t][i] = (cos, sin)(t * theta^(-2i/hd)), angle and functions in fp64, t < n_tok.
+__global__ void k_rope_table(float2* __restrict__ tab, int n_tok, int hd, float theta) {
+  const int half = hd / 2;
+  const size_t total = (size_t)n_tok * half;
+  for (size_t id = blockIdx.x * (size_t)blockDim.x + threadIdx.x; id < total;
+       id += (size_t)gridDim.x * blockDim.x) {
+    const int i = (int)(id % half);
+    const int t = (int)(id / half);
+    const double inv_freq = pow((double)theta, -2.0 * (double)i / (double)hd);
+    double sn, cs;
+    sincos((double)t * inv_freq, &sn, &cs);
+    tab[id] = make_float2((float)cs, (float)sn);
+  }
+}
+
 template <typename T>
 __global__ void k_swiglu(const float* __restrict__ gu, int M, int F, T* __restrict__ out) {
   const size_t total = (size_t)M * F;
@@ -87,6 +102,13 @@ cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H
                               float theta, float* q, float* k, float* v, cudaStream_t s) {
   if (M <= 0) return cudaSuccess;
   k_rope_split<<<grid_for((size_t)M * H * hd / 2), 256, 0, s>>>(qkv, pos, M, H, hd, theta, q, k, v);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(float2* tab, int n_tok, int hd, float theta, cudaStream_t s) {
+  if (n_tok <= 0) return cudaSuccess;
+  k_rope_table<<<grid_for((size_t)n_tok * hd / 2), 256, 0, s>>>(tab, n_tok, hd, theta);
   count_launch();
   return cudaGetLastError();
 }

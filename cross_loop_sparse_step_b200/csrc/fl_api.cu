@@ -19,6 +19,10 @@ bool gemm_tc_supported(int M, int N, int K);
 bool gemm_swiglu_supported(int M, int F, int K);
 cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int F, int K,
                                cudaStream_t s);
+bool gemm_qkv_supported(int M, int d, int hd);
+cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
+                            const int32_t* pos, const float2* rope, int M, int d, int hd,
+                            cudaStream_t s);
 
 int* status_word() {
   static int* cache[128] = {nullptr};
@@ -142,21 +146,44 @@ fl_status check_model(const fl_model* m) {
   return FL_OK;
 }
 
+// Block workspace: [RoPE (cos, sin) table of every position][scratch of one half-layer].
+size_t rope_tab_bytes(const fl_model* m) {
+  return align_up((size_t)m->n_tok * (m->head_dim / 2) * sizeof(float2));
+}
+
 size_t block_ws(const fl_model* m, int n) {
   const size_t d = m->d_model, F = m->d_ffn, e = dt_size(m->dt);
   const size_t qkv_path = align_up(n * d * e) + align_up(n * 3 * d * 4);
   const size_t ffn_path = align_up(n * d * e) + align_up(n * 2 * F * 4) + align_up(n * F * e);
-  return qkv_path > ffn_path ? qkv_path : ffn_path;
+  return rope_tab_bytes(m) + (qkv_path > ffn_path ? qkv_path : ffn_path);
+}
+
+bool qkv_fused(const fl_model* m, int n) {
+  return m->dt == FL_BF16 && gemm_qkv_supported(n, m->d_model, m->head_dim);
+}
+
+// Fills the RoPE table at the head of the block workspace (once per call or loop step).
+fl_status prepare_rope(const fl_model* m, void* ws, cudaStream_t s) {
+  FL_TRY(launch_rope_table(static_cast<float2*>(ws), m->n_tok, m->head_dim, m->rope_theta, s));
+  return FL_OK;
 }
 
 fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int32_t* pos,
                   float* q, float* k, float* v, void* ws, cudaStream_t s) {
   const fl_layer_weights& w = m->layers[layer];
   const int d = m->d_model;
-  Carver c(ws);
+  const float2* rope = static_cast<const float2*>(ws);
+  Carver c(static_cast<uint8_t*>(ws) + rope_tab_bytes(m));
   void* a = c.take((size_t)n * d * dt_size(m->dt));
-  float* qkv = (float*)c.take((size_t)n * 3 * d * 4);
   FL_TRY(launch_rmsnorm(x, w.g_attn, m->rms_eps, a, m->dt, n, d, s));
+  if (qkv_fused(m, n)) {
+    timing_begin(TIMED_GEMM, s);
+    cudaError_t e = launch_gemm_qkv(a, w.w_qkv, q, k, v, pos, rope, n, d, m->head_dim, s);
+    timing_end(TIMED_GEMM, s);
+    FL_TRY(e);
+    return FL_OK;
+  }
+  float* qkv = (float*)c.take((size_t)n * 3 * d * 4);
   FL_TRY(launch_gemm(m->dt, a, w.w_qkv, qkv, n, 3 * d, d, 3 * d, EPI_STORE, s));
   FL_TRY(launch_rope_split(qkv, pos, n, m->n_heads, m->head_dim, m->rope_theta, q, k, v, s));
   return FL_OK;
@@ -166,7 +193,7 @@ fl_status run_out_ffn(const fl_model* m, int layer, float* x, int n, const void*
                       cudaStream_t s) {
   const fl_layer_weights& w = m->layers[layer];
   const int d = m->d_model, F = m->d_ffn;
-  Carver c(ws);
+  Carver c(static_cast<uint8_t*>(ws) + rope_tab_bytes(m));
   void* a = c.take((size_t)n * d * dt_size(m->dt));
   float* gu = (float*)c.take((size_t)n * 2 * F * 4);
   void* mid = c.take((size_t)n * F * dt_size(m->dt));
@@ -344,6 +371,8 @@ fl_status fl_block_qkv(const fl_model* m, int32_t layer, const float* x, int32_t
   if (n_rows == 0) return FL_OK;
   FL_CHECK(x && pos && q && k && v, FL_ERR_INVALID_ARG);
   FL_CHECK(ws && ws_bytes >= block_ws(m, n_rows), FL_ERR_WORKSPACE);
+  fl_status rc = prepare_rope(m, ws, S(stream));
+  if (rc != FL_OK) return rc;
   return run_qkv(m, layer, x, n_rows, pos, q, k, v, ws, S(stream));
 }
 
@@ -458,6 +487,8 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
     FL_TRY(cudaMemcpyAsync(st->x_cur, st->x_prev, (size_t)M * row_bytes, cudaMemcpyDeviceToDevice, s));
     X = st->x_cur;
   }
+  rc = prepare_rope(m, blk, s);
+  if (rc != FL_OK) return rc;
   for (int l = 0; l < L; ++l) {
     rc = run_qkv(m, l, X, M, act, q, k, v, blk, s);
     if (rc != FL_OK) return rc;

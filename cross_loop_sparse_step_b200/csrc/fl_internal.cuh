@@ -127,6 +127,8 @@ struct AttnParams {
 
 bool sparse_fast_eligible(const AttnParams& P);
 cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s);
+bool dense_fast_eligible(const AttnParams& P);
+cudaError_t launch_attn_dense_fast(const AttnParams& P, cudaStream_t s);
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);
 template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
@@ -165,6 +167,7 @@ cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* 
                            fl_dtype dt, int M, int d, cudaStream_t s);
 cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H, int hd,
                               float theta, float* q, float* k, float* v, cudaStream_t s);
+cudaError_t launch_rope_table(float2* tab, int n_tok, int hd, float theta, cudaStream_t s);
 cudaError_t launch_swiglu(const float* gu, int M, int F, void* out, fl_dtype dt,
                           cudaStream_t s);
 cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s);

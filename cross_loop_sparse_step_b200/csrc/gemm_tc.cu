@@ -32,6 +32,17 @@ constexpr int BM = 128, BK = 64;
 // matching BN/2 up rows (two TMA boxes), and the epilogue writes silu(g) * u as bf16 into
 // Y [M x half].
 constexpr int EPI_SWIGLU = 2;
+// EPI_QKV: W = w_qkv [3d x d]; a tile of 128 columns lies in q, k or v; the epilogue writes
+// it to q / k / v [M x d] (fp32), rotating q and k by RoPE at position pos[row] with the
+// (cos, sin) table rope[pos][i], i < hd/2 (rotate-half pairs (i, i + hd/2)).
+constexpr int EPI_QKV = 3;
+
+struct QkvOut {
+  float* q; float* k; float* v;
+  const int32_t* pos;
+  const float2* rope;
+  int d, hd;
+};
 
 // Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
 // (M-tile fastest, so the CTAs running together share each weight tile through L2).
@@ -40,7 +51,7 @@ template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
               float* __restrict__ C, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int ldc,
-              int half, int* st) {
+              int half, const QkvOut qo, int* st) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -165,6 +176,41 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
+      } else if constexpr (EPI == EPI_QKV) {
+        const int n0 = nt * BN;
+        const int which = n0 / qo.d, col0 = n0 % qo.d;
+        float* out = which == 0 ? qo.q : (which == 1 ? qo.k : qo.v);
+        const int hh = qo.hd / 2;
+        const int prow = row < M ? qo.pos[row] : 0;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int off = (c * 32) % qo.hd;   // offset inside the head
+          if (which < 2 && off >= hh) continue;  // second halves go with their partners
+          float a[32];
+          tmem_ld32(t_base + (uint32_t)(c * 32), a);
+          if (which == 2) {
+            if (row < M) {
+              float4* dst = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+            }
+            continue;
+          }
+          float b[32];
+          tmem_ld32(t_base + (uint32_t)(c * 32 + hh), b);
+          if (row < M) {
+            const float2* cs = qo.rope + (size_t)prow * hh + off;
+            float* dx = out + (size_t)row * qo.d + col0 + c * 32;
+            float* dy = dx + hh;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 r = cs[j];
+              dx[j] = a[j] * r.x - b[j] * r.y;
+              dy[j] = a[j] * r.y + b[j] * r.x;
+            }
+          }
+        }
       } else {
         const int n0 = nt * BN;
 #pragma unroll 1
@@ -268,7 +314,7 @@ bool get_map(const void* p, int rows, int cols, int box_rows, CUtensorMap* out) 
 
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, int M, int N,
-                      int K, int ldc, cudaStream_t s) {
+                      int K, int ldc, cudaStream_t s, QkvOut qo = QkvOut{}) {
   CUtensorMap ma, mb;
   const int box_b = EPI == EPI_SWIGLU ? BN / 2 : BN;
   if (!get_map(A, M, K, BM, &ma) || !get_map(W, N, K, box_b, &mb)) return cudaErrorInvalidValue;
@@ -288,7 +334,7 @@ cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, 
   static int sms[128] = {0};
   if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
   const int grid = tiles < sms[dev] ? tiles : sms[dev];
-  kern<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, status_word());
+  kern<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, status_word());
   count_launch();
   return cudaGetLastError();
 }
@@ -318,6 +364,21 @@ cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int
     return cudaErrorInvalidValue;
   return launch_bn<128, 6, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
                                        2 * F, K, 0, s);
+}
+
+bool gemm_qkv_supported(int M, int d, int hd) {
+  return gemm_tc_supported(M, 3 * d, d) && (hd == 64 || hd == 128) && d % 128 == 0;
+}
+
+// q, k, v [M x d] fp32 = split(A . w_qkv^T), q and k rotated by RoPE (table `rope`).
+cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
+                            const int32_t* pos, const float2* rope, int M, int d, int hd,
+                            cudaStream_t s) {
+  if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)q % 16 || (uintptr_t)k % 16 ||
+      (uintptr_t)v % 16)
+    return cudaErrorInvalidValue;
+  QkvOut qo{q, k, v, pos, rope, d, hd};
+  return launch_bn<128, 6, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
 }
 
 }  // namespace fl

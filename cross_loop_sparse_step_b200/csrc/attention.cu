@@ -12,6 +12,7 @@
 //   4. o = u + sum P V^ (u = carried unselected contribution, 0 when dense), and the
 //      next loop's m' and u' from the kept / dropped columns.
 #include <float.h>
+#include <vector>
 #include "fl_internal.cuh"
 
 namespace fl {
@@ -327,6 +328,33 @@ cudaError_t launch_t(const AttnParams& P, int max_cols, cudaStream_t s) {
 size_t attention_ws_bytes(const fl_attn_args& a) {
   (void)a;
   return 0;
+}
+
+AttnParams make_attn_params(const fl_attn_args& a, int* st) {
+  AttnParams P;
+  P.q = a.q; P.q_bf16 = a.q_dt == FL_BF16;
+  P.q_tok = a.q_tok; P.n_q = a.n_q; P.H = a.kv->n_heads; P.hd = a.kv->head_dim;
+  P.scale = 1.0f / sqrtf((float)P.hd);
+  P.kv = make_view(*a.kv); P.loop = a.loop; P.bias = a.col_bias;
+  P.sel = a.sel; P.mass = a.mass; P.unsel = a.unsel;
+  P.stat_rows = a.stat_rows; P.sel_stride = a.sel_stride; P.q_row = a.q_row;
+  P.k_next = a.k_next; P.sel_out = a.sel_out; P.mass_out = a.mass_out; P.unsel_out = a.unsel_out;
+  P.out_stride = a.out_stride; P.stat_kind = a.stat_kind; P.vnorm = a.kv->vnorm;
+  P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
+  return P;
+}
+
+size_t attention_batched_ws_bytes(int n) { return (size_t)(n > 0 ? n : 0) * sizeof(AttnParams); }
+
+cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, int* st,
+                                     cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  std::vector<AttnParams> host(n);
+  for (int i = 0; i < n; ++i) host[i] = make_attn_params(args[i], st);
+  // pageable source: the copy is staged before this call returns
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), n * sizeof(AttnParams), cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return e;
+  return launch_attn_sparse_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
 }
 
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {

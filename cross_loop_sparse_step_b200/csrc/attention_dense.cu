@@ -16,6 +16,7 @@
 #include <float.h>
 
 #include "fl_internal.cuh"
+#include "sm100_f32x2.cuh"
 
 namespace fl {
 namespace {
@@ -27,28 +28,14 @@ __host__ __device__ inline size_t dense_warp_smem(int n_tok) {
   return a16((size_t)n_tok * 4) + a16((size_t)n_tok) + 256 * 4;
 }
 
-__device__ __forceinline__ float byte_to_f(uint32_t w, int i) {
-  const uint32_t sel = (uint32_t)i | (4u << 4) | (4u << 8) | (7u << 12);
-  return __uint_as_float(__byte_perm(w, 0x4B000000u, sel)) - 8388608.0f;
-}
-
-// 8-bit codes [e0, e0 + EL) of one base row as floats, and the row's (s, z) for them.
+// 8-bit codes [e0, e0 + EL) of one base row as pairs, and the row's (s, z) for them.
 template <int EL>
 __device__ __forceinline__ void base_part(const KvView& kv, int which, size_t bh, int e0,
-                                          int gidx, int ngrp, float* c, float* s, float* z) {
+                                          int gidx, int ngrp, float2* c, float* s, float* z) {
   const uint32_t pair = reinterpret_cast<const uint32_t*>(kv.sz[which][1])[bh * ngrp + gidx];
   *s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
   *z = half_bits_to_float((uint16_t)(pair >> 16));
-  const uint4* p = reinterpret_cast<const uint4*>(kv.codes[which][1] + bh * (size_t)(EL * 4) + e0);
-#pragma unroll
-  for (int k = 0; k < EL / 16; ++k) {
-    const uint4 u = p[k];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) c[16 * k + 4 * j + i] = byte_to_f(w[j], i);
-  }
+  f2::load_pairs<EL>(kv.codes[which][1] + bh * (size_t)(EL * 4), 8, e0, c);
 }
 
 template <int HD>
@@ -78,15 +65,24 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
     return;
   }
   const int n_cols = t + 1;
-  float qv[EL];
+  float2 qv[EL / 2];
   float qsum = 0.f;
   {
     const size_t off = ((size_t)qi * H + h) * HD + e0;
 #pragma unroll
-    for (int j = 0; j < EL; ++j) {
-      qv[j] = P.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(P.q)[off + j])
-                       : reinterpret_cast<const float*>(P.q)[off + j];
-      qsum += qv[j];
+    for (int k = 0; k < EL / 2; ++k) {
+      float a, b;
+      if (P.q_bf16) {
+        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(P.q) + off;
+        a = __bfloat162float(qb[2 * k]);
+        b = __bfloat162float(qb[2 * k + 1]);
+      } else {
+        const float2 v = reinterpret_cast<const float2*>(reinterpret_cast<const float*>(P.q) + off)[k];
+        a = v.x;
+        b = v.y;
+      }
+      qv[k] = make_float2(a, b);
+      qsum += a + b;
     }
   }
 
@@ -98,12 +94,10 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
     for (int u = 0; u < 2; ++u) {
       const int c = i0 + 8 * u + cg;
       if (c < n_cols) {
-        float cf[EL], s, z;
+        float2 cf[EL / 2];
+        float s, z;
         base_part<EL>(kv, 0, (size_t)c * H + h, e0, gidx, ngrp, cf, &s, &z);
-        float d = 0.f;
-#pragma unroll
-        for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
-        part[u] = fmaf(s, d, z * qsum);
+        part[u] = fmaf(s, f2::dot_pairs<EL>(qv, cf), z * qsum);
       }
     }
 #pragma unroll
@@ -185,9 +179,9 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
   }
 
   // ---- V pass
-  float o[EL], ua[EL];
+  float2 o[EL / 2], ua[EL / 2];
 #pragma unroll
-  for (int j = 0; j < EL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
+  for (int k = 0; k < EL / 2; ++k) { o[k] = make_float2(0.f, 0.f); ua[k] = make_float2(0.f, 0.f); }
   float oz = 0.f, uz = 0.f;
   for (int i0 = 0; i0 < n_cols; i0 += 16) {
 #pragma unroll
@@ -195,40 +189,43 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
       const int c = i0 + 8 * u + cg;
       if (c >= n_cols) continue;
       const float wgt = p[c];
-      float cf[EL], s, z;
+      float2 cf[EL / 2];
+      float s, z;
       base_part<EL>(kv, 1, (size_t)c * H + h, e0, gidx, ngrp, cf, &s, &z);
       const float ws = wgt * s;
-#pragma unroll
-      for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+      f2::axpy_pairs<EL>(ws, cf, o);
       oz = fmaf(wgt, z, oz);
       if (prune && !mark[c]) {
-#pragma unroll
-        for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+        f2::axpy_pairs<EL>(ws, cf, ua);
         uz = fmaf(wgt, z, uz);
       }
     }
   }
+  const float2 oz2 = make_float2(oz, oz), uz2 = make_float2(uz, uz);
 #pragma unroll
-  for (int j = 0; j < EL; ++j) {
-    o[j] += oz;
-    ua[j] += uz;
+  for (int k = 0; k < EL / 2; ++k) {
+    o[k] = f2::add2(o[k], oz2);
+    ua[k] = f2::add2(ua[k], uz2);
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
-      o[j] += __shfl_xor_sync(0xffffffffu, o[j], off);
-      ua[j] += __shfl_xor_sync(0xffffffffu, ua[j], off);
+      o[k].x += __shfl_xor_sync(0xffffffffu, o[k].x, off);
+      o[k].y += __shfl_xor_sync(0xffffffffu, o[k].y, off);
+      ua[k].x += __shfl_xor_sync(0xffffffffu, ua[k].x, off);
+      ua[k].y += __shfl_xor_sync(0xffffffffu, ua[k].y, off);
     }
   }
   if (cg == 0) {
     const size_t ob = ((size_t)qi * H + h) * HD + e0;
 #pragma unroll
     for (int j = 0; j < EL; ++j) {
-      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(o[j]);
-      else reinterpret_cast<float*>(P.out)[ob + j] = o[j];
+      const float ov = (j & 1) ? o[j >> 1].y : o[j >> 1].x;
+      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(ov);
+      else reinterpret_cast<float*>(P.out)[ob + j] = ov;
     }
     if (want_stats) {
       float* u_out = P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + e0;
 #pragma unroll
-      for (int j = 0; j < EL; ++j) u_out[j] = prune ? ua[j] : 0.f;
+      for (int j = 0; j < EL; ++j) u_out[j] = prune ? ((j & 1) ? ua[j >> 1].y : ua[j >> 1].x) : 0.f;
     }
   }
   if (!want_stats) return;

@@ -8,7 +8,8 @@
 //   of the head slice (one quantisation group at head_dim 128) and keeps its part of q
 //   in registers.
 //   K pass: every stored row of the column's chain (base, then each loop that rewrote
-//     it) contributes s * (q . codes) + z * sum(q) - dequantisation folded into the dot.
+//     it) contributes s * (q . codes) + z * sum(q) - dequantisation folded into the dot;
+//     codes are decoded in pairs and the dots use packed binary32 pair FMAs.
 //   softmax over the column set, p~ = m * softmax (m = cached mass).
 //   optional budget shrink: warp radix select over the binary32 bits of p~ * ||V^||
 //     (ties to the smaller column), ballot-ordered so the kept set stays ascending.
@@ -17,6 +18,7 @@
 #include <float.h>
 
 #include "fl_internal.cuh"
+#include "sm100_f32x2.cuh"
 
 namespace fl {
 namespace {
@@ -32,50 +34,6 @@ __host__ __device__ inline size_t warp_smem(int hd, int stride) {
          align16((size_t)stride) + 256 * 4 + align16((size_t)stride * 2) + align16((size_t)stride * 4);
 }
 
-__device__ __forceinline__ float byte_f(uint32_t w, int i) {
-  // (float)((w >> 8i) & 0xFF), exact: the byte under the exponent of 2^23, minus 2^23
-  const uint32_t sel = (uint32_t)i | (4u << 4) | (4u << 8) | (7u << 12);
-  return __uint_as_float(__byte_perm(w, 0x4B000000u, sel)) - 8388608.0f;
-}
-
-__device__ __forceinline__ float nib_f(uint32_t w, int i, int bits) {
-  const uint32_t c = (w >> (i * bits)) & ((1u << bits) - 1u);
-  return __uint_as_float(0x4B000000u | c) - 8388608.0f;
-}
-
-// Codes [e0, e0 + EL) of one stored row (b bits, little-endian) as floats.
-template <int EL>
-__device__ __forceinline__ void load_codes(const uint8_t* row, int bits, int e0, float* c) {
-  if (bits == 8) {
-    const uint4* p = reinterpret_cast<const uint4*>(row + e0);
-#pragma unroll
-    for (int k = 0; k < EL / 16; ++k) {
-      const uint4 u = p[k];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) c[16 * k + 4 * j + i] = byte_f(w[j], i);
-    }
-  } else if (bits == 4) {
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + e0 / 2);
-#pragma unroll
-    for (int k = 0; k < EL / 8; ++k) {
-      const uint32_t w = p[k];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) c[8 * k + i] = nib_f(w, i, 4);
-    }
-  } else {  // 2 bits
-    const uint32_t* p = reinterpret_cast<const uint32_t*>(row + e0 / 4);
-#pragma unroll
-    for (int k = 0; k < EL / 16; ++k) {
-      const uint32_t w = p[k];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) c[16 * k + i] = nib_f(w, i, 2);
-    }
-  }
-}
-
 __device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s, float* z) {
   const uint32_t pair = reinterpret_cast<const uint32_t*>(sz)[idx];
   *s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
@@ -86,13 +44,12 @@ __device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s
 // the head slice, EL = HD / 4 (32 at HD 128), which lie in one quantisation group.
 // SHRINK: the call may shrink the budget (k_next below the carried set size), so the
 // dropped columns' contribution is accumulated too.
+// One warp's work: (query, head) number gw of the call described by P, with `base` the
+// warp's shared-memory slice. No CTA-wide barrier is used.
 template <int HD, bool SHRINK>
-__global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__ AttnParams P) {
-  extern __shared__ __align__(16) uint8_t smem[];
+__device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, uint8_t* base) {
   constexpr int EL = HD / 4;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * NW + w;
-  if (gw >= P.n_q * P.H) return;  // whole warp leaves; no CTA-wide barrier below
+  const int lane = threadIdx.x & 31;
   const int qi = gw / P.H, h = gw % P.H;
   const int H = P.H, n_tok = P.kv.n_tok, gs = P.kv.g, stride = P.sel_stride;
   const KvView& kv = P.kv;
@@ -101,7 +58,6 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
   const int gidx = e0 / gs;                  // quantisation group of this lane's part
   const int ngrp = HD / gs;
 
-  uint8_t* base = smem + (size_t)w * warp_smem(HD, stride);
   float* p = reinterpret_cast<float*>(base + align16((size_t)HD * 4 + 16));
   uint16_t* cols = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p) + align16((size_t)stride * 4));
   uint8_t* mark = reinterpret_cast<uint8_t*>(cols) + align16((size_t)stride * 2);
@@ -129,15 +85,24 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     n_cols += __popc(__ballot_sync(0xffffffffu, c != FL_SENTINEL));
   }
   const float m_in = P.mass[(size_t)h * P.stat_rows + srow];
-  float qv[EL];
+  float2 qv[EL / 2];
   float qsum = 0.f;
   {
     const size_t off = ((size_t)qi * H + h) * HD + e0;
 #pragma unroll
-    for (int j = 0; j < EL; ++j) {
-      qv[j] = P.q_bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(P.q)[off + j])
-                       : reinterpret_cast<const float*>(P.q)[off + j];
-      qsum += qv[j];
+    for (int k = 0; k < EL / 2; ++k) {
+      float a, b;
+      if (P.q_bf16) {
+        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(P.q) + off;
+        a = __bfloat162float(qb[2 * k]);
+        b = __bfloat162float(qb[2 * k + 1]);
+      } else {
+        const float2 v = reinterpret_cast<const float2*>(reinterpret_cast<const float*>(P.q) + off)[k];
+        a = v.x;
+        b = v.y;
+      }
+      qv[k] = make_float2(a, b);
+      qsum += a + b;
     }
   }
   __syncwarp();
@@ -183,12 +148,11 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     if (valid) {
       if (P.bias && l4 == 0) bias_c = P.bias[c];
       const size_t bh = (size_t)c * H + h;
-      float cf[EL], sb, zb;
+      float2 cf[EL / 2];
+      float sb, zb;
       load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb, &zb);
-      load_codes<EL>(kv.codes[0][1] + bh * HD, 8, e0, cf);
-      float d = 0.f;
-#pragma unroll
-      for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
+      f2::load_pairs<EL>(kv.codes[0][1] + bh * HD, 8, e0, cf);
+      const float d = f2::dot_pairs<EL>(qv, cf);
       part = fmaf(sb, d, zb * qsum);
     }
     part += __shfl_xor_sync(0xffffffffu, part, 1);
@@ -213,12 +177,11 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
       float part = 0.f;
       if (li < n_r) {
         const size_t rh = (size_t)list_row[li] * H + h;
-        float cf[EL], sr, zr;
+        float2 cf[EL / 2];
+        float sr, zr;
         load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr, &zr);
-        load_codes<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
-        float d = 0.f;
-#pragma unroll
-        for (int j = 0; j < EL; ++j) d = fmaf(qv[j], cf[j], d);
+        f2::load_pairs<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
+        const float d = f2::dot_pairs<EL>(qv, cf);
         part = fmaf(sr, d, zr * qsum);
       }
       part += __shfl_xor_sync(0xffffffffu, part, 1);
@@ -297,9 +260,9 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
   }
 
   // ---- V passes: o part += (w s) codes + w z for every stored row of the chain
-  float o[EL], ua[EL];
+  float2 o[EL / 2], ua[EL / 2];
 #pragma unroll
-  for (int j = 0; j < EL; ++j) { o[j] = 0.f; ua[j] = 0.f; }
+  for (int k = 0; k < EL / 2; ++k) { o[k] = make_float2(0.f, 0.f); ua[k] = make_float2(0.f, 0.f); }
   float oz = 0.f, uz = 0.f;   // the offsets' share, added to every element at the end
   for (int i0 = 0; i0 < n_cols; i0 += 8) {
     const int idx = i0 + cg;
@@ -308,16 +271,15 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
     if (c > t || c >= n_tok) continue;
     const float wgt = p[idx];
     const size_t bh = (size_t)c * H + h;
-    float cf[EL], s, z;
+    float2 cf[EL / 2];
+    float s, z;
     load_sz(kv.sz[1][1], bh * ngrp + gidx, &s, &z);
-    load_codes<EL>(kv.codes[1][1] + bh * HD, 8, e0, cf);
+    f2::load_pairs<EL>(kv.codes[1][1] + bh * HD, 8, e0, cf);
     const float ws = wgt * s;
-#pragma unroll
-    for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+    f2::axpy_pairs<EL>(ws, cf, o);
     oz = fmaf(wgt, z, oz);
     if (SHRINK && prune && !mark[idx]) {
-#pragma unroll
-      for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+      f2::axpy_pairs<EL>(ws, cf, ua);
       uz = fmaf(wgt, z, uz);
     }
   }
@@ -330,30 +292,36 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
       const int idx = list_idx[li];
       const float wgt = p[idx];
       const size_t rh = (size_t)list_row[li] * H + h;
-      float cf[EL], s, z;
+      float2 cf[EL / 2];
+      float s, z;
       load_sz(kv.sz[1][r], rh * ngrp + gidx, &s, &z);
-      load_codes<EL>(kv.codes[1][r] + rh * (HD * b / 8), b, e0, cf);
+      f2::load_pairs<EL>(kv.codes[1][r] + rh * (HD * b / 8), b, e0, cf);
       const float ws = wgt * s;
-#pragma unroll
-      for (int j = 0; j < EL; ++j) o[j] = fmaf(ws, cf[j], o[j]);
+      f2::axpy_pairs<EL>(ws, cf, o);
       oz = fmaf(wgt, z, oz);
       if (SHRINK && prune && !mark[idx]) {
-#pragma unroll
-        for (int j = 0; j < EL; ++j) ua[j] = fmaf(ws, cf[j], ua[j]);
+        f2::axpy_pairs<EL>(ws, cf, ua);
         uz = fmaf(wgt, z, uz);
       }
     }
   }
   // reduce the 8 column groups (lanes with the same part differ in bits 2..4)
+  const float2 oz2 = make_float2(oz, oz), uz2 = make_float2(uz, uz);
 #pragma unroll
-  for (int j = 0; j < EL; ++j) {
-    o[j] += oz;
+  for (int k = 0; k < EL / 2; ++k) {
+    o[k] = f2::add2(o[k], oz2);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) o[j] += __shfl_xor_sync(0xffffffffu, o[j], off);
+    for (int off = 4; off < 32; off <<= 1) {
+      o[k].x += __shfl_xor_sync(0xffffffffu, o[k].x, off);
+      o[k].y += __shfl_xor_sync(0xffffffffu, o[k].y, off);
+    }
     if (SHRINK) {
-      ua[j] += uz;
+      ua[k] = f2::add2(ua[k], uz2);
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) ua[j] += __shfl_xor_sync(0xffffffffu, ua[j], off);
+      for (int off = 4; off < 32; off <<= 1) {
+        ua[k].x += __shfl_xor_sync(0xffffffffu, ua[k].x, off);
+        ua[k].y += __shfl_xor_sync(0xffffffffu, ua[k].y, off);
+      }
     }
   }
 
@@ -365,10 +333,10 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
 #pragma unroll
     for (int j = 0; j < EL; ++j) {
       const float ui = u_in[j];
-      const float val = ui + o[j];
+      const float val = ui + ((j & 1) ? o[j >> 1].y : o[j >> 1].x);
       if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(val);
       else reinterpret_cast<float*>(P.out)[ob + j] = val;
-      if (want_stats) u_out[j] = prune ? ui + ua[j] : ui;
+      if (want_stats) u_out[j] = prune ? ui + ((j & 1) ? ua[j >> 1].y : ua[j >> 1].x) : ui;
     }
   }
   if (!want_stats) return;
@@ -389,6 +357,27 @@ __global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__
 #pragma unroll
   for (int o2 = 16; o2 > 0; o2 >>= 1) lm += __shfl_xor_sync(0xffffffffu, lm, o2);
   if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = prune ? lm : m_in;
+}
+
+template <int HD, bool SHRINK>
+__global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__ AttnParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int w = threadIdx.x >> 5;
+  const int gw = blockIdx.x * NW + w;
+  if (gw >= P.n_q * P.H) return;  // whole warp leaves
+  attn_sparse_warp<HD, SHRINK>(P, gw, smem + (size_t)w * warp_smem(HD, P.sel_stride));
+}
+
+// Many independent calls in one launch (batched decode: one store per sequence). The
+// calls share n_q, heads, head_dim and carried-set stride; `per` = n_q * H warps each.
+template <int HD, bool SHRINK>
+__global__ void __launch_bounds__(NW * 32)
+    k_attn_sparse_batched(const AttnParams* __restrict__ Ps, int n_calls, int per, int stride) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int w = threadIdx.x >> 5;
+  const int gw = blockIdx.x * NW + w;
+  if (gw >= n_calls * per) return;
+  attn_sparse_warp<HD, SHRINK>(Ps[gw / per], gw % per, smem + (size_t)w * warp_smem(HD, stride));
 }
 
 }  // namespace
@@ -423,6 +412,31 @@ cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s) {
     have = (int)sm;
   }
   kern<<<blocks, NW * 32, sm, s>>>(P);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Ps: device array of n AttnParams (already copied by the caller, same shapes).
+cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
+                                       cudaStream_t s) {
+  const size_t sm = (size_t)NW * warp_smem(P0.hd, P0.sel_stride);
+  const int per = P0.n_q * P0.H;
+  const long long warps = (long long)per * n;
+  const int blocks = (int)((warps + NW - 1) / NW);
+  const bool shrink = P0.sel_out != nullptr && P0.k_next + 1 < P0.sel_stride;
+  auto kern = P0.hd == 128 ? (shrink ? k_attn_sparse_batched<128, true> : k_attn_sparse_batched<128, false>)
+                           : (shrink ? k_attn_sparse_batched<64, true> : k_attn_sparse_batched<64, false>);
+  static int attr_bytes[4][128] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  int& have = attr_bytes[(P0.hd == 128 ? 2 : 0) + (shrink ? 1 : 0)][dev];
+  if ((int)sm > have) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    have = (int)sm;
+  }
+  kern<<<blocks, NW * 32, sm, s>>>(Ps_dev, n, per, P0.sel_stride);
   count_launch();
   return cudaGetLastError();
 }

@@ -346,6 +346,28 @@ fl_status fl_kv_residual_quant(const fl_kv_desc* kv, int32_t loop, const void* k
                                  S(stream)));
 }
 
+fl_status fl_kv_append(const fl_kv_desc* kv, int32_t loop, const void* k_new, const void* v_new,
+                       fl_dtype dt, const int32_t* act_tok, int32_t n_act, int32_t row0,
+                       void* stream) {
+  fl_status st = check_kv(kv);
+  if (st != FL_OK) return st;
+  FL_CHECK(k_new && v_new && act_tok, FL_ERR_INVALID_ARG);
+  FL_CHECK(valid_dt(dt), FL_ERR_UNSUPPORTED);
+  FL_CHECK(loop >= 1 && loop <= kv->n_loops, FL_ERR_SHAPE);
+  FL_CHECK(n_act >= 0 && n_act <= kv->n_tok && row0 >= 0, FL_ERR_SHAPE);
+  if (n_act == 0) return FL_OK;
+  const int bits = loop == 1 ? kv->base_bits : kv->res_bits[loop];
+  FL_CHECK(kv->codes[0][loop] && kv->codes[1][loop], FL_ERR_INVALID_ARG);
+  if (bits != 0) FL_CHECK(kv->sz[0][loop] && kv->sz[1][loop], FL_ERR_INVALID_ARG);
+  for (int r = 1; r < loop; ++r) {
+    FL_CHECK(kv->codes[0][r] && kv->codes[1][r], FL_ERR_INVALID_ARG);
+    const int br = r == 1 ? kv->base_bits : kv->res_bits[r];
+    if (br != 0) FL_CHECK(kv->sz[0][r] && kv->sz[1][r], FL_ERR_INVALID_ARG);
+  }
+  return cuda_st(launch_kv_quant(*kv, loop, k_new, v_new, dt, act_tok, n_act, status_word(),
+                                 S(stream), loop == 1 ? 0 : row0, true));
+}
+
 size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a) {
   return a ? attention_ws_bytes(*a) : 0;
 }
@@ -355,6 +377,35 @@ fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream) {
   if (st != FL_OK) return st;
   if (a->n_q == 0) return FL_OK;
   return cuda_st(launch_attention_timed(*a, status_word(), S(stream)));
+}
+
+size_t fl_sparse_loop_attn_batched_workspace_bytes(int32_t n) {
+  return align_up(attention_batched_ws_bytes(n));
+}
+
+fl_status fl_sparse_loop_attn_batched(const fl_attn_args* args, int32_t n, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  FL_CHECK(args && n >= 0, FL_ERR_INVALID_ARG);
+  if (n == 0) return FL_OK;
+  FL_CHECK(ws && ws_bytes >= fl_sparse_loop_attn_batched_workspace_bytes(n), FL_ERR_WORKSPACE);
+  const fl_attn_args& a0 = args[0];
+  for (int i = 0; i < n; ++i) {
+    const fl_attn_args& a = args[i];
+    fl_status st = check_attn(&a);
+    if (st != FL_OK) return st;
+    FL_CHECK(a.sel != nullptr, FL_ERR_UNSUPPORTED);
+    FL_CHECK(a.n_q == a0.n_q && a.kv->n_heads == a0.kv->n_heads &&
+             a.kv->head_dim == a0.kv->head_dim && a.sel_stride == a0.sel_stride &&
+             a.q_dt == a0.q_dt && a.out_dt == a0.out_dt && a.stat_kind == a0.stat_kind &&
+             (a.sel_out != nullptr) == (a0.sel_out != nullptr) && a.k_next == a0.k_next,
+             FL_ERR_SHAPE);
+    FL_CHECK(sparse_fast_eligible(make_attn_params(a, nullptr)), FL_ERR_UNSUPPORTED);
+  }
+  if (a0.n_q == 0) return FL_OK;
+  timing_begin(TIMED_ATTN, S(stream));
+  cudaError_t e = launch_attention_batched(args, n, ws, status_word(), S(stream));
+  timing_end(TIMED_ATTN, S(stream));
+  return cuda_st(e);
 }
 
 size_t fl_block_workspace_bytes(const fl_model* m, int32_t n_rows) {

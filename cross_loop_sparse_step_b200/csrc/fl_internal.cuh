@@ -127,6 +127,12 @@ struct AttnParams {
 
 bool sparse_fast_eligible(const AttnParams& P);
 cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s);
+cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
+                                       cudaStream_t s);
+AttnParams make_attn_params(const fl_attn_args& a, int* st);
+size_t attention_batched_ws_bytes(int n);
+cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, int* st,
+                                     cudaStream_t s);
 bool dense_fast_eligible(const AttnParams& P);
 cudaError_t launch_attn_dense_fast(const AttnParams& P, cudaStream_t s);
 
@@ -153,9 +159,11 @@ cudaError_t launch_topk_rows(const float* delta, int n, int k, const int32_t* ro
 cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const int32_t* idx,
                                   int n_idx, int n_full, size_t row_bytes, int* st,
                                   cudaStream_t s);
+// append: keep the slot entries of other tokens and write rows row0.. (decode);
+// otherwise rows 0.. and slot[loop] rewritten for exactly the given tokens.
 cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
                             const void* v_new, fl_dtype dt, const int32_t* act_tok, int n_act,
-                            int* st, cudaStream_t s);
+                            int* st, cudaStream_t s, int row0 = 0, bool append = false);
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s);
 size_t attention_ws_bytes(const fl_attn_args& a);
 

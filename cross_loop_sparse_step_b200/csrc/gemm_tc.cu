@@ -200,14 +200,19 @@ __global__ void __launch_bounds__(192, 1)
           float b[32];
           tmem_ld32(t_base + (uint32_t)(c * 32 + hh), b);
           if (row < M) {
-            const float2* cs = qo.rope + (size_t)prow * hh + off;
-            float* dx = out + (size_t)row * qo.d + col0 + c * 32;
-            float* dy = dx + hh;
+            // (cos, sin) of 4 consecutive angles = 2 float4; 16-byte loads and stores
+            const float4* cs = reinterpret_cast<const float4*>(qo.rope + (size_t)prow * hh + off);
+            float4* dx = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
+            float4* dy = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32 + hh);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 r = cs[j];
-              dx[j] = a[j] * r.x - b[j] * r.y;
-              dy[j] = a[j] * r.y + b[j] * r.x;
+            for (int q = 0; q < 8; ++q) {
+              const float4 r01 = cs[2 * q], r23 = cs[2 * q + 1];
+              const float* x = a + 4 * q;
+              const float* y = b + 4 * q;
+              dx[q] = make_float4(x[0] * r01.x - y[0] * r01.y, x[1] * r01.z - y[1] * r01.w,
+                                  x[2] * r23.x - y[2] * r23.y, x[3] * r23.z - y[3] * r23.w);
+              dy[q] = make_float4(x[0] * r01.y + y[0] * r01.x, x[1] * r01.w + y[1] * r01.z,
+                                  x[2] * r23.y + y[2] * r23.x, x[3] * r23.w + y[3] * r23.z);
             }
           }
         }

@@ -23,6 +23,7 @@ struct QuantOut {
   uint16_t* sz[2];
   int32_t* slot_row;  // slot[loop][*] (loop >= 2) or nullptr
   float* vnorm;       // [n_tok][H] or nullptr
+  int row0;           // first residual row written (loop >= 2)
 };
 
 template <int EPL, typename T>
@@ -60,7 +61,7 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
 #pragma unroll
     for (int j = 0; j < EPL; ++j) x[j] = xin[j];
   }
-  const int row = loop == 1 ? t : i;
+  const int row = loop == 1 ? t : out.row0 + i;
   float hat[EPL];
   if (bits == 0) {
     float* dst = reinterpret_cast<float*>(out.codes[which]) + ((size_t)row * H + h) * hd + e0;
@@ -120,7 +121,7 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) out.vnorm[(size_t)t * H + h] = sqrtf(ss);
   }
-  if (loop >= 2 && which == 0 && h == 0 && lane == 0 && out.slot_row) out.slot_row[t] = i;
+  if (loop >= 2 && which == 0 && h == 0 && lane == 0 && out.slot_row) out.slot_row[t] = row;
 }
 
 template <int EPL>
@@ -143,19 +144,22 @@ cudaError_t launch_epl(const KvView& v, const QuantOut& o, int loop, const void*
 
 cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
                             const void* v_new, fl_dtype dt, const int32_t* act_tok, int n_act,
-                            int* st, cudaStream_t s) {
+                            int* st, cudaStream_t s, int row0, bool append) {
   if (n_act <= 0) return cudaSuccess;
   KvView v = make_view(kv);
   QuantOut o;
   for (int w = 0; w < 2; ++w) { o.codes[w] = kv.codes[w][loop]; o.sz[w] = kv.sz[w][loop]; }
   o.slot_row = nullptr;
   o.vnorm = kv.vnorm;
+  o.row0 = row0;
   cudaError_t e;
   if (loop >= 2) {
     o.slot_row = kv.slot + (size_t)loop * kv.n_tok;
-    e = launch_fill_i32(o.slot_row, -1, (size_t)kv.n_tok, s);
-    if (e != cudaSuccess) return e;
-  } else if (kv.slot) {
+    if (!append) {
+      e = launch_fill_i32(o.slot_row, -1, (size_t)kv.n_tok, s);
+      if (e != cudaSuccess) return e;
+    }
+  } else if (kv.slot && !append) {
     e = launch_iota(kv.slot + kv.n_tok, kv.n_tok, s);
     if (e != cudaSuccess) return e;
   }

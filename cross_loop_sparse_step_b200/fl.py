@@ -99,6 +99,10 @@ _select = _sig("fl_select_active", c_i32,
 _gs = _sig("fl_gather_scatter", c_i32, [c_i32, vp, vp, vp, c_i32, c_i32, c_i32, c_i32, vp])
 _quant = _sig("fl_kv_residual_quant", c_i32,
               [ctypes.POINTER(KvDesc), c_i32, vp, vp, c_i32, vp, c_i32, vp])
+_append = _sig("fl_kv_append", c_i32,
+               [ctypes.POINTER(KvDesc), c_i32, vp, vp, c_i32, vp, c_i32, c_i32, vp])
+_attn_b_ws = _sig("fl_sparse_loop_attn_batched_workspace_bytes", c_sz, [c_i32])
+_attn_b = _sig("fl_sparse_loop_attn_batched", c_i32, [ctypes.POINTER(AttnArgs), c_i32, vp, c_sz, vp])
 _attn_ws = _sig("fl_sparse_loop_attn_workspace_bytes", c_sz, [ctypes.POINTER(AttnArgs)])
 _attn = _sig("fl_sparse_loop_attn", c_i32, [ctypes.POINTER(AttnArgs), vp])
 _blk_ws = _sig("fl_block_workspace_bytes", c_sz, [ctypes.POINTER(Model), c_i32])
@@ -235,9 +239,16 @@ def kv_residual_quant(store, loop, k_new, v_new, act_tok=None, stream=None):
                ptr(act_tok), n_act, stream_handle(stream)), "fl_kv_residual_quant")
 
 
-def sparse_loop_attn(q, q_tok, store, loop, out, col_bias=None, sel=None, mass=None, unsel=None,
-                     q_row=None, k_next=0, sel_out=None, mass_out=None, unsel_out=None,
-                     stat_kind=STAT_PV, stat_rows=None, stream=None):
+def kv_append(store, loop, k_new, v_new, act_tok, row0=0, stream=None):
+    """Decode: add the tokens act_tok to loop `loop` (rows row0.. for loop >= 2)."""
+    _ok(_append(ctypes.byref(store.desc), loop, ptr(k_new), ptr(v_new), dtype_code(k_new),
+                ptr(act_tok), act_tok.numel(), row0, stream_handle(stream)), "fl_kv_append")
+
+
+def make_attn_args(q, q_tok, store, loop, out, col_bias=None, sel=None, mass=None, unsel=None,
+                   q_row=None, k_next=0, sel_out=None, mass_out=None, unsel_out=None,
+                   stat_kind=STAT_PV, stat_rows=None):
+    """fl_attn_args for tensors that the caller keeps alive during the call."""
     a = AttnArgs()
     a.q, a.q_dt, a.n_q, a.q_tok = q.data_ptr(), dtype_code(q), q.shape[0], q_tok.data_ptr()
     a.kv = ctypes.pointer(store.desc)
@@ -253,11 +264,30 @@ def sparse_loop_attn(q, q_tok, store, loop, out, col_bias=None, sel=None, mass=N
     a.out_stride = sel_out.shape[2] if sel_out is not None else 0
     a.stat_kind = stat_kind
     a.out, a.out_dt = out.data_ptr(), dtype_code(out)
+    return a
+
+
+def sparse_loop_attn(q, q_tok, store, loop, out, col_bias=None, sel=None, mass=None, unsel=None,
+                     q_row=None, k_next=0, sel_out=None, mass_out=None, unsel_out=None,
+                     stat_kind=STAT_PV, stat_rows=None, stream=None):
+    a = make_attn_args(q, q_tok, store, loop, out, col_bias, sel, mass, unsel, q_row, k_next,
+                       sel_out, mass_out, unsel_out, stat_kind, stat_rows)
     nb = _attn_ws(ctypes.byref(a))
     ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device) if nb else None
     a.ws, a.ws_bytes = ptr(ws), nb
     _ok(_attn(ctypes.byref(a), stream_handle(stream)), "fl_sparse_loop_attn")
     return out
+
+
+def sparse_loop_attn_batched(args, stream=None):
+    """One launch over several calls' fl_attn_args (see make_attn_args)."""
+    n = len(args)
+    arr = (AttnArgs * n)(*args)
+    nb = _attn_b_ws(n)
+    dev = torch.cuda.current_device()
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device=f"cuda:{dev}")
+    _ok(_attn_b(arr, n, ptr(ws), nb, stream_handle(stream)), "fl_sparse_loop_attn_batched")
+    return ws
 
 
 class LoopModel:

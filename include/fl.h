@@ -175,6 +175,16 @@ fl_status fl_kv_residual_quant(const fl_kv_desc* kv, int32_t loop, const void* k
                                const void* v_new, fl_dtype dt, const int32_t* act_tok,
                                int32_t n_act, void* stream);
 
+/* Append tokens to loop `loop` of the store without disturbing the other tokens (a
+ * decode step's new token, §4.3 applied to generation). loop 1: base rows of the tokens
+ * act_tok[i] (the row of a token is its id). loop >= 2: residual rows row0 + i against
+ * the tokens' reconstruction at loop - 1 (which must exist), slot[loop][act_tok[i]] =
+ * row0 + i; other slot entries are kept. k_new, v_new: device [n_act][H][hd] of dtype dt;
+ * act_tok: device int32 [n_act]. Refreshes vnorm for the written tokens. */
+fl_status fl_kv_append(const fl_kv_desc* kv, int32_t loop, const void* k_new, const void* v_new,
+                       fl_dtype dt, const int32_t* act_tok, int32_t n_act, int32_t row0,
+                       void* stream);
+
 /* ------------------------------------------------------------------------- *
  * Loop-aware sparse attention (§4.2), and the dense causal attention of a loop
  * whose successor is sparse (the producer of the statistics).
@@ -218,6 +228,16 @@ typedef struct {
 
 size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a);
 fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream);
+
+/* n sparse calls (sel != NULL) in one launch - batched decode, where every sequence has
+ * its own store and statistics. The calls must agree on n_q, heads, head_dim, sel_stride,
+ * dtypes, stat_kind, k_next and whether statistics are written; stores must be quantised
+ * throughout (8-bit base, 2/4/8-bit residuals). ws: device workspace of
+ * fl_sparse_loop_attn_batched_workspace_bytes(n) bytes, receiving the calls' arguments
+ * (copied from host memory during the call, so the call is not meant for stream capture). */
+size_t fl_sparse_loop_attn_batched_workspace_bytes(int32_t n);
+fl_status fl_sparse_loop_attn_batched(const fl_attn_args* args, int32_t n, void* ws,
+                                      size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- *
  * The shared block on compact rows (§1: a shared N-layer block applied R times;

@@ -93,6 +93,41 @@ class LayerKV:
         self.slot[r][act_tok] = np.arange(len(act_tok), dtype=np.int32)
         self.hat[r] = hat
 
+    def append(self, r, tokens, k, v):
+        """Decode: add ``tokens`` (new positions) to loop r without touching the other
+        tokens. Loop 1 writes their base rows (row = token id); loop r >= 2 appends
+        residual rows (against each token's loop r-1 reconstruction) after the existing
+        rows. k, v float32 [n, H, hd]. The base arrays must already span the tokens."""
+        tokens = np.asarray(tokens, np.int64)
+        if r == 1:
+            bits = self.base_bits
+            for kv, x in enumerate((k, v)):
+                x = np.asarray(x, np.float32)
+                codes, sz, deq = self._encode(x, bits)
+                self.codes[(1, kv)][tokens] = codes
+                if sz is not None:
+                    self.sz[(1, kv)][tokens] = sz
+                self.hat[1][kv][tokens] = deq
+            return
+        bits = self.res_bits[r]
+        prev = self.hat[r - 1]
+        hat = self.hat[r]
+        row0 = len(self.rows[r])
+        for kv, x in enumerate((k, v)):
+            x = np.asarray(x, np.float32)
+            if bits == 0:
+                codes, sz, newv = x.copy(), None, x.copy()
+            else:
+                resid = (x - prev[kv][tokens]).astype(np.float32)
+                codes, sz, deq = self._encode(resid, bits)
+                newv = (prev[kv][tokens] + deq).astype(np.float32)
+            self.codes[(r, kv)] = np.concatenate([self.codes[(r, kv)], codes])
+            if sz is not None:
+                self.sz[(r, kv)] = np.concatenate([self.sz[(r, kv)], sz])
+            hat[kv][tokens] = newv
+        self.rows[r] = np.concatenate([self.rows[r], tokens.astype(np.int32)])
+        self.slot[r][tokens] = row0 + np.arange(len(tokens), dtype=np.int32)
+
     def carry(self, r):
         """A loop that writes nothing for this layer keeps the previous state."""
         self.hat[r] = self.hat[r - 1]

@@ -115,3 +115,32 @@ def test_c1_runs_and_is_reproducible():
     assert len(a["act"][2]) == 64
     b = loop.run(layers, h0, sched, cfg["n_heads"], cfg["head_dim"])
     assert np.array_equal(a["h"][4], b["h"][4])
+
+
+def test_append_equals_full_write():
+    """Decode append (§4.3 applied to a generated token): appending a token to loop r
+    gives it the same codes and reconstruction as writing loop r with the token among the
+    active set, and leaves every other token untouched."""
+    from oracle import kvstore
+    g = synth.rng(77)
+    n, H, hd = 40, 2, 64
+    base_k, base_v = synth.kv_values(g, n, H, hd), synth.kv_values(g, n, H, hd)
+    act = np.array([3, 9, 17], np.int32)
+    new = 39
+    rk = (base_k[act] + 0.1 * g.normal(size=(3, H, hd))).astype(np.float32)
+    rv = (base_v[act] + 0.1 * g.normal(size=(3, H, hd))).astype(np.float32)
+    tk = (base_k[[new]] + 0.1 * g.normal(size=(1, H, hd))).astype(np.float32)
+    tv = (base_v[[new]] + 0.1 * g.normal(size=(1, H, hd))).astype(np.float32)
+    a = kvstore.LayerKV(n, H, hd, 32, 8, {2: 4}, 2)
+    a.write_base(base_k, base_v)
+    a.write_residual(2, act, rk, rv)
+    a.append(2, [new], tk, tv)
+    b = kvstore.LayerKV(n, H, hd, 32, 8, {2: 4}, 2)
+    b.write_base(base_k, base_v)
+    b.write_residual(2, np.append(act, new), np.concatenate([rk, tk]), np.concatenate([rv, tv]))
+    for kv in range(2):
+        assert np.array_equal(a.codes[(2, kv)], b.codes[(2, kv)])
+        assert np.array_equal(a.hat[2][kv], b.hat[2][kv])
+    assert np.array_equal(a.slot, b.slot)
+    K, V = a.reconstruct(2, np.arange(n))
+    assert np.array_equal(K, a.hat[2][0]) and np.array_equal(V, a.hat[2][1])

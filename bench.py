@@ -409,12 +409,14 @@ def main():
         arm_hooks()
     for i in range(args.steps):
         restore(W)
+        torch.cuda.nvtx.range_push("timed_step")   # lets a profiler select the timed work
         starts[i].record(stream)
         if graph is not None:
             graph.replay()
         else:
             step_loops(W)
         ends[i].record(stream)
+        torch.cuda.nvtx.range_pop()
         if graph is not None:   # the graph re-records one step's kernel events per replay
             ends[i].synchronize()
             for kind in (0, 1):

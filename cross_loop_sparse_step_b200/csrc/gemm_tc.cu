@@ -15,6 +15,7 @@
 // in time; a wait that runs out records FL_ERR_TIMEOUT and the CTA drains its copies
 // in flight, frees TMEM and returns.
 #include <mutex>
+#include <stdlib.h>
 #include <unordered_map>
 
 #include "fl_internal.cuh"
@@ -346,6 +347,30 @@ cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, 
 
 }  // namespace
 
+// Tile width: 128 or 256 output columns. A 256-wide tile moves 48 KB per k-block for twice
+// the MACs of a 128-wide one (32 KB), so it costs between 1.5x (operand-bandwidth bound)
+// and 2x (tensor bound) as long; the persistent grid runs ceil(tiles / SMs) rounds.
+// The wider tile is taken when its rounds x cost are lower. FL_GEMM_BN=128|256 forces it.
+int pick_bn(int M, int n_cols, bool pairs) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("FL_GEMM_BN");
+    forced = e ? atoi(e) : 0;
+  }
+  // pairs (SwiGLU): a tile of width BN produces BN / 2 output columns
+  const int out128 = pairs ? 64 : 128, out256 = pairs ? 128 : 256;
+  if (n_cols % out256 != 0) return 128;
+  if (forced == 128 || forced == 256) return forced;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int mt = (M + BM - 1) / BM;
+  const long t128 = (long)mt * (n_cols / out128), t256 = (long)mt * (n_cols / out256);
+  const double c128 = (double)((t128 + sms - 1) / sms);
+  const double c256 = 1.75 * (double)((t256 + sms - 1) / sms);
+  return c256 < c128 ? 256 : 128;
+}
+
 bool gemm_tc_supported(int M, int N, int K) {
   return M >= 1 && K >= BK && K % BK == 0 && N % 128 == 0 && encode_fn() != nullptr;
 }
@@ -354,8 +379,12 @@ cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N,
                            GemmEpi epi, cudaStream_t s) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)C % 16 || ldc % 4)
     return cudaErrorInvalidValue;
-  if (epi == EPI_ADD) return launch_bn<128, 6, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s);
-  return launch_bn<128, 6, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s);
+  const bool wide = pick_bn(M, N, false) == 256;
+  if (epi == EPI_ADD)
+    return wide ? launch_bn<256, 4, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s)
+                : launch_bn<128, 6, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s);
+  return wide ? launch_bn<256, 4, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s)
+              : launch_bn<128, 6, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s);
 }
 
 bool gemm_swiglu_supported(int M, int F, int K) {
@@ -367,6 +396,9 @@ cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int
                                cudaStream_t s) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)Y % 16 || F % 64)
     return cudaErrorInvalidValue;
+  if (pick_bn(M, F, true) == 256)
+    return launch_bn<256, 4, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
+                                         2 * F, K, 0, s);
   return launch_bn<128, 6, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
                                        2 * F, K, 0, s);
 }
@@ -383,6 +415,8 @@ cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, fl
       (uintptr_t)v % 16)
     return cudaErrorInvalidValue;
   QkvOut qo{q, k, v, pos, rope, d, hd};
+  if (d % 256 == 0 && pick_bn(M, 3 * d, false) == 256)
+    return launch_bn<256, 4, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
   return launch_bn<128, 6, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
 }
 

@@ -354,7 +354,9 @@ cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, 
   // pageable source: the copy is staged before this call returns
   cudaError_t e = cudaMemcpyAsync(ws, host.data(), n * sizeof(AttnParams), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return e;
-  return launch_attn_sparse_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
+  int loop_max = 1;   // shared-memory slices sized for the deepest call
+  for (int i = 0; i < n; ++i) loop_max = host[i].loop > loop_max ? host[i].loop : loop_max;
+  return launch_attn_sparse_batched(host[0], static_cast<const AttnParams*>(ws), n, loop_max, s);
 }
 
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {

@@ -4,12 +4,18 @@
 // K/V of the selected columns are gathered, here straight from the quantised store).
 //
 // Used when the store is quantised throughout (int8 base, 2/4/8-bit residuals).
-//   Four lanes per column, eight columns in flight per warp; each lane owns a quarter
-//   of the head slice (one quantisation group at head_dim 128) and keeps its part of q
-//   in registers.
+//   Four lanes per column; each lane owns a quarter of the head slice (one quantisation
+//   group at head_dim 128) and keeps its part of q in registers. Every gather pass takes
+//   sixteen stored rows per warp iteration (two per lane group), both rows' loads issued
+//   before either is decoded, so each iteration waits for one round of L2 latency.
+//   Residual work lists: for the loops that rewrote some carried columns, the (column,
+//   loop, row) items are compacted once per loop chunk - slot lookups of several loops
+//   issued together - and the K and V passes walk them as one stream, so no lane idles
+//   on a column that a loop did not touch.
 //   K pass: every stored row of the column's chain (base, then each loop that rewrote
 //     it) contributes s * (q . codes) + z * sum(q) - dequantisation folded into the dot;
-//     codes are decoded in pairs and the dots use packed binary32 pair FMAs.
+//     codes are decoded in pairs and the dots use packed binary32 pair FMAs. The
+//     residual items' parts are added to the logits loop by loop, in loop order.
 //   softmax over the column set, p~ = m * softmax (m = cached mass).
 //   optional budget shrink: warp radix select over the binary32 bits of p~ * ||V^||
 //     (ties to the smaller column), ballot-ordered so the kept set stays ascending.
@@ -23,15 +29,31 @@
 namespace fl {
 namespace {
 
-constexpr int NW = 4;  // warps per CTA
+constexpr int NW = 4;              // warps per CTA
+// resident CTAs per SM the register budget is cut for (no spills at either setting)
+__host__ __device__ constexpr int min_ctas(bool shrink) { return shrink ? 3 : 5; }
+constexpr int ITEM_BYTES = 11;     // u16 column index + u8 loop + i32 row + f32 logit part
+constexpr int ITEM_BUDGET = 6144;  // per-warp bytes for residual items beyond one loop's
 
 __host__ __device__ inline size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
-// Per-warp shared memory: (reserved) [HD + 4] f32 | p [stride] f32 | cols [stride] u16 |
-// mark [stride] u8 | hist [256] i32 | list_idx [stride] u16 | list_row [stride] i32.
-__host__ __device__ inline size_t warp_smem(int hd, int stride) {
-  return align16((size_t)hd * 4 + 16) + align16((size_t)stride * 4) + align16((size_t)stride * 2) +
-         align16((size_t)stride) + 256 * 4 + align16((size_t)stride * 2) + align16((size_t)stride * 4);
+// Residual loops whose item lists are held at once (each loop's list needs up to `stride`
+// items); at least one.
+__host__ __device__ inline int chunk_loops(int loop, int stride) {
+  if (loop < 2) return 1;
+  int cl = ITEM_BUDGET / (stride * ITEM_BYTES);
+  if (cl < 1) cl = 1;
+  return cl < loop - 1 ? cl : loop - 1;
+}
+
+// Per-warp shared memory: p [stride] f32 | cols [stride] u16 | mark [stride] u8 |
+// hist [256] i32 | loff [FL_MAX_LOOPS + 1] i32 | items: it_part [cap] f32 | it_row [cap]
+// i32 | it_idx [cap] u16 | it_loop [cap] u8, cap = chunk_loops * stride.
+__host__ __device__ inline size_t warp_smem(int stride, int loop) {
+  const size_t cap = (size_t)chunk_loops(loop, stride) * stride;
+  return align16((size_t)stride * 4) + align16((size_t)stride * 2) + align16((size_t)stride) +
+         256 * 4 + align16((FL_MAX_LOOPS + 1) * 4) + 2 * align16(cap * 4) + align16(cap * 2) +
+         align16(cap);
 }
 
 __device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s, float* z) {
@@ -40,12 +62,107 @@ __device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s
   *z = half_bits_to_float((uint16_t)(pair >> 16));
 }
 
-// Four lanes per column: lane part l4 = lane % 4 owns elements [l4 * EL, (l4 + 1) * EL) of
-// the head slice, EL = HD / 4 (32 at HD 128), which lie in one quantisation group.
-// SHRINK: the call may shrink the budget (k_next below the carried set size), so the
-// dropped columns' contribution is accumulated too.
+// This lane's EL codes [e0, e0 + EL) of a stored row, as raw words (EL * bits / 8 bytes,
+// at most 32): loaded first, decoded later, so several rows' loads can be in flight.
+template <int EL>
+struct Raw {
+  uint4 w[EL / 16];
+};
+
+template <int EL>
+__device__ __forceinline__ void load_raw(const uint8_t* row, int bits, int e0, Raw<EL>& r) {
+  const uint8_t* src = row + (size_t)e0 * bits / 8;
+  if (bits == 8) {
+#pragma unroll
+    for (int k = 0; k < EL / 16; ++k) r.w[k] = reinterpret_cast<const uint4*>(src)[k];
+  } else if (bits == 4) {   // EL / 2 bytes
+    if constexpr (EL == 32) {
+      r.w[0] = *reinterpret_cast<const uint4*>(src);
+    } else {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
+    }
+  } else {                  // 2 bits: EL / 4 bytes
+    if constexpr (EL == 32) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
+    } else {
+      r.w[0] = make_uint4(*reinterpret_cast<const uint32_t*>(src), 0u, 0u, 0u);
+    }
+  }
+}
+
+template <int EL>
+__device__ __forceinline__ uint32_t raw_word(const Raw<EL>& r, int i) {
+  const uint4 u = r.w[i >> 2];
+  return (i & 3) == 0 ? u.x : (i & 3) == 1 ? u.y : (i & 3) == 2 ? u.z : u.w;
+}
+
+// sum_j q[j] * code[j] over the lane's EL elements (q held as EL/2 pairs)
+template <int EL>
+__device__ __forceinline__ float dot_raw(const float2* q, const Raw<EL>& r, int bits) {
+  float2 acc = make_float2(0.f, 0.f);
+  float2 c[8];
+  if (bits == 8) {
+#pragma unroll
+    for (int i = 0; i < EL / 4; ++i) {
+      f2::dec8(raw_word(r, i), c);
+      acc = f2::fma2(q[2 * i], c[0], acc);
+      acc = f2::fma2(q[2 * i + 1], c[1], acc);
+    }
+  } else if (bits == 4) {
+#pragma unroll
+    for (int i = 0; i < EL / 8; ++i) {
+      f2::dec4(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc = f2::fma2(q[4 * i + k], c[k], acc);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EL / 16; ++i) {
+      f2::dec2(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc = f2::fma2(q[8 * i + k], c[k], acc);
+    }
+  }
+  return acc.x + acc.y;
+}
+
+// o[j] += w * code[j]
+template <int EL>
+__device__ __forceinline__ void axpy_raw(float w, const Raw<EL>& r, int bits, float2* o) {
+  const float2 ww = make_float2(w, w);
+  float2 c[8];
+  if (bits == 8) {
+#pragma unroll
+    for (int i = 0; i < EL / 4; ++i) {
+      f2::dec8(raw_word(r, i), c);
+      o[2 * i] = f2::fma2(ww, c[0], o[2 * i]);
+      o[2 * i + 1] = f2::fma2(ww, c[1], o[2 * i + 1]);
+    }
+  } else if (bits == 4) {
+#pragma unroll
+    for (int i = 0; i < EL / 8; ++i) {
+      f2::dec4(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[4 * i + k] = f2::fma2(ww, c[k], o[4 * i + k]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EL / 16; ++i) {
+      f2::dec2(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[8 * i + k] = f2::fma2(ww, c[k], o[8 * i + k]);
+    }
+  }
+}
+
 // One warp's work: (query, head) number gw of the call described by P, with `base` the
 // warp's shared-memory slice. No CTA-wide barrier is used.
+// Lane part l4 = lane % 4 owns elements [l4 * EL, (l4 + 1) * EL) of the head slice,
+// EL = HD / 4, which lie in one quantisation group; lane group cg = lane / 4 (0..7).
+// SHRINK: the call may shrink the budget (k_next below the carried set size), so the
+// dropped columns' contribution is accumulated too.
 template <int HD, bool SHRINK>
 __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, uint8_t* base) {
   constexpr int EL = HD / 4;
@@ -53,15 +170,23 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   const int qi = gw / P.H, h = gw % P.H;
   const int H = P.H, n_tok = P.kv.n_tok, gs = P.kv.g, stride = P.sel_stride;
   const KvView& kv = P.kv;
-  const int l4 = lane & 3, cg = lane >> 2;   // part of the column, column group (0..7)
+  const int l4 = lane & 3, cg = lane >> 2;
   const int e0 = l4 * EL;
   const int gidx = e0 / gs;                  // quantisation group of this lane's part
   const int ngrp = HD / gs;
+  const int loop = P.loop;
+  const int CL = chunk_loops(loop, stride);
+  const int cap = CL * stride;
 
-  float* p = reinterpret_cast<float*>(base + align16((size_t)HD * 4 + 16));
-  uint16_t* cols = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p) + align16((size_t)stride * 4));
+  float* p = reinterpret_cast<float*>(base);
+  uint16_t* cols = reinterpret_cast<uint16_t*>(base + align16((size_t)stride * 4));
   uint8_t* mark = reinterpret_cast<uint8_t*>(cols) + align16((size_t)stride * 2);
   int* hist = reinterpret_cast<int*>(mark + align16((size_t)stride));
+  int* loff = hist + 256;
+  float* it_part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(loff) + align16((FL_MAX_LOOPS + 1) * 4));
+  int32_t* it_row = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(it_part) + align16((size_t)cap * 4));
+  uint16_t* it_idx = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(it_row) + align16((size_t)cap * 4));
+  uint8_t* it_loop = reinterpret_cast<uint8_t*>(it_idx) + align16((size_t)cap * 2);
 
   const int t = P.q_tok[qi];
   const int srow = P.q_row ? P.q_row[qi] : t;
@@ -93,9 +218,10 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     for (int k = 0; k < EL / 2; ++k) {
       float a, b;
       if (P.q_bf16) {
-        const __nv_bfloat16* qb = reinterpret_cast<const __nv_bfloat16*>(P.q) + off;
-        a = __bfloat162float(qb[2 * k]);
-        b = __bfloat162float(qb[2 * k + 1]);
+        const __nv_bfloat162 v = reinterpret_cast<const __nv_bfloat162*>(
+            reinterpret_cast<const __nv_bfloat16*>(P.q) + off)[k];
+        a = __low2float(v);
+        b = __high2float(v);
       } else {
         const float2 v = reinterpret_cast<const float2*>(reinterpret_cast<const float*>(P.q) + off)[k];
         a = v.x;
@@ -107,89 +233,151 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   }
   __syncwarp();
 
-  // Work is split so every lane stays busy: a base pass over all columns, then one pass
-  // per loop r = 2..loop over the compacted list of columns that loop rewrote.
-  uint16_t* list_idx = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(hist) + 256 * 4);
-  int32_t* list_row = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(list_idx) + align16((size_t)stride * 2));
-  // compacts {idx : slot[r][cols[idx]] >= 0} into list_idx / list_row; returns its length
-  auto build_list = [&](int r) -> int {
-    int n = 0;
-    const int32_t* srow_r = kv.slot + (size_t)r * n_tok;
+  // Residual items of loops [r0, r1): (column index, loop, row) for every carried column
+  // that loop rewrote, compacted loop after loop into it_*; loff[k] = first item of loop
+  // r0 + k. Each loop's items are first written to a region of `stride` entries (its
+  // count held by lane r - r0), the slot lookups of four loops issued together.
+  auto build_items = [&](int r0, int r1) -> int {
+    int cnt = 0;   // lane k: items of loop r0 + k so far
     for (int b0 = 0; b0 < n_cols; b0 += 32) {
       const int idx = b0 + lane;
-      int row = -1;
+      int c = -1;
       if (idx < n_cols) {
-        const int c = cols[idx];
-        if (c <= t && c < n_tok) row = srow_r[c];
+        c = cols[idx];
+        if (c > t || c >= n_tok) c = -1;
       }
-      const uint32_t bal = __ballot_sync(0xffffffffu, row >= 0);
-      if (row >= 0) {
-        const int pos = n + __popc(bal & ((1u << lane) - 1u));
-        list_idx[pos] = (uint16_t)idx;
-        list_row[pos] = row;
+      for (int ra = r0; ra < r1; ra += 4) {
+        int row[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          row[u] = (c >= 0 && ra + u < r1) ? kv.slot[(size_t)(ra + u) * n_tok + c] : -1;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = ra + u - r0;
+          if (ra + u >= r1) break;
+          const uint32_t bal = __ballot_sync(0xffffffffu, row[u] >= 0);
+          const int have = __shfl_sync(0xffffffffu, cnt, k);
+          if (row[u] >= 0) {
+            const int pos = k * stride + have + __popc(bal & ((1u << lane) - 1u));
+            it_idx[pos] = (uint16_t)idx;
+            it_row[pos] = row[u];
+          }
+          if (lane == k) cnt += __popc(bal);
+        }
       }
-      n += __popc(bal);
     }
+    // exclusive prefix of the counts over lanes 0..r1-r0-1
+    const int nl = r1 - r0;
+    int incl = lane < nl ? cnt : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - (lane < nl ? cnt : 0);
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (lane <= nl) loff[lane] = lane < nl ? excl : total;
     __syncwarp();
-    return n;
+    // move region k down to loff[k] (destinations never pass their sources)
+    for (int k = 0; k < nl; ++k) {
+      const int n_k = __shfl_sync(0xffffffffu, cnt, k);
+      const int dst0 = __shfl_sync(0xffffffffu, excl, k);
+      for (int j0 = 0; j0 < n_k; j0 += 32) {
+        const int j = j0 + lane;
+        uint16_t ix = 0;
+        int32_t rw = 0;
+        if (j < n_k) { ix = it_idx[k * stride + j]; rw = it_row[k * stride + j]; }
+        __syncwarp();
+        if (j < n_k) {
+          it_idx[dst0 + j] = ix;
+          it_row[dst0 + j] = rw;
+          it_loop[dst0 + j] = (uint8_t)(r0 + k);
+        }
+        __syncwarp();
+      }
+    }
+    return total;
   };
+  const bool one_chunk = loop < 2 || CL >= loop - 1;
+  int n_items = 0;   // items of the current chunk (all residual loops when one_chunk)
 
-  // ---- K base pass: 8 columns in flight, score part = s (q . codes) + z sum(q)
-  for (int i0 = 0; i0 < n_cols; i0 += 8) {
-    const int idx = i0 + cg;
-    float part = 0.f;
-    int c = -1;
-    bool valid = idx < n_cols;
-    if (valid) {
-      c = cols[idx];
-      valid = c <= t && c < n_tok;
+  // ---- K base pass: two columns per lane group, score part = s (q . codes) + z sum(q)
+  for (int i0 = 0; i0 < n_cols; i0 += 16) {
+    Raw<EL> raw[2];
+    float sb[2], zb[2], bias_c[2];
+    int idx[2];
+    bool valid[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      idx[u] = i0 + 8 * u + cg;
+      valid[u] = false;
+      bias_c[u] = 0.f;
+      if (idx[u] < n_cols) {
+        const int c = cols[idx[u]];
+        valid[u] = c <= t && c < n_tok;
+        if (valid[u]) {
+          if (P.bias && l4 == 0) bias_c[u] = P.bias[c];
+          const size_t bh = (size_t)c * H + h;
+          load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb[u], &zb[u]);
+          load_raw<EL>(kv.codes[0][1] + bh * HD, 8, e0, raw[u]);
+        }
+      }
     }
-    float bias_c = 0.f;
-    if (valid) {
-      if (P.bias && l4 == 0) bias_c = P.bias[c];
-      const size_t bh = (size_t)c * H + h;
-      float2 cf[EL / 2];
-      float sb, zb;
-      load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb, &zb);
-      f2::load_pairs<EL>(kv.codes[0][1] + bh * HD, 8, e0, cf);
-      const float d = f2::dot_pairs<EL>(qv, cf);
-      part = fmaf(sb, d, zb * qsum);
-    }
-    part += __shfl_xor_sync(0xffffffffu, part, 1);
-    part += __shfl_xor_sync(0xffffffffu, part, 2);
-    if (idx < n_cols && l4 == 0) {
-      if (!valid) {
-        record_error(P.st, FL_ERR_RANGE);
-        p[idx] = -INFINITY;
-      } else {
-        p[idx] = part * P.scale + bias_c;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float part = valid[u] ? fmaf(sb[u], dot_raw<EL>(qv, raw[u], 8), zb[u] * qsum) : 0.f;
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (idx[u] < n_cols && l4 == 0) {
+        if (!valid[u]) {
+          record_error(P.st, FL_ERR_RANGE);
+          p[idx[u]] = -INFINITY;
+        } else {
+          p[idx[u]] = part * P.scale + bias_c[u];
+        }
       }
     }
   }
   __syncwarp();
-  // ---- K residual passes
-  for (int r = 2; r <= P.loop; ++r) {
-    const int n_r = build_list(r);
-    const int b = kv.res_bits[r];
+
+  // ---- K residual passes: items of a chunk as one stream, parts added in loop order
+  for (int r0 = 2; r0 <= loop; r0 += CL) {
+    const int r1 = min(loop + 1, r0 + CL);
+    n_items = build_items(r0, r1);
     const float sc = P.scale;
-    for (int i0 = 0; i0 < n_r; i0 += 8) {
-      const int li = i0 + cg;
-      float part = 0.f;
-      if (li < n_r) {
-        const size_t rh = (size_t)list_row[li] * H + h;
-        float2 cf[EL / 2];
-        float sr, zr;
-        load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr, &zr);
-        f2::load_pairs<EL>(kv.codes[0][r] + rh * (HD * b / 8), b, e0, cf);
-        const float d = f2::dot_pairs<EL>(qv, cf);
-        part = fmaf(sr, d, zr * qsum);
+    for (int i0 = 0; i0 < n_items; i0 += 16) {
+      Raw<EL> raw[2];
+      float sr[2], zr[2];
+      int bits[2];
+      bool on[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = i0 + 8 * u + cg;
+        on[u] = it < n_items;
+        bits[u] = 8;
+        if (on[u]) {
+          const int r = it_loop[it];
+          bits[u] = kv.res_bits[r];
+          const size_t rh = (size_t)it_row[it] * H + h;
+          load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr[u], &zr[u]);
+          load_raw<EL>(kv.codes[0][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
+        }
       }
-      part += __shfl_xor_sync(0xffffffffu, part, 1);
-      part += __shfl_xor_sync(0xffffffffu, part, 2);
-      if (li < n_r && l4 == 0) p[list_idx[li]] += part * sc;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float part = on[u] ? fmaf(sr[u], dot_raw<EL>(qv, raw[u], bits[u]), zr[u] * qsum) : 0.f;
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if (on[u] && l4 == 0) it_part[i0 + 8 * u + cg] = part * sc;
+      }
     }
     __syncwarp();
+    for (int k = 0; k < r1 - r0; ++k) {   // loop order; a loop lists a column at most once
+      for (int x = loff[k] + lane; x < loff[k + 1]; x += 32) p[it_idx[x]] += it_part[x];
+      __syncwarp();
+    }
   }
+
   float lmax = -FLT_MAX;
   for (int idx = lane; idx < n_cols; idx += 32) lmax = fmaxf(lmax, p[idx]);
 #pragma unroll
@@ -259,51 +447,80 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     __syncwarp();
   }
 
+
   // ---- V passes: o part += (w s) codes + w z for every stored row of the chain
   float2 o[EL / 2], ua[EL / 2];
 #pragma unroll
   for (int k = 0; k < EL / 2; ++k) { o[k] = make_float2(0.f, 0.f); ua[k] = make_float2(0.f, 0.f); }
   float oz = 0.f, uz = 0.f;   // the offsets' share, added to every element at the end
-  for (int i0 = 0; i0 < n_cols; i0 += 8) {
-    const int idx = i0 + cg;
-    if (idx >= n_cols) continue;
-    const int c = cols[idx];
-    if (c > t || c >= n_tok) continue;
-    const float wgt = p[idx];
-    const size_t bh = (size_t)c * H + h;
-    float2 cf[EL / 2];
-    float s, z;
-    load_sz(kv.sz[1][1], bh * ngrp + gidx, &s, &z);
-    f2::load_pairs<EL>(kv.codes[1][1] + bh * HD, 8, e0, cf);
-    const float ws = wgt * s;
-    f2::axpy_pairs<EL>(ws, cf, o);
-    oz = fmaf(wgt, z, oz);
-    if (SHRINK && prune && !mark[idx]) {
-      f2::axpy_pairs<EL>(ws, cf, ua);
-      uz = fmaf(wgt, z, uz);
-    }
-  }
-  for (int r = 2; r <= P.loop; ++r) {
-    const int n_r = build_list(r);
-    const int b = kv.res_bits[r];
-    for (int i0 = 0; i0 < n_r; i0 += 8) {
-      const int li = i0 + cg;
-      if (li >= n_r) continue;
-      const int idx = list_idx[li];
-      const float wgt = p[idx];
-      const size_t rh = (size_t)list_row[li] * H + h;
-      float2 cf[EL / 2];
-      float s, z;
-      load_sz(kv.sz[1][r], rh * ngrp + gidx, &s, &z);
-      f2::load_pairs<EL>(kv.codes[1][r] + rh * (HD * b / 8), b, e0, cf);
-      const float ws = wgt * s;
-      f2::axpy_pairs<EL>(ws, cf, o);
-      oz = fmaf(wgt, z, oz);
-      if (SHRINK && prune && !mark[idx]) {
-        f2::axpy_pairs<EL>(ws, cf, ua);
-        uz = fmaf(wgt, z, uz);
+  for (int i0 = 0; i0 < n_cols; i0 += 16) {
+    Raw<EL> raw[2];
+    float s[2], z[2], wgt[2];
+    bool valid[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int idx = i0 + 8 * u + cg;
+      valid[u] = false;
+      if (idx < n_cols) {
+        const int c = cols[idx];
+        valid[u] = c <= t && c < n_tok;
+        if (valid[u]) {
+          wgt[u] = p[idx];
+          const size_t bh = (size_t)c * H + h;
+          load_sz(kv.sz[1][1], bh * ngrp + gidx, &s[u], &z[u]);
+          load_raw<EL>(kv.codes[1][1] + bh * HD, 8, e0, raw[u]);
+        }
       }
     }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (!valid[u]) continue;
+      const float ws = wgt[u] * s[u];
+      axpy_raw<EL>(ws, raw[u], 8, o);
+      oz = fmaf(wgt[u], z[u], oz);
+      if (SHRINK && prune && !mark[i0 + 8 * u + cg]) {
+        axpy_raw<EL>(ws, raw[u], 8, ua);
+        uz = fmaf(wgt[u], z[u], uz);
+      }
+    }
+  }
+  for (int r0 = 2; r0 <= loop; r0 += CL) {
+    const int r1 = min(loop + 1, r0 + CL);
+    if (!one_chunk) n_items = build_items(r0, r1);   // else still held from the K pass
+    for (int i0 = 0; i0 < n_items; i0 += 16) {
+      Raw<EL> raw[2];
+      float s[2], z[2], wgt[2];
+      int bits[2], idx[2];
+      bool on[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = i0 + 8 * u + cg;
+        on[u] = it < n_items;
+        bits[u] = 8;
+        idx[u] = 0;
+        if (on[u]) {
+          const int r = it_loop[it];
+          bits[u] = kv.res_bits[r];
+          idx[u] = it_idx[it];
+          wgt[u] = p[idx[u]];
+          const size_t rh = (size_t)it_row[it] * H + h;
+          load_sz(kv.sz[1][r], rh * ngrp + gidx, &s[u], &z[u]);
+          load_raw<EL>(kv.codes[1][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!on[u]) continue;
+        const float ws = wgt[u] * s[u];
+        axpy_raw<EL>(ws, raw[u], bits[u], o);
+        oz = fmaf(wgt[u], z[u], oz);
+        if (SHRINK && prune && !mark[idx[u]]) {
+          axpy_raw<EL>(ws, raw[u], bits[u], ua);
+          uz = fmaf(wgt[u], z[u], uz);
+        }
+      }
+    }
+    __syncwarp();
   }
   // reduce the 8 column groups (lanes with the same part differ in bits 2..4)
   const float2 oz2 = make_float2(oz, oz), uz2 = make_float2(uz, uz);
@@ -359,25 +576,28 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = prune ? lm : m_in;
 }
 
+
 template <int HD, bool SHRINK>
-__global__ void __launch_bounds__(NW * 32) k_attn_sparse(const __grid_constant__ AttnParams P) {
+__global__ void __launch_bounds__(NW * 32, min_ctas(SHRINK)) k_attn_sparse(const __grid_constant__ AttnParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int w = threadIdx.x >> 5;
   const int gw = blockIdx.x * NW + w;
   if (gw >= P.n_q * P.H) return;  // whole warp leaves
-  attn_sparse_warp<HD, SHRINK>(P, gw, smem + (size_t)w * warp_smem(HD, P.sel_stride));
+  attn_sparse_warp<HD, SHRINK>(P, gw, smem + (size_t)w * warp_smem(P.sel_stride, P.loop));
 }
 
 // Many independent calls in one launch (batched decode: one store per sequence). The
-// calls share n_q, heads, head_dim and carried-set stride; `per` = n_q * H warps each.
+// calls share n_q, heads, head_dim and carried-set stride; `per` = n_q * H warps each;
+// `loop` is the deepest call's loop (a warp's slice holds that call's layout).
 template <int HD, bool SHRINK>
-__global__ void __launch_bounds__(NW * 32)
-    k_attn_sparse_batched(const AttnParams* __restrict__ Ps, int n_calls, int per, int stride) {
+__global__ void __launch_bounds__(NW * 32, min_ctas(SHRINK))
+    k_attn_sparse_batched(const AttnParams* __restrict__ Ps, int n_calls, int per, int stride,
+                          int loop) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int w = threadIdx.x >> 5;
   const int gw = blockIdx.x * NW + w;
   if (gw >= n_calls * per) return;
-  attn_sparse_warp<HD, SHRINK>(Ps[gw / per], gw % per, smem + (size_t)w * warp_smem(HD, stride));
+  attn_sparse_warp<HD, SHRINK>(Ps[gw / per], gw % per, smem + (size_t)w * warp_smem(stride, loop));
 }
 
 }  // namespace
@@ -391,11 +611,11 @@ bool sparse_fast_eligible(const AttnParams& P) {
   }
   if (P.sel_stride < 1 || P.sel_stride > 4096) return false;
   if (P.sel_out && P.stat_kind == FL_STAT_PV && !P.vnorm) return false;
-  return (size_t)NW * warp_smem(P.hd, P.sel_stride) <= 200 * 1024;
+  return (size_t)NW * warp_smem(P.sel_stride, P.loop) <= 200 * 1024;
 }
 
 cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s) {
-  const size_t sm = (size_t)NW * warp_smem(P.hd, P.sel_stride);
+  const size_t sm = (size_t)NW * warp_smem(P.sel_stride, P.loop);
   const int warps = P.n_q * P.H;
   const int blocks = (warps + NW - 1) / NW;
   const bool shrink = P.sel_out != nullptr && P.k_next + 1 < P.sel_stride;
@@ -416,10 +636,11 @@ cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// Ps: device array of n AttnParams (already copied by the caller, same shapes).
+// Ps: device array of n AttnParams (already copied by the caller, same shapes; loops up
+// to loop_max, which sizes every warp's shared-memory slice).
 cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
-                                       cudaStream_t s) {
-  const size_t sm = (size_t)NW * warp_smem(P0.hd, P0.sel_stride);
+                                       int loop_max, cudaStream_t s) {
+  const size_t sm = (size_t)NW * warp_smem(P0.sel_stride, loop_max);
   const int per = P0.n_q * P0.H;
   const long long warps = (long long)per * n;
   const int blocks = (int)((warps + NW - 1) / NW);
@@ -436,7 +657,7 @@ cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* P
     if (e != cudaSuccess) return e;
     have = (int)sm;
   }
-  kern<<<blocks, NW * 32, sm, s>>>(Ps_dev, n, per, P0.sel_stride);
+  kern<<<blocks, NW * 32, sm, s>>>(Ps_dev, n, per, P0.sel_stride, loop_max);
   count_launch();
   return cudaGetLastError();
 }

@@ -22,7 +22,7 @@ cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int
 bool gemm_qkv_supported(int M, int d, int hd);
 cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
                             const int32_t* pos, const float2* rope, int M, int d, int hd,
-                            cudaStream_t s);
+                            cudaStream_t s, const fl_kv_desc* fuse = nullptr, int loop = 0);
 
 int* status_word() {
   static int* cache[128] = {nullptr};
@@ -168,8 +168,24 @@ fl_status prepare_rope(const fl_model* m, void* ws, cudaStream_t s) {
   return FL_OK;
 }
 
+// The store update of `loop` can ride in the QKV epilogue: bf16 projections, group 32,
+// an 8-bit base and 2/4/8-bit residual loops up to `loop`.
+bool kv_fusable(const fl_model* m, int n, const fl_kv_desc* kv, int loop) {
+  if (!kv || !qkv_fused(m, n) || kv->group != 32 || kv->base_bits != 8) return false;
+  if (kv->n_heads != m->n_heads || kv->head_dim != m->head_dim || loop < 1 || loop > kv->n_loops)
+    return false;
+  for (int r = 2; r <= loop; ++r) {
+    const int b = kv->res_bits[r];
+    if (b != 2 && b != 4 && b != 8) return false;
+  }
+  return true;
+}
+
+// RMSNorm, QKV projection, RoPE; with `fuse` the KV store update of `loop` happens in the
+// projection's epilogue (k, v may then be null).
 fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int32_t* pos,
-                  float* q, float* k, float* v, void* ws, cudaStream_t s) {
+                  float* q, float* k, float* v, void* ws, cudaStream_t s,
+                  const fl_kv_desc* fuse = nullptr, int loop = 0) {
   const fl_layer_weights& w = m->layers[layer];
   const int d = m->d_model;
   const float2* rope = static_cast<const float2*>(ws);
@@ -177,8 +193,11 @@ fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int
   void* a = c.take((size_t)n * d * dt_size(m->dt));
   FL_TRY(launch_rmsnorm(x, w.g_attn, m->rms_eps, a, m->dt, n, d, s));
   if (qkv_fused(m, n)) {
+    if (fuse && loop >= 2)
+      FL_TRY(launch_fill_i32(fuse->slot + (size_t)loop * fuse->n_tok, -1, (size_t)fuse->n_tok, s));
+    if (fuse && loop == 1 && fuse->slot) FL_TRY(launch_iota(fuse->slot + fuse->n_tok, fuse->n_tok, s));
     timing_begin(TIMED_GEMM, s);
-    cudaError_t e = launch_gemm_qkv(a, w.w_qkv, q, k, v, pos, rope, n, d, m->head_dim, s);
+    cudaError_t e = launch_gemm_qkv(a, w.w_qkv, q, k, v, pos, rope, n, d, m->head_dim, s, fuse, loop);
     timing_end(TIMED_GEMM, s);
     FL_TRY(e);
     return FL_OK;
@@ -427,6 +446,28 @@ fl_status fl_block_qkv(const fl_model* m, int32_t layer, const float* x, int32_t
   return run_qkv(m, layer, x, n_rows, pos, q, k, v, ws, S(stream));
 }
 
+fl_status fl_block_qkv_kv(const fl_model* m, int32_t layer, const fl_kv_desc* kv, int32_t loop,
+                          const float* x, int32_t n_rows, const int32_t* pos, float* q,
+                          float* k_out, float* v_out, void* ws, size_t ws_bytes, void* stream) {
+  fl_status st = check_model(m);
+  if (st != FL_OK) return st;
+  st = check_kv(kv);
+  if (st != FL_OK) return st;
+  FL_CHECK(layer >= 0 && layer < m->n_layers && n_rows >= 0, FL_ERR_SHAPE);
+  FL_CHECK(kv->n_tok == m->n_tok, FL_ERR_SHAPE);
+  if (n_rows == 0) return FL_OK;
+  FL_CHECK(x && pos && q, FL_ERR_INVALID_ARG);
+  FL_CHECK(loop != 1 || n_rows == kv->n_tok, FL_ERR_SHAPE);
+  FL_CHECK(kv_fusable(m, n_rows, kv, loop), FL_ERR_UNSUPPORTED);
+  for (int r = 1; r <= loop; ++r) {
+    FL_CHECK(kv->codes[0][r] && kv->codes[1][r] && kv->sz[0][r] && kv->sz[1][r], FL_ERR_INVALID_ARG);
+  }
+  FL_CHECK(ws && ws_bytes >= block_ws(m, n_rows), FL_ERR_WORKSPACE);
+  fl_status rc = prepare_rope(m, ws, S(stream));
+  if (rc != FL_OK) return rc;
+  return run_qkv(m, layer, x, n_rows, pos, q, k_out, v_out, ws, S(stream), kv, loop);
+}
+
 fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n_rows,
                            const void* attn, void* ws, size_t ws_bytes, void* stream) {
   fl_status st = check_model(m);
@@ -541,9 +582,19 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
   rc = prepare_rope(m, blk, s);
   if (rc != FL_OK) return rc;
   for (int l = 0; l < L; ++l) {
-    rc = run_qkv(m, l, X, M, act, q, k, v, blk, s);
-    if (rc != FL_OK) return rc;
-    FL_TRY(launch_kv_quant(st->kv[l], loop, k, v, FL_F32, loop == 1 ? nullptr : act, M, sw, s));
+    // Loop 1 writes the base codes in the projection epilogue. Later loops quantise the
+    // residual against K^_{r-1}, whose chain decode is a string of dependent gathers; in
+    // the four epilogue warps of the GEMM those stall the tensor pipe (measured: the fused
+    // QKV launch took 2.1x the projection plus the separate quantiser), so they keep the
+    // separate, wider quantiser launch.
+    if (loop == 1 && kv_fusable(m, M, &st->kv[l], loop)) {
+      rc = run_qkv(m, l, X, M, act, q, nullptr, nullptr, blk, s, &st->kv[l], loop);
+      if (rc != FL_OK) return rc;
+    } else {
+      rc = run_qkv(m, l, X, M, act, q, k, v, blk, s);
+      if (rc != FL_OK) return rc;
+      FL_TRY(launch_kv_quant(st->kv[l], loop, k, v, FL_F32, loop == 1 ? nullptr : act, M, sw, s));
+    }
     fl_attn_args a;
     memset(&a, 0, sizeof(a));
     a.q = q; a.q_dt = FL_F32; a.n_q = M; a.q_tok = act;

@@ -128,7 +128,7 @@ struct AttnParams {
 bool sparse_fast_eligible(const AttnParams& P);
 cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s);
 cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
-                                       cudaStream_t s);
+                                       int loop_max, cudaStream_t s);
 AttnParams make_attn_params(const fl_attn_args& a, int* st);
 size_t attention_batched_ws_bytes(int n);
 cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, int* st,

@@ -20,6 +20,7 @@
 
 #include "fl_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "kv_epilogue.cuh"
 
 namespace fl {
 namespace {
@@ -39,10 +40,12 @@ constexpr int EPI_SWIGLU = 2;
 constexpr int EPI_QKV = 3;
 
 struct QkvOut {
-  float* q; float* k; float* v;
+  float* q; float* k; float* v;   // k, v may be null when the store update is fused
   const int32_t* pos;
   const float2* rope;
   int d, hd;
+  KvFuse kf;                      // fused KV quantisation of k and v (kf.on)
+  KvView kv;                      // the store read for the residual's reference
 };
 
 // Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
@@ -52,7 +55,7 @@ template <int BN, int STAGES, int EPI>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
               float* __restrict__ C, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int ldc,
-              int half, const QkvOut qo, int* st) {
+              int half, const __grid_constant__ QkvOut qo, int* st) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -181,39 +184,62 @@ __global__ void __launch_bounds__(192, 1)
         const int n0 = nt * BN;
         const int which = n0 / qo.d, col0 = n0 % qo.d;
         float* out = which == 0 ? qo.q : (which == 1 ? qo.k : qo.v);
+        const bool quant = qo.kf.on && which >= 1;
         const int hh = qo.hd / 2;
         const int prow = row < M ? qo.pos[row] : 0;
+        float vss = 0.f;   // ||V^||^2 of the current head (fused V tiles)
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           const int off = (c * 32) % qo.hd;   // offset inside the head
+          const int head = (col0 + c * 32) / qo.hd;
           if (which < 2 && off >= hh) continue;  // second halves go with their partners
           float a[32];
           tmem_ld32(t_base + (uint32_t)(c * 32), a);
           if (which == 2) {
             if (row < M) {
-              float4* dst = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
+              if (out) {
+                float4* dst = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
 #pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                for (int q = 0; q < 8; ++q)
+                  dst[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+              }
+              if (quant) {
+                vss += fuse_group(qo.kv, qo.kf, 1, a, row, prow, head, off, st);
+                if (off + 32 == qo.hd && qo.kf.vnorm)
+                  qo.kf.vnorm[(size_t)prow * qo.kv.H + head] = sqrtf(vss);
+              }
             }
+            if (off + 32 == qo.hd) vss = 0.f;
             continue;
           }
           float b[32];
           tmem_ld32(t_base + (uint32_t)(c * 32 + hh), b);
           if (row < M) {
-            // (cos, sin) of 4 consecutive angles = 2 float4; 16-byte loads and stores
+            // rotate: (a, b) -> (a cos - b sin, a sin + b cos); (cos, sin) of 4 angles = 2 float4
             const float4* cs = reinterpret_cast<const float4*>(qo.rope + (size_t)prow * hh + off);
-            float4* dx = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
-            float4* dy = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32 + hh);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
               const float4 r01 = cs[2 * q], r23 = cs[2 * q + 1];
-              const float* x = a + 4 * q;
-              const float* y = b + 4 * q;
-              dx[q] = make_float4(x[0] * r01.x - y[0] * r01.y, x[1] * r01.z - y[1] * r01.w,
-                                  x[2] * r23.x - y[2] * r23.y, x[3] * r23.z - y[3] * r23.w);
-              dy[q] = make_float4(x[0] * r01.y + y[0] * r01.x, x[1] * r01.w + y[1] * r01.z,
-                                  x[2] * r23.y + y[2] * r23.x, x[3] * r23.w + y[3] * r23.z);
+              const float cr[4] = {r01.x, r01.z, r23.x, r23.z}, sr[4] = {r01.y, r01.w, r23.y, r23.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float x = a[4 * q + e], y = b[4 * q + e];
+                a[4 * q + e] = x * cr[e] - y * sr[e];
+                b[4 * q + e] = x * sr[e] + y * cr[e];
+              }
+            }
+            if (out) {
+              float4* dx = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32);
+              float4* dy = reinterpret_cast<float4*>(out + (size_t)row * qo.d + col0 + c * 32 + hh);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                dx[q] = make_float4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+                dy[q] = make_float4(b[4 * q], b[4 * q + 1], b[4 * q + 2], b[4 * q + 3]);
+              }
+            }
+            if (quant) {
+              fuse_group(qo.kv, qo.kf, 0, a, row, prow, head, off, st);
+              fuse_group(qo.kv, qo.kf, 0, b, row, prow, head, off + hh, st);
             }
           }
         }
@@ -410,11 +436,21 @@ bool gemm_qkv_supported(int M, int d, int hd) {
 // q, k, v [M x d] fp32 = split(A . w_qkv^T), q and k rotated by RoPE (table `rope`).
 cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
                             const int32_t* pos, const float2* rope, int M, int d, int hd,
-                            cudaStream_t s) {
+                            cudaStream_t s, const fl_kv_desc* fuse, int loop) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)q % 16 || (uintptr_t)k % 16 ||
       (uintptr_t)v % 16)
     return cudaErrorInvalidValue;
-  QkvOut qo{q, k, v, pos, rope, d, hd};
+  QkvOut qo{};
+  qo.q = q; qo.k = k; qo.v = v; qo.pos = pos; qo.rope = rope; qo.d = d; qo.hd = hd;
+  qo.kf.on = 0;
+  if (fuse) {
+    qo.kv = make_view(*fuse);
+    qo.kf.on = 1;
+    qo.kf.loop = loop;
+    for (int w = 0; w < 2; ++w) { qo.kf.codes[w] = fuse->codes[w][loop]; qo.kf.sz[w] = fuse->sz[w][loop]; }
+    qo.kf.slot_row = loop >= 2 ? fuse->slot + (size_t)loop * fuse->n_tok : nullptr;
+    qo.kf.vnorm = fuse->vnorm;
+  }
   if (d % 256 == 0 && pick_bn(M, 3 * d, false) == 256)
     return launch_bn<256, 4, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
   return launch_bn<128, 6, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);

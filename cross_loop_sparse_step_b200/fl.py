@@ -108,6 +108,9 @@ _attn = _sig("fl_sparse_loop_attn", c_i32, [ctypes.POINTER(AttnArgs), vp])
 _blk_ws = _sig("fl_block_workspace_bytes", c_sz, [ctypes.POINTER(Model), c_i32])
 _blk_qkv = _sig("fl_block_qkv", c_i32,
                 [ctypes.POINTER(Model), c_i32, vp, c_i32, vp, vp, vp, vp, vp, c_sz, vp])
+_blk_qkv_kv = _sig("fl_block_qkv_kv", c_i32,
+                   [ctypes.POINTER(Model), c_i32, ctypes.POINTER(KvDesc), c_i32, vp, c_i32, vp,
+                    vp, vp, vp, vp, c_sz, vp])
 _blk_ffn = _sig("fl_block_out_ffn", c_i32,
                 [ctypes.POINTER(Model), c_i32, vp, c_i32, vp, vp, c_sz, vp])
 _loop_ws = _sig("fl_loop_step_workspace_bytes", c_sz,
@@ -315,6 +318,13 @@ class LoopModel:
 def block_qkv(model, layer, x, pos, q, k, v, ws, stream=None):
     _ok(_blk_qkv(ctypes.byref(model.c), layer, ptr(x), x.shape[0], ptr(pos), ptr(q), ptr(k),
                  ptr(v), ptr(ws), ws.numel(), stream_handle(stream)), "fl_block_qkv")
+
+
+def block_qkv_kv(model, layer, store, loop, x, pos, q, ws, k=None, v=None, stream=None):
+    """block_qkv with loop `loop`'s KV store update done in the projection epilogue."""
+    _ok(_blk_qkv_kv(ctypes.byref(model.c), layer, ctypes.byref(store.desc), loop, ptr(x),
+                    x.shape[0], ptr(pos), ptr(q), ptr(k), ptr(v), ptr(ws), ws.numel(),
+                    stream_handle(stream)), "fl_block_qkv_kv")
 
 
 def block_out_ffn(model, layer, x, attn, ws, stream=None):

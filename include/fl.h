@@ -269,6 +269,16 @@ size_t fl_block_workspace_bytes(const fl_model* m, int32_t n_rows);
 fl_status fl_block_qkv(const fl_model* m, int32_t layer, const float* x, int32_t n_rows,
                        const int32_t* pos, float* q, float* k, float* v,
                        void* ws, size_t ws_bytes, void* stream);
+/* fl_block_qkv with the KV store update of loop `loop` (fl_kv_residual_quant's
+ * computation, bit for bit) done in the projection's epilogue - the fusion of the
+ * cross-loop KV update and quantisation with the projection that §4.4 describes.
+ * The rows' tokens are pos[i] (loop 1: every token, in order; loop >= 2: ascending,
+ * residual row i), and slot[loop] is rewritten. k_out / v_out (nullable) also receive
+ * the post-RoPE k and v. Needs bf16 weights, group 32, an 8-bit base and 2/4/8-bit
+ * residual loops (otherwise FL_ERR_UNSUPPORTED). Workspace: fl_block_workspace_bytes. */
+fl_status fl_block_qkv_kv(const fl_model* m, int32_t layer, const fl_kv_desc* kv, int32_t loop,
+                          const float* x, int32_t n_rows, const int32_t* pos, float* q,
+                          float* k_out, float* v_out, void* ws, size_t ws_bytes, void* stream);
 /* x += attn W_o^T, then the SwiGLU FFN with residual, in place on x (device float
  * [n][d]); attn is device [n][d] of dtype m->dt. */
 fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n_rows,

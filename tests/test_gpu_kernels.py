@@ -378,3 +378,68 @@ def test_block_qkv_and_out_ffn(_lib, n, d, H, hd, F, dt):
     _status_ok(fl)
     want = oblk.out_ffn(X, attn, w)
     assert_close(host(x), want, what="x")
+
+
+# ------------------------------------------- KV update fused into the projection
+FUSED_CASES = [
+    # n_tok, d, H, hd, F, residual bits, active rows per loop
+    (4096, 2048, 16, 128, 5632, {2: 4, 3: 4}, {2: 820, 3: 656}),   # the 4K workload's layer
+    (1000, 256, 4, 64, 512, {2: 2, 3: 8}, {2: 333, 3: 1}),          # ragged, one-row tail
+    (129, 512, 4, 128, 512, {2: 8, 3: 2}, {2: 129, 3: 64}),          # every token active
+]
+
+
+@pytest.mark.parametrize("n_tok,d,H,hd,F,rb,na", FUSED_CASES)
+def test_block_qkv_fused_kv_update_bit_exact(_lib, n_tok, d, H, hd, F, rb, na):
+    """Codes, scale/offset pairs and slots written by the projection epilogue equal the
+    oracle store's for the k and v the same call returns; q, k, v match the oracle."""
+    fl = _lib
+    rs = synth.rng(n_tok + d + hd)
+    w, wt = _weights(rs, d, F, True)
+    model = fl.LoopModel([wt], n_tok, H, hd)
+    R = 3
+    ost = okv.LayerKV(n_tok, H, hd, 32, 8, rb, R)
+    store = fl.KVStore(n_tok, H, hd, 32, 8, rb, R, na)
+    ws = torch.empty(model.block_ws_bytes(n_tok), dtype=torch.uint8, device="cuda")
+    act = np.arange(n_tok, dtype=np.int32)
+    for r in range(1, R + 1):
+        if r >= 2:
+            act = np.sort(rs.choice(act, size=na[r], replace=False)).astype(np.int32)
+        X = synth.embeddings(rs, len(act), d)
+        q = torch.zeros(len(act), H, hd, device="cuda")
+        k, v = torch.zeros_like(q), torch.zeros_like(q)
+        fl.block_qkv_kv(model, 0, store, r, dev(X), dev(act), q, ws, k=k, v=v)
+        _status_ok(fl)
+        qo, ko, vo = oblk.qkv(X, act, w, H, hd)
+        assert_close(host(q), qo, what=f"q loop {r}")
+        assert_close(host(k), ko, what=f"k loop {r}")
+        assert_close(host(v), vo, what=f"v loop {r}")
+        kh, vh = host(k), host(v)
+        if r == 1:
+            ost.write_base(kh, vh)
+        else:
+            ost.write_residual(r, act, kh, vh)
+        rows = len(act)
+        for kv in range(2):
+            want = np.ascontiguousarray(ost.codes[(r, kv)]).view(np.uint8).reshape(rows, H, -1)
+            assert np.array_equal(host(store.codes[(r, kv)])[:rows], want), (r, kv, "codes")
+            assert np.array_equal(host(store.sz[(r, kv)])[:rows].view(np.uint16),
+                                  ost.sz[(r, kv)].view(np.uint16)), (r, kv, "scale/offset")
+        assert np.array_equal(host(store.slot)[1:r + 1], ost.slot[1:r + 1]), (r, "slots")
+        vn = np.sqrt((ost.hat[r][1].astype(np.float64) ** 2).sum(-1))
+        assert_close(host(store.vnorm), vn, max_abs=1e-4, rel_l1=1e-6, what=f"vnorm loop {r}")
+    assert not ost.range_error
+
+
+def test_block_qkv_fused_rejects_unsupported_store(_lib):
+    """A store the epilogue cannot write (group 64) is refused, not silently split."""
+    fl = _lib
+    rs = synth.rng(7)
+    w, wt = _weights(rs, 256, 512, True)
+    model = fl.LoopModel([wt], 64, 2, 128)
+    store = fl.KVStore(64, 2, 128, 64, 8, {2: 4}, 2, {2: 8})
+    ws = torch.empty(model.block_ws_bytes(64), dtype=torch.uint8, device="cuda")
+    q = torch.zeros(64, 2, 128, device="cuda")
+    with pytest.raises(fl.FLError, match="unsupported"):
+        fl.block_qkv_kv(model, 0, store, 1, dev(synth.embeddings(rs, 64, 256)),
+                        dev(np.arange(64, dtype=np.int32)), q, ws)

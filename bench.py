@@ -443,6 +443,17 @@ def main():
     gemm_s = sum(kern_ms[0]) / 1e3
     gemm_tflops = gemm_flops_per_step(W) * args.steps / gemm_s / 1e12
     peak_t = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    # the four projections of a layer are recorded in order: QKV, O, gate/up, down
+    d_, F_ = W["d"], W["F"]
+    proj = {"qkv": 3 * d_ * d_, "o": d_ * d_, "gate_up": 2 * F_ * d_, "down": F_ * d_}
+    rows_per_launch = [W["n_active"][r] for r in range(2, R + 1) for _ in range(W["L"])]
+    per_gemm = {}
+    for j, (name, macs_per_row) in enumerate(proj.items()):
+        ms = kern_ms[0][j::4]
+        rows = (rows_per_launch * args.steps)[:len(ms)]
+        per_gemm[name] = {"avg_us": round(sum(ms) / len(ms) * 1e3, 2),
+                          "tflops": round(sum(2 * macs_per_row * n for n in rows)
+                                          / (sum(ms) / 1e3) / 1e12, 1)}
     attn_ms = kern_ms[1]
     abytes = attention_bytes_per_launch(W, torch)
     per_loop_launch = W["L"] * args.steps
@@ -502,7 +513,8 @@ def main():
                          "achieved": gemm_tflops, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": gemm_tflops / peak_t, "traffic": None,
                          "peak_source": f"{pk_kind} bf16 sustained",
-                         "share_of_step": gemm_s * 1e3 / step_total_ms},
+                         "share_of_step": gemm_s * 1e3 / step_total_ms,
+                         "per_gemm": per_gemm},
             "attention_roofline": {"bound": "hbm", "kernel": "k_attention (sparse, carried mass)",
                                    "achieved": attn_gbs, "peak": peak_h, "unit": "GB/s",
                                    "frac": attn_gbs / peak_h,

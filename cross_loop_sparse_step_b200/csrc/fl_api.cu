@@ -14,15 +14,16 @@ namespace fl {
 cudaError_t launch_gemm_simt(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
                              int K, int ldc, GemmEpi epi, cudaStream_t s);
 cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N, int K,
-                           int ldc, GemmEpi epi, cudaStream_t s);
+                           int ldc, GemmEpi epi, cudaStream_t s, const GemmScratch* scr);
 bool gemm_tc_supported(int M, int N, int K);
 bool gemm_swiglu_supported(int M, int F, int K);
 cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int F, int K,
-                               cudaStream_t s);
+                               cudaStream_t s, const GemmScratch* scr);
 bool gemm_qkv_supported(int M, int d, int hd);
 cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
                             const int32_t* pos, const float2* rope, int M, int d, int hd,
-                            cudaStream_t s, const fl_kv_desc* fuse = nullptr, int loop = 0);
+                            cudaStream_t s, const fl_kv_desc* fuse, int loop,
+                            const GemmScratch* scr);
 
 int* status_word() {
   static int* cache[128] = {nullptr};
@@ -66,11 +67,11 @@ void timing_end(int kind, cudaStream_t s) {
 }
 
 cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
-                        int K, int ldc, GemmEpi epi, cudaStream_t s) {
+                        int K, int ldc, GemmEpi epi, cudaStream_t s, const GemmScratch* scr) {
   timing_begin(TIMED_GEMM, s);
   cudaError_t e;
   if (dt == FL_BF16 && gemm_tc_supported(M, N, K))
-    e = launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s);
+    e = launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s, scr);
   else
     e = launch_gemm_simt(dt, A, W, C, M, N, K, ldc, epi, s);
   timing_end(TIMED_GEMM, s);
@@ -146,25 +147,37 @@ fl_status check_model(const fl_model* m) {
   return FL_OK;
 }
 
-// Block workspace: [RoPE (cos, sin) table of every position][scratch of one half-layer].
+// Block workspace: [RoPE (cos, sin) table of every position][GEMM stream-K scratch]
+// [scratch of one half-layer].
 size_t rope_tab_bytes(const fl_model* m) {
   return align_up((size_t)m->n_tok * (m->head_dim / 2) * sizeof(float2));
+}
+
+size_t block_head_bytes(const fl_model* m) {
+  return rope_tab_bytes(m) + align_up(gemm_scratch_bytes());
+}
+
+GemmScratch block_scratch(const fl_model* m, void* ws) {
+  return gemm_scratch_at(static_cast<uint8_t*>(ws) + rope_tab_bytes(m));
 }
 
 size_t block_ws(const fl_model* m, int n) {
   const size_t d = m->d_model, F = m->d_ffn, e = dt_size(m->dt);
   const size_t qkv_path = align_up(n * d * e) + align_up(n * 3 * d * 4);
   const size_t ffn_path = align_up(n * d * e) + align_up(n * 2 * F * 4) + align_up(n * F * e);
-  return rope_tab_bytes(m) + (qkv_path > ffn_path ? qkv_path : ffn_path);
+  return block_head_bytes(m) + (qkv_path > ffn_path ? qkv_path : ffn_path);
 }
 
 bool qkv_fused(const fl_model* m, int n) {
   return m->dt == FL_BF16 && gemm_qkv_supported(n, m->d_model, m->head_dim);
 }
 
-// Fills the RoPE table at the head of the block workspace (once per call or loop step).
+// Fills the RoPE table at the head of the block workspace and clears the GEMM hand-over
+// flags (once per call or loop step).
 fl_status prepare_rope(const fl_model* m, void* ws, cudaStream_t s) {
   FL_TRY(launch_rope_table(static_cast<float2*>(ws), m->n_tok, m->head_dim, m->rope_theta, s));
+  FL_TRY(cudaMemsetAsync(static_cast<uint8_t*>(ws) + rope_tab_bytes(m), 0,
+                         gemm_scratch_flag_bytes(), s));
   return FL_OK;
 }
 
@@ -189,7 +202,8 @@ fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int
   const fl_layer_weights& w = m->layers[layer];
   const int d = m->d_model;
   const float2* rope = static_cast<const float2*>(ws);
-  Carver c(static_cast<uint8_t*>(ws) + rope_tab_bytes(m));
+  const GemmScratch scr = block_scratch(m, ws);
+  Carver c(static_cast<uint8_t*>(ws) + block_head_bytes(m));
   void* a = c.take((size_t)n * d * dt_size(m->dt));
   FL_TRY(launch_rmsnorm(x, w.g_attn, m->rms_eps, a, m->dt, n, d, s));
   if (qkv_fused(m, n)) {
@@ -197,13 +211,14 @@ fl_status run_qkv(const fl_model* m, int layer, const float* x, int n, const int
       FL_TRY(launch_fill_i32(fuse->slot + (size_t)loop * fuse->n_tok, -1, (size_t)fuse->n_tok, s));
     if (fuse && loop == 1 && fuse->slot) FL_TRY(launch_iota(fuse->slot + fuse->n_tok, fuse->n_tok, s));
     timing_begin(TIMED_GEMM, s);
-    cudaError_t e = launch_gemm_qkv(a, w.w_qkv, q, k, v, pos, rope, n, d, m->head_dim, s, fuse, loop);
+    cudaError_t e =
+        launch_gemm_qkv(a, w.w_qkv, q, k, v, pos, rope, n, d, m->head_dim, s, fuse, loop, &scr);
     timing_end(TIMED_GEMM, s);
     FL_TRY(e);
     return FL_OK;
   }
   float* qkv = (float*)c.take((size_t)n * 3 * d * 4);
-  FL_TRY(launch_gemm(m->dt, a, w.w_qkv, qkv, n, 3 * d, d, 3 * d, EPI_STORE, s));
+  FL_TRY(launch_gemm(m->dt, a, w.w_qkv, qkv, n, 3 * d, d, 3 * d, EPI_STORE, s, &scr));
   FL_TRY(launch_rope_split(qkv, pos, n, m->n_heads, m->head_dim, m->rope_theta, q, k, v, s));
   return FL_OK;
 }
@@ -212,22 +227,23 @@ fl_status run_out_ffn(const fl_model* m, int layer, float* x, int n, const void*
                       cudaStream_t s) {
   const fl_layer_weights& w = m->layers[layer];
   const int d = m->d_model, F = m->d_ffn;
-  Carver c(static_cast<uint8_t*>(ws) + rope_tab_bytes(m));
+  const GemmScratch scr = block_scratch(m, ws);
+  Carver c(static_cast<uint8_t*>(ws) + block_head_bytes(m));
   void* a = c.take((size_t)n * d * dt_size(m->dt));
   float* gu = (float*)c.take((size_t)n * 2 * F * 4);
   void* mid = c.take((size_t)n * F * dt_size(m->dt));
-  FL_TRY(launch_gemm(m->dt, attn, w.w_o, x, n, d, d, d, EPI_ADD, s));
+  FL_TRY(launch_gemm(m->dt, attn, w.w_o, x, n, d, d, d, EPI_ADD, s, &scr));
   FL_TRY(launch_rmsnorm(x, w.g_ffn, m->rms_eps, a, m->dt, n, d, s));
   if (m->dt == FL_BF16 && gemm_swiglu_supported(n, F, d)) {
     timing_begin(TIMED_GEMM, s);
-    cudaError_t e = launch_gemm_swiglu(a, w.w_gate_up, mid, n, F, d, s);
+    cudaError_t e = launch_gemm_swiglu(a, w.w_gate_up, mid, n, F, d, s, &scr);
     timing_end(TIMED_GEMM, s);
     FL_TRY(e);
   } else {
-    FL_TRY(launch_gemm(m->dt, a, w.w_gate_up, gu, n, 2 * F, d, 2 * F, EPI_STORE, s));
+    FL_TRY(launch_gemm(m->dt, a, w.w_gate_up, gu, n, 2 * F, d, 2 * F, EPI_STORE, s, &scr));
     FL_TRY(launch_swiglu(gu, n, F, mid, m->dt, s));
   }
-  FL_TRY(launch_gemm(m->dt, mid, w.w_down, x, n, d, F, d, EPI_ADD, s));
+  FL_TRY(launch_gemm(m->dt, mid, w.w_down, x, n, d, F, d, EPI_ADD, s, &scr));
   return FL_OK;
 }
 
@@ -476,6 +492,8 @@ fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n
   if (n_rows == 0) return FL_OK;
   FL_CHECK(x && attn, FL_ERR_INVALID_ARG);
   FL_CHECK(ws && ws_bytes >= block_ws(m, n_rows), FL_ERR_WORKSPACE);
+  FL_TRY(cudaMemsetAsync(static_cast<uint8_t*>(ws) + rope_tab_bytes(m), 0,
+                         gemm_scratch_flag_bytes(), S(stream)));
   return run_out_ffn(m, layer, x, n_rows, attn, ws, S(stream));
 }
 

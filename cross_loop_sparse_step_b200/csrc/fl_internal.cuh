@@ -167,10 +167,21 @@ cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s);
 size_t attention_ws_bytes(const fl_attn_args& a);
 
+// Scratch of the tensor-core GEMM's stream-K split: hand-over flags (zero before the first
+// launch that uses them; every launch leaves them at zero) and partial accumulator tiles.
+struct GemmScratch {
+  int* flag; int n_flag;
+  float* part; size_t part_bytes;
+};
+size_t gemm_scratch_bytes();            // for the current device
+GemmScratch gemm_scratch_at(void* p);   // the layout of gemm_scratch_bytes() bytes at p
+size_t gemm_scratch_flag_bytes();       // the leading flag block (to zero)
+
 // C[M x N] (binary32, leading dim ldc) = or += A[M x K] . W[N x K]^T
 enum GemmEpi { EPI_STORE = 0, EPI_ADD = 1 };
 cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
-                        int K, int ldc, GemmEpi epi, cudaStream_t s);
+                        int K, int ldc, GemmEpi epi, cudaStream_t s,
+                        const GemmScratch* scr = nullptr);
 cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* out,
                            fl_dtype dt, int M, int d, cudaStream_t s);
 cudaError_t launch_rope_split(const float* qkv, const int32_t* pos, int M, int H, int hd,

@@ -38,6 +38,8 @@ constexpr int EPI_SWIGLU = 2;
 // it to q / k / v [M x d] (fp32), rotating q and k by RoPE at position pos[row] with the
 // (cos, sin) table rope[pos][i], i < hd/2 (rotate-half pairs (i, i + hd/2)).
 constexpr int EPI_QKV = 3;
+// EPI_QKV_KV: EPI_QKV plus the KV store update of k and v in the epilogue (qo.kf).
+constexpr int EPI_QKV_KV = 4;
 
 struct QkvOut {
   float* q; float* k; float* v;   // k, v may be null when the store update is fused
@@ -48,14 +50,67 @@ struct QkvOut {
   KvView kv;                      // the store read for the residual's reference
 };
 
-// Persistent: one CTA per SM walks the tiles blockIdx.x, blockIdx.x + gridDim.x, ...
-// (M-tile fastest, so the CTAs running together share each weight tile through L2).
-// Two TMEM accumulators: the epilogue drains tile i while the MMA warp fills tile i+1.
-template <int BN, int STAGES, int EPI>
+// Stream-K split (when the tiles do not fill whole rounds of the grid): the tiles x
+// k-blocks units are cut into gridDim.x equal contiguous ranges, one per CTA. A tile cut
+// between CTAs is finished by its owner (the CTA holding its k-block 0, which reaches it
+// last in its range); each other CTA holding a piece of it (its first segment) stores the
+// fp32 partial accumulator to part[cta] and raises flag[cta]. The owner waits for those
+// flags, adds the partials in CTA order (a fixed summation order: results do not depend
+// on timing) and runs the epilogue; it lowers the flags again for the next launch.
+struct SkPlan {
+  int on;
+  float* part;   // [gridDim.x][BM * BN] float4-interleaved partial tiles
+  int* flag;     // [gridDim.x], all zero at launch
+};
+
+// Work segment: k-blocks [kb0, kb1) of tile `tile`.
+struct Seg {
+  int tile, kb0, kb1;
+};
+
+__device__ __forceinline__ long long sk_begin(long long units, int cta, int grid) {
+  return units * cta / grid;
+}
+
+// Walks one CTA's segments: whole tiles blockIdx.x, +gridDim.x, ... without stream-K;
+// otherwise its unit range cut at tile boundaries.
+struct SegWalk {
+  long long cur, end;
+  int nk, tiles, sk;
+  __device__ SegWalk(bool on, int nk_, int tiles_) : nk(nk_), tiles(tiles_), sk(on) {
+    if (sk) {
+      const long long units = (long long)tiles * nk;
+      cur = sk_begin(units, blockIdx.x, gridDim.x);
+      end = sk_begin(units, blockIdx.x + 1, gridDim.x);
+    } else {
+      cur = blockIdx.x;
+      end = tiles;
+    }
+  }
+  __device__ bool next(Seg& g) {
+    if (cur >= end) return false;
+    if (!sk) {
+      g.tile = (int)cur; g.kb0 = 0; g.kb1 = nk;
+      cur += gridDim.x;
+      return true;
+    }
+    g.tile = (int)(cur / nk);
+    g.kb0 = (int)(cur % nk);
+    const long long left = end - cur;
+    g.kb1 = left < (long long)(nk - g.kb0) ? g.kb0 + (int)left : nk;
+    cur += g.kb1 - g.kb0;
+    return true;
+  }
+};
+
+// Persistent: one CTA per SM walks its segments (M-tile fastest, so the CTAs running
+// together share each weight tile through L2).
+// Two TMEM accumulators: the epilogue drains segment i while the MMA warp fills i+1.
+template <int BN, int STAGES, int EPI, bool SK>
 __global__ void __launch_bounds__(192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
               float* __restrict__ C, __nv_bfloat16* __restrict__ Y, int M, int N, int K, int ldc,
-              int half, const __grid_constant__ QkvOut qo, int* st) {
+              int half, const __grid_constant__ QkvOut qo, const SkPlan sk, int* st) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
@@ -91,11 +146,13 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      int g = 0;  // k-blocks issued over all tiles
-      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x) {
-        const int m0 = (tile % m_tiles) * BM;
-        const int nt = tile / m_tiles;
-        for (int kb = 0; kb < nk; ++kb, ++g) {
+      int g = 0;  // k-blocks issued over all segments
+      SegWalk walk(SK, nk, tiles);
+      Seg sg;
+      while (!*abort && walk.next(sg)) {
+        const int m0 = (sg.tile % m_tiles) * BM;
+        const int nt = sg.tile / m_tiles;
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++g) {
           const int s = g % STAGES, i = g / STAGES;
           if (i > 0 && !mbar_wait(&empty_bar[s], (i - 1) & 1, abort)) break;
           uint8_t* a_dst = smem + s * STAGE_BYTES;
@@ -122,13 +179,15 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(BM, BN);
       int g = 0, lt = 0;
-      for (int tile = blockIdx.x; tile < tiles && !*abort; tile += gridDim.x, ++lt) {
+      SegWalk walk(SK, nk, tiles);
+      Seg sg;
+      for (; !*abort && walk.next(sg); ++lt) {
         const int a = lt & 1, j = lt >> 1;
         if (lt >= 2 && !mbar_wait(&acce_bar[a], (j - 1) & 1, abort)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * BN);
         bool ok = true;
-        for (int kb = 0; kb < nk; ++kb, ++g) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++g) {
           const int s = g % STAGES, i = g / STAGES;
           if (!mbar_wait(&full_bar[s], i & 1, abort)) { ok = false; break; }
           tc_fence_after();
@@ -137,7 +196,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             mma_bf16(d_tmem, desc_sw128_kmajor(a_base + kk * 32),
-                     desc_sw128_kmajor(b_base + kk * 32), idesc, (kb | kk) != 0 ? 1u : 0u);
+                     desc_sw128_kmajor(b_base + kk * 32), idesc,
+                     (kb > sg.kb0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&empty_bar[s]);
         }
@@ -148,21 +208,67 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     const int ew = warp & 3;  // TMEM lanes [32 ew, 32 ew + 32) belong to this warp
+    const int lrow = ew * 32 + lane;
     int lt = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+    SegWalk walk(SK, nk, tiles);
+    Seg sg;
+    for (; walk.next(sg); ++lt) {
       const int a = lt & 1, j = lt >> 1;
       if (!mbar_wait(&accf_bar[a], j & 1, abort)) break;
       tc_fence_after();
-      const int row = (tile % m_tiles) * BM + ew * 32 + lane;
+      const int tile = sg.tile;
+      const int row = (tile % m_tiles) * BM + lrow;
       const int nt = tile / m_tiles;
       const uint32_t t_base = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(a * BN);
+      if (SK && sg.kb0 > 0) {
+        // a piece of a tile owned by an earlier CTA: park the partial, hand the rows over
+        float4* dst = reinterpret_cast<float4*>(sk.part + (size_t)blockIdx.x * (BM * BN));
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(t_base + (uint32_t)(c * 32), v);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[(c * 8 + q) * BM + lrow] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&acce_bar[a]);
+          flag_release(&sk.flag[blockIdx.x * 4 + ew]);
+        }
+        continue;
+      }
+      // owner of a cut tile: the pieces of CTAs blockIdx.x + 1 .. j_end - 1 are added
+      int j_end = blockIdx.x + 1;
+      if (SK && sg.kb1 < nk) {
+        const long long units = (long long)tiles * nk, tile_end = (long long)(tile + 1) * nk;
+        while (j_end < (int)gridDim.x && sk_begin(units, j_end, gridDim.x) < tile_end) ++j_end;
+        if (lane == 0) {
+          for (int jj = blockIdx.x + 1; jj < j_end; ++jj)
+            if (!flag_acquire_reset(&sk.flag[jj * 4 + ew])) { record_error(st, FL_ERR_TIMEOUT); *abort = 1; }
+        }
+        __syncwarp();
+      }
+      // accumulator columns [col, col + 32) of this thread's row, pieces included
+      auto ld_acc = [&](int col, float* v) {
+        tmem_ld32(t_base + (uint32_t)col, v);
+        for (int jj = blockIdx.x + 1; SK && jj < j_end; ++jj) {
+          const float4* src = reinterpret_cast<const float4*>(sk.part + (size_t)jj * (BM * BN));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 pv = __ldcg(src + ((col / 32) * 8 + q) * BM + lrow);
+            v[4 * q] += pv.x; v[4 * q + 1] += pv.y; v[4 * q + 2] += pv.z; v[4 * q + 3] += pv.w;
+          }
+        }
+      };
       if constexpr (EPI == EPI_SWIGLU) {
         const int f0 = nt * (BN / 2);
 #pragma unroll 1
         for (int c = 0; c < BN / 64; ++c) {
           float gv[32], uv[32];
-          tmem_ld32(t_base + (uint32_t)(c * 32), gv);
-          tmem_ld32(t_base + (uint32_t)(BN / 2 + c * 32), uv);
+          ld_acc(c * 32, gv);
+          ld_acc(BN / 2 + c * 32, uv);
           if (row < M) {
             uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * half + f0 + c * 32);
 #pragma unroll
@@ -180,11 +286,11 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
-      } else if constexpr (EPI == EPI_QKV) {
+      } else if constexpr (EPI == EPI_QKV || EPI == EPI_QKV_KV) {
         const int n0 = nt * BN;
         const int which = n0 / qo.d, col0 = n0 % qo.d;
         float* out = which == 0 ? qo.q : (which == 1 ? qo.k : qo.v);
-        const bool quant = qo.kf.on && which >= 1;
+        const bool quant = EPI == EPI_QKV_KV && which >= 1;
         const int hh = qo.hd / 2;
         const int prow = row < M ? qo.pos[row] : 0;
         float vss = 0.f;   // ||V^||^2 of the current head (fused V tiles)
@@ -194,7 +300,7 @@ __global__ void __launch_bounds__(192, 1)
           const int head = (col0 + c * 32) / qo.hd;
           if (which < 2 && off >= hh) continue;  // second halves go with their partners
           float a[32];
-          tmem_ld32(t_base + (uint32_t)(c * 32), a);
+          ld_acc(c * 32, a);
           if (which == 2) {
             if (row < M) {
               if (out) {
@@ -213,7 +319,7 @@ __global__ void __launch_bounds__(192, 1)
             continue;
           }
           float b[32];
-          tmem_ld32(t_base + (uint32_t)(c * 32 + hh), b);
+          ld_acc(c * 32 + hh, b);
           if (row < M) {
             // rotate: (a, b) -> (a cos - b sin, a sin + b cos); (cos, sin) of 4 angles = 2 float4
             const float4* cs = reinterpret_cast<const float4*>(qo.rope + (size_t)prow * hh + off);
@@ -248,7 +354,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           float v[32];
-          tmem_ld32(t_base + (uint32_t)(c * 32), v);
+          ld_acc(c * 32, v);
           if (row < M) {
             float4* dst = reinterpret_cast<float4*>(C + (size_t)row * ldc + n0 + c * 32);
 #pragma unroll
@@ -344,29 +450,72 @@ bool get_map(const void* p, int rows, int cols, int box_rows, CUtensorMap* out) 
   return true;
 }
 
+int sm_count() {
+  static int sms[128] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return 148;
+  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
+  return sms[dev] > 0 ? sms[dev] : 148;
+}
+
+// Stream-K unless switched off (FL_GEMM_SK=0).
+bool sk_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("FL_GEMM_SK");
+    on = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return on == 1;
+}
+
+constexpr int SK_MAX_GRID = 1024;
+
+// Stream-K is taken for 256-wide tiles that do not fill whole rounds of the grid and
+// give every CTA at least 64 k-blocks: below that the partial hand-over and the owner's
+// longer last epilogue cost more than the balance gains (measured on the projection
+// shapes of 820 active rows: a win for the gate/up GEMM at 67 k-blocks per CTA, losses
+// for QKV at 36, down at 33 and O at 12).
+bool use_sk(int tiles, int nk, int bn) {
+  const int sms = sm_count();
+  const long long units = (long long)tiles * nk;
+  return sk_enabled() && bn == 256 && tiles % sms != 0 && units >= 64LL * sms;
+}
+
 template <int BN, int STAGES, int EPI>
 cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, int M, int N,
-                      int K, int ldc, cudaStream_t s, QkvOut qo = QkvOut{}) {
+                      int K, int ldc, cudaStream_t s, const GemmScratch* scr,
+                      QkvOut qo = QkvOut{}) {
   CUtensorMap ma, mb;
   const int box_b = EPI == EPI_SWIGLU ? BN / 2 : BN;
   if (!get_map(A, M, K, BM, &ma) || !get_map(W, N, K, box_b, &mb)) return cudaErrorInvalidValue;
   const size_t smem = (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
-  auto kern = k_gemm_tc<BN, STAGES, EPI>;
+  auto kern_dp = k_gemm_tc<BN, STAGES, EPI, false>;
+  auto kern_sk = k_gemm_tc<BN, STAGES, EPI, true>;
   static bool attr_set[128] = {false};   // per device; set on the first (uncaptured) call
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kern_dp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern_sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
   const int tiles_n = EPI == EPI_SWIGLU ? (N / 2) / (BN / 2) : N / BN;
   const int tiles = tiles_n * ((M + BM - 1) / BM);
-  static int sms[128] = {0};
-  if (!sms[dev]) cudaDeviceGetAttribute(&sms[dev], cudaDevAttrMultiProcessorCount, dev);
-  const int grid = tiles < sms[dev] ? tiles : sms[dev];
-  kern<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, status_word());
+  const int sms = sm_count();
+  int grid = tiles < sms ? tiles : sms;
+  SkPlan plan{0, nullptr, nullptr};
+  if (use_sk(tiles, K / BK, BN) && scr && scr->flag && scr->part && sms * 4 <= scr->n_flag &&
+      (size_t)sms * BM * BN * 4 <= scr->part_bytes) {
+    grid = sms;
+    plan = SkPlan{1, scr->part, scr->flag};
+    kern_sk<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, plan, status_word());
+  } else {
+    kern_dp<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, plan, status_word());
+  }
   count_launch();
   return cudaGetLastError();
 }
@@ -377,7 +526,7 @@ cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, 
 // the MACs of a 128-wide one (32 KB), so it costs between 1.5x (operand-bandwidth bound)
 // and 2x (tensor bound) as long; the persistent grid runs ceil(tiles / SMs) rounds.
 // The wider tile is taken when its rounds x cost are lower. FL_GEMM_BN=128|256 forces it.
-int pick_bn(int M, int n_cols, bool pairs) {
+int pick_bn(int M, int n_cols, bool pairs, int K, bool sk) {
   static int forced = -1;
   if (forced < 0) {
     const char* e = getenv("FL_GEMM_BN");
@@ -387,14 +536,30 @@ int pick_bn(int M, int n_cols, bool pairs) {
   const int out128 = pairs ? 64 : 128, out256 = pairs ? 128 : 256;
   if (n_cols % out256 != 0) return 128;
   if (forced == 128 || forced == 256) return forced;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = sm_count();
   const int mt = (M + BM - 1) / BM;
   const long t128 = (long)mt * (n_cols / out128), t256 = (long)mt * (n_cols / out256);
+  // stream-K (balanced to a k-block) runs with 256-wide tiles
+  if (sk && use_sk((int)t256, K / BK, 256)) return 256;
   const double c128 = (double)((t128 + sms - 1) / sms);
   const double c256 = 1.75 * (double)((t256 + sms - 1) / sms);
   return c256 < c128 ? 256 : 128;
+}
+
+// Stream-K scratch: SK_MAX_GRID x 4 flags, then one 128 x 256 fp32 partial tile per SM.
+size_t gemm_scratch_flag_bytes() { return (size_t)SK_MAX_GRID * 4 * sizeof(int); }
+
+size_t gemm_scratch_bytes() {
+  return gemm_scratch_flag_bytes() + (size_t)sm_count() * BM * 256 * sizeof(float);
+}
+
+GemmScratch gemm_scratch_at(void* p) {
+  GemmScratch g;
+  g.flag = static_cast<int*>(p);
+  g.n_flag = SK_MAX_GRID * 4;
+  g.part = reinterpret_cast<float*>(static_cast<uint8_t*>(p) + gemm_scratch_flag_bytes());
+  g.part_bytes = gemm_scratch_bytes() - gemm_scratch_flag_bytes();
+  return g;
 }
 
 bool gemm_tc_supported(int M, int N, int K) {
@@ -402,15 +567,15 @@ bool gemm_tc_supported(int M, int N, int K) {
 }
 
 cudaError_t launch_gemm_tc(const void* A, const void* W, float* C, int M, int N, int K, int ldc,
-                           GemmEpi epi, cudaStream_t s) {
+                           GemmEpi epi, cudaStream_t s, const GemmScratch* scr) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)C % 16 || ldc % 4)
     return cudaErrorInvalidValue;
-  const bool wide = pick_bn(M, N, false) == 256;
+  const bool wide = pick_bn(M, N, false, K, scr != nullptr) == 256;
   if (epi == EPI_ADD)
-    return wide ? launch_bn<256, 4, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s)
-                : launch_bn<128, 6, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s);
-  return wide ? launch_bn<256, 4, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s)
-              : launch_bn<128, 6, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s);
+    return wide ? launch_bn<256, 4, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s, scr)
+                : launch_bn<128, 6, EPI_ADD>(A, W, C, nullptr, M, N, K, ldc, s, scr);
+  return wide ? launch_bn<256, 4, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s, scr)
+              : launch_bn<128, 6, EPI_STORE>(A, W, C, nullptr, M, N, K, ldc, s, scr);
 }
 
 bool gemm_swiglu_supported(int M, int F, int K) {
@@ -419,14 +584,14 @@ bool gemm_swiglu_supported(int M, int F, int K) {
 
 // Y[M x F] bf16 = silu(A . W_gate^T) * (A . W_up^T), W = [gate; up] of [2F x K].
 cudaError_t launch_gemm_swiglu(const void* A, const void* W, void* Y, int M, int F, int K,
-                               cudaStream_t s) {
+                               cudaStream_t s, const GemmScratch* scr) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)Y % 16 || F % 64)
     return cudaErrorInvalidValue;
-  if (pick_bn(M, F, true) == 256)
+  if (pick_bn(M, F, true, K, scr != nullptr) == 256)
     return launch_bn<256, 4, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
-                                         2 * F, K, 0, s);
+                                         2 * F, K, 0, s, scr);
   return launch_bn<128, 6, EPI_SWIGLU>(A, W, nullptr, reinterpret_cast<__nv_bfloat16*>(Y), M,
-                                       2 * F, K, 0, s);
+                                       2 * F, K, 0, s, scr);
 }
 
 bool gemm_qkv_supported(int M, int d, int hd) {
@@ -436,7 +601,8 @@ bool gemm_qkv_supported(int M, int d, int hd) {
 // q, k, v [M x d] fp32 = split(A . w_qkv^T), q and k rotated by RoPE (table `rope`).
 cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, float* v,
                             const int32_t* pos, const float2* rope, int M, int d, int hd,
-                            cudaStream_t s, const fl_kv_desc* fuse, int loop) {
+                            cudaStream_t s, const fl_kv_desc* fuse, int loop,
+                            const GemmScratch* scr) {
   if ((uintptr_t)A % 16 || (uintptr_t)W % 16 || (uintptr_t)q % 16 || (uintptr_t)k % 16 ||
       (uintptr_t)v % 16)
     return cudaErrorInvalidValue;
@@ -451,9 +617,11 @@ cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, fl
     qo.kf.slot_row = loop >= 2 ? fuse->slot + (size_t)loop * fuse->n_tok : nullptr;
     qo.kf.vnorm = fuse->vnorm;
   }
-  if (d % 256 == 0 && pick_bn(M, 3 * d, false) == 256)
-    return launch_bn<256, 4, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
-  return launch_bn<128, 6, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, qo);
+  if (d % 256 == 0 && pick_bn(M, 3 * d, false, d, scr != nullptr) == 256)
+    return fuse ? launch_bn<256, 4, EPI_QKV_KV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, scr, qo)
+                : launch_bn<256, 4, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, scr, qo);
+  return fuse ? launch_bn<128, 6, EPI_QKV_KV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, scr, qo)
+              : launch_bn<128, 6, EPI_QKV>(A, W, nullptr, nullptr, M, 3 * d, d, 0, s, scr, qo);
 }
 
 }  // namespace fl

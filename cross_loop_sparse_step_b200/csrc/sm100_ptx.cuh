@@ -68,6 +68,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // 2-D tiled TMA load into shared memory, completion counted on `bar` (bytes).
+// Cross-CTA hand-over of data in global memory: the writer's stores (ordered before
+// this call by __syncwarp) become visible before the flag does.
+__device__ __forceinline__ void flag_release(int* flag) {
+  asm volatile("fence.acq_rel.gpu;\n\tst.relaxed.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1)
+               : "memory");
+}
+// Waits (bounded) until *flag is 1, then lowers it to 0; false on timeout.
+__device__ __forceinline__ bool flag_acquire_reset(int* flag) {
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    if (v == 1) break;
+    if (globaltimer() - t0 > kWaitLimitNs) return false;
+  }
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(0) : "memory");
+  return true;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int x, int y) {
   asm volatile(

@@ -341,6 +341,8 @@ BLOCK_CASES = [
     (128, 256, 2, 128, 512, "bf16"),     # exactly one tile
     (129, 256, 2, 128, 512, "bf16"),     # one row into the next tile
     (4096, 2048, 16, 128, 5632, "bf16"), # every token (loop 1)
+    (820, 2048, 16, 128, 5632, "bf16"),  # active rows: tiles cut between CTAs (stream-K)
+    (300, 1024, 8, 128, 1536, "bf16"),   # ragged rows, three tile rows cut across CTAs
 ]
 
 

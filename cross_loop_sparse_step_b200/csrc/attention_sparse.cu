@@ -4,27 +4,31 @@
 // K/V of the selected columns are gathered, here straight from the quantised store).
 //
 // Used when the store is quantised throughout (int8 base, 2/4/8-bit residuals).
-//   Four lanes per column; each lane owns a quarter of the head slice (one quantisation
-//   group at head_dim 128) and keeps its part of q in registers. Every gather pass takes
-//   sixteen stored rows per warp iteration (two per lane group), both rows' loads issued
-//   before either is decoded, so each iteration waits for one round of L2 latency.
+//   The products run on the tensor cores (warp-level m16n8k16 MMAs, binary32
+//   accumulation) with exact operands: codes as the fp16 values c * 2^-24, and q and the
+//   softmax weights as hi + lo fp16 pairs after a power-of-two scaling (22 significant
+//   bits; see attn_mma.cuh). Dequantisation stays folded: a stored row contributes
+//   s * (q . codes) + z * sum(q) to a logit and (p~ s) codes + p~ z to the output.
+//   Every pass takes sixteen stored rows per warp iteration, their loads issued before
+//   any is used, so each iteration waits for one round of L2 latency.
 //   Residual work lists: for the loops that rewrote some carried columns, the (column,
 //   loop, row) items are compacted once per loop chunk - slot lookups of several loops
 //   issued together - and the K and V passes walk them as one stream, so no lane idles
 //   on a column that a loop did not touch.
-//   K pass: every stored row of the column's chain (base, then each loop that rewrote
-//     it) contributes s * (q . codes) + z * sum(q) - dequantisation folded into the dot;
-//     codes are decoded in pairs and the dots use packed binary32 pair FMAs. The
-//     residual items' parts are added to the logits loop by loop, in loop order.
+//   K pass (rows = 16 stored rows, k = head elements, n = hi/lo of each quarter of q):
+//     lane (g, l) holds quarter l of rows g and g + 8 and gets back its quarter's dot
+//     for both; the scale/offset of the quarter's group are applied and the quarters
+//     summed by shuffles. Residual parts are added to the logits loop by loop.
 //   softmax over the column set, p~ = m * softmax (m = cached mass).
 //   optional budget shrink: warp radix select over the binary32 bits of p~ * ||V^||
 //     (ties to the smaller column), ballot-ordered so the kept set stays ascending.
-//   V pass: o += (p~ s) codes + p~ z over the chain's rows, and for dropped columns the
-//     same into the next loop's u'; the eight column groups are reduced by shuffles.
+//   V pass (rows = head elements, k = 16 stored rows, n = hi/lo of the weights of each
+//     quarter): o = sum (p~ s) codes + sum p~ z, and for dropped columns the same into
+//     the next loop's u'. Lane (g, g / 2) ends up with elements [g hd/8, (g+1) hd/8).
 #include <float.h>
 
 #include "fl_internal.cuh"
-#include "sm100_f32x2.cuh"
+#include "attn_mma.cuh"
 
 namespace fl {
 namespace {
@@ -98,62 +102,49 @@ __device__ __forceinline__ uint32_t raw_word(const Raw<EL>& r, int i) {
   return (i & 3) == 0 ? u.x : (i & 3) == 1 ? u.y : (i & 3) == 2 ? u.z : u.w;
 }
 
-// sum_j q[j] * code[j] over the lane's EL elements (q held as EL/2 pairs)
+// This lane's EL codes as one code per byte (EL / 4 words), from raw words of `bits` bits.
 template <int EL>
-__device__ __forceinline__ float dot_raw(const float2* q, const Raw<EL>& r, int bits) {
-  float2 acc = make_float2(0.f, 0.f);
-  float2 c[8];
+__device__ __forceinline__ void to_bytes(const Raw<EL>& r, int bits, uint32_t* wb) {
   if (bits == 8) {
 #pragma unroll
-    for (int i = 0; i < EL / 4; ++i) {
-      f2::dec8(raw_word(r, i), c);
-      acc = f2::fma2(q[2 * i], c[0], acc);
-      acc = f2::fma2(q[2 * i + 1], c[1], acc);
-    }
+    for (int i = 0; i < EL / 4; ++i) wb[i] = raw_word(r, i);
   } else if (bits == 4) {
 #pragma unroll
-    for (int i = 0; i < EL / 8; ++i) {
-      f2::dec4(raw_word(r, i), c);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) acc = f2::fma2(q[4 * i + k], c[k], acc);
-    }
+    for (int i = 0; i < EL / 8; ++i) mma::spread4(raw_word(r, i), wb + 2 * i);
   } else {
 #pragma unroll
-    for (int i = 0; i < EL / 16; ++i) {
-      f2::dec2(raw_word(r, i), c);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc = f2::fma2(q[8 * i + k], c[k], acc);
-    }
+    for (int i = 0; i < EL / 16; ++i) mma::spread2(raw_word(r, i), wb + 4 * i);
   }
-  return acc.x + acc.y;
 }
 
-// o[j] += w * code[j]
-template <int EL>
-__device__ __forceinline__ void axpy_raw(float w, const Raw<EL>& r, int bits, float2* o) {
-  const float2 ww = make_float2(w, w);
-  float2 c[8];
+// Chunk [CE cg, CE cg + CE) of a stored row (CE = hd / 8 codes) as raw words.
+template <int CE>
+__device__ __forceinline__ uint4 load_chunk(const uint8_t* row, int bits, int cg) {
+  const uint8_t* src = row + (size_t)CE * cg * bits / 8;
+  const int bytes = CE * bits / 8;   // 16, 8, 4 or 2
+  if (bytes == 16) return *reinterpret_cast<const uint4*>(src);
+  if (bytes == 8) {
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    return make_uint4(u.x, u.y, 0u, 0u);
+  }
+  if (bytes == 4) return make_uint4(*reinterpret_cast<const uint32_t*>(src), 0u, 0u, 0u);
+  return make_uint4((uint32_t)*reinterpret_cast<const uint16_t*>(src), 0u, 0u, 0u);
+}
+
+// The chunk as one code per byte: CE / 4 words.
+template <int CE>
+__device__ __forceinline__ void chunk_bytes(uint4 u, int bits, uint32_t* wb) {
   if (bits == 8) {
-#pragma unroll
-    for (int i = 0; i < EL / 4; ++i) {
-      f2::dec8(raw_word(r, i), c);
-      o[2 * i] = f2::fma2(ww, c[0], o[2 * i]);
-      o[2 * i + 1] = f2::fma2(ww, c[1], o[2 * i + 1]);
-    }
+    wb[0] = u.x; wb[1] = u.y;
+    if (CE == 16) { wb[2] = u.z; wb[3] = u.w; }
   } else if (bits == 4) {
-#pragma unroll
-    for (int i = 0; i < EL / 8; ++i) {
-      f2::dec4(raw_word(r, i), c);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) o[4 * i + k] = f2::fma2(ww, c[k], o[4 * i + k]);
-    }
+    mma::spread4(u.x, wb);
+    if (CE == 16) mma::spread4(u.y, wb + 2);
   } else {
+    uint32_t t[4];
+    mma::spread2(u.x, t);
 #pragma unroll
-    for (int i = 0; i < EL / 16; ++i) {
-      f2::dec2(raw_word(r, i), c);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) o[8 * i + k] = f2::fma2(ww, c[k], o[8 * i + k]);
-    }
+    for (int i = 0; i < CE / 4; ++i) wb[i] = t[i];
   }
 }
 
@@ -177,6 +168,7 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   const int loop = P.loop;
   const int CL = chunk_loops(loop, stride);
   const int cap = CL * stride;
+  float dot_unscale = 1.f;
 
   float* p = reinterpret_cast<float*>(base);
   uint16_t* cols = reinterpret_cast<uint16_t*>(base + align16((size_t)stride * 4));
@@ -210,9 +202,14 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     n_cols += __popc(__ballot_sync(0xffffffffu, c != FL_SENTINEL));
   }
   const float m_in = P.mass[(size_t)h * P.stat_rows + srow];
-  float2 qv[EL / 2];
-  float qsum = 0.f;
+  // this lane's quarter of q; the score MMAs take it as hi + lo fp16 parts scaled by
+  // qscale, lane (g, l) feeding column n = g of B (hi for even g, lo for odd g) with
+  // quarter g / 2 and zeros elsewhere, so column pair (2l, 2l + 1) of D is quarter l's dot
+  constexpr int KS = HD / 16;
+  float qsum = 0.f, qmax = 0.f;
+  uint32_t bq[KS][2];
   {
+    float qx[EL];
     const size_t off = ((size_t)qi * H + h) * HD + e0;
 #pragma unroll
     for (int k = 0; k < EL / 2; ++k) {
@@ -227,9 +224,28 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
         a = v.x;
         b = v.y;
       }
-      qv[k] = make_float2(a, b);
+      qx[2 * k] = a;
+      qx[2 * k + 1] = b;
       qsum += a + b;
+      qmax = fmaxf(qmax, fmaxf(fabsf(a), fabsf(b)));
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+    const float qscale = mma::pow2_scale_for(qmax, 14);
+    const bool feeds = l4 == (cg >> 1);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      __half part[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        __half lo;
+        const __half hi = mma::split_hi(qx[4 * ks + j] * qscale, &lo);
+        part[j] = (cg & 1) ? lo : hi;
+      }
+      bq[ks][0] = feeds ? mma::pack_h2(part[0], part[1]) : 0u;
+      bq[ks][1] = feeds ? mma::pack_h2(part[2], part[3]) : 0u;
+    }
+    dot_unscale = mma::kCodeUnscale / qscale;   // a power of two
   }
   __syncwarp();
 
@@ -301,7 +317,10 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   const bool one_chunk = loop < 2 || CL >= loop - 1;
   int n_items = 0;   // items of the current chunk (all residual loops when one_chunk)
 
-  // ---- K base pass: two columns per lane group, score part = s (q . codes) + z sum(q)
+  float smax_v = 0.f;   // largest V scale of the rows this lane touches (bounds the weights)
+
+  // ---- K base pass: 16 columns per iteration; lane (g, l) loads quarter l of columns
+  // i0 + g and i0 + 8 + g
   for (int i0 = 0; i0 < n_cols; i0 += 16) {
     Raw<EL> raw[2];
     float sb[2], zb[2], bias_c[2];
@@ -312,6 +331,9 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
       idx[u] = i0 + 8 * u + cg;
       valid[u] = false;
       bias_c[u] = 0.f;
+      sb[u] = zb[u] = 0.f;
+#pragma unroll
+      for (int k = 0; k < EL / 16; ++k) raw[u].w[k] = make_uint4(0u, 0u, 0u, 0u);
       if (idx[u] < n_cols) {
         const int c = cols[idx[u]];
         valid[u] = c <= t && c < n_tok;
@@ -319,13 +341,24 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
           if (P.bias && l4 == 0) bias_c[u] = P.bias[c];
           const size_t bh = (size_t)c * H + h;
           load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb[u], &zb[u]);
+          float sv, zv;
+          load_sz(kv.sz[1][1], bh * ngrp + gidx, &sv, &zv);
+          smax_v = fmaxf(smax_v, sv);
           load_raw<EL>(kv.codes[0][1] + bh * HD, 8, e0, raw[u]);
         }
       }
     }
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const uint32_t w0 = raw_word(raw[0], ks), w1 = raw_word(raw[1], ks);
+      mma::m16n8k16(d, mma::code_pair(w0, 0, 1), mma::code_pair(w1, 0, 1),
+                    mma::code_pair(w0, 2, 3), mma::code_pair(w1, 2, 3), bq[ks][0], bq[ks][1]);
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      float part = valid[u] ? fmaf(sb[u], dot_raw<EL>(qv, raw[u], 8), zb[u] * qsum) : 0.f;
+      const float dot = (d[2 * u] + d[2 * u + 1]) * dot_unscale;
+      float part = valid[u] ? fmaf(sb[u], dot, zb[u] * qsum) : 0.f;
       part += __shfl_xor_sync(0xffffffffu, part, 1);
       part += __shfl_xor_sync(0xffffffffu, part, 2);
       if (idx[u] < n_cols && l4 == 0) {
@@ -355,17 +388,34 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
         const int it = i0 + 8 * u + cg;
         on[u] = it < n_items;
         bits[u] = 8;
+        sr[u] = zr[u] = 0.f;
+#pragma unroll
+        for (int k = 0; k < EL / 16; ++k) raw[u].w[k] = make_uint4(0u, 0u, 0u, 0u);
         if (on[u]) {
           const int r = it_loop[it];
           bits[u] = kv.res_bits[r];
           const size_t rh = (size_t)it_row[it] * H + h;
           load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr[u], &zr[u]);
+          float sv, zv;
+          load_sz(kv.sz[1][r], rh * ngrp + gidx, &sv, &zv);
+          smax_v = fmaxf(smax_v, sv);
           load_raw<EL>(kv.codes[0][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
         }
       }
+      uint32_t wb0[EL / 4], wb1[EL / 4];
+      to_bytes<EL>(raw[0], bits[0], wb0);
+      to_bytes<EL>(raw[1], bits[1], wb1);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        mma::m16n8k16(d, mma::code_pair(wb0[ks], 0, 1), mma::code_pair(wb1[ks], 0, 1),
+                      mma::code_pair(wb0[ks], 2, 3), mma::code_pair(wb1[ks], 2, 3),
+                      bq[ks][0], bq[ks][1]);
+      }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        float part = on[u] ? fmaf(sr[u], dot_raw<EL>(qv, raw[u], bits[u]), zr[u] * qsum) : 0.f;
+        const float dot = (d[2 * u] + d[2 * u + 1]) * dot_unscale;
+        float part = on[u] ? fmaf(sr[u], dot, zr[u] * qsum) : 0.f;
         part += __shfl_xor_sync(0xffffffffu, part, 1);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         if (on[u] && l4 == 0) it_part[i0 + 8 * u + cg] = part * sc;
@@ -448,112 +498,163 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   }
 
 
-  // ---- V passes: o part += (w s) codes + w z for every stored row of the chain
-  float2 o[EL / 2], ua[EL / 2];
+
+  // ---- V passes: rows = head elements (lane (g, l) holds elements CE g + 2 mt and
+  // CE g + 2 mt + 1 of tile mt), k = the 16 stored rows of an iteration (lane (g, l) loads
+  // rows 2l, 2l + 1, 2l + 8, 2l + 9), n = hi/lo weights of each quarter (lane (g, l)
+  // feeds n = g: quarter g / 2, hi for even g). D column pair (2l, 2l + 1) is quarter l's
+  // sum, kept by the lanes with l = g / 2, whose elements lie in that quarter.
+  constexpr int MT = HD / 16, CE = HD / 8;
+  const int vgrp = ((cg >> 1) * EL) / gs;   // group of the quarter this lane feeds
 #pragma unroll
-  for (int k = 0; k < EL / 2; ++k) { o[k] = make_float2(0.f, 0.f); ua[k] = make_float2(0.f, 0.f); }
-  float oz = 0.f, uz = 0.f;   // the offsets' share, added to every element at the end
+  for (int o = 16; o > 0; o >>= 1) smax_v = fmaxf(smax_v, __shfl_xor_sync(0xffffffffu, smax_v, o));
+  // p~ <= m, so every weight p~ s stays below 2^14 after the scaling
+  const float wscale = mma::pow2_scale_for(fabsf(m_in) * smax_v, 14);
+  const float o_unscale = mma::kCodeUnscale / wscale;   // a power of two
+  float dv[MT][4], du[SHRINK ? MT : 1][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dv[mt][j] = 0.f;
+#pragma unroll
+  for (int mt = 0; mt < (SHRINK ? MT : 1); ++mt)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) du[mt][j] = 0.f;
+  float oz = 0.f, uz = 0.f;   // sums of p~ z
+
+  auto v_batch = [&](const uint4* ch, const int* bt, const float* w, const float* s,
+                     const float* z, const bool* drop) {
+    uint32_t cw[4][CE / 4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) chunk_bytes<CE>(ch[kk], bt[kk], cw[kk]);
+    __half hv[4], hu[4];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      __half lo;
+      const __half hi = mma::split_hi(w[kk] * s[kk] * wscale, &lo);
+      oz = fmaf(w[kk], z[kk], oz);
+      hv[kk] = (cg & 1) ? lo : hi;
+      hu[kk] = __float2half(0.f);
+      if (SHRINK && drop[kk]) {
+        hu[kk] = hv[kk];
+        uz = fmaf(w[kk], z[kk], uz);
+      }
+    }
+    const uint32_t b0 = mma::pack_h2(hv[0], hv[1]), b1 = mma::pack_h2(hv[2], hv[3]);
+    const uint32_t c0 = mma::pack_h2(hu[0], hu[1]), c1 = mma::pack_h2(hu[2], hu[3]);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
+      const uint32_t t1 = __byte_perm(cw[0][mt >> 1], cw[1][mt >> 1], sel);
+      const uint32_t t2 = __byte_perm(cw[2][mt >> 1], cw[3][mt >> 1], sel);
+      const uint32_t a0 = mma::code_pair(t1, 0, 2), a1 = mma::code_pair(t1, 1, 3);
+      const uint32_t a2 = mma::code_pair(t2, 0, 2), a3 = mma::code_pair(t2, 1, 3);
+      mma::m16n8k16(dv[mt], a0, a1, a2, a3, b0, b1);
+      if (SHRINK && prune) mma::m16n8k16(du[SHRINK ? mt : 0], a0, a1, a2, a3, c0, c1);
+    }
+  };
+
   for (int i0 = 0; i0 < n_cols; i0 += 16) {
-    Raw<EL> raw[2];
-    float s[2], z[2], wgt[2];
-    bool valid[2];
+    uint4 ch[4];
+    int bt[4];
+    float w[4], s[4], z[4];
+    bool drop[4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int idx = i0 + 8 * u + cg;
-      valid[u] = false;
+    for (int kk = 0; kk < 4; ++kk) {
+      const int idx = i0 + 2 * l4 + (kk & 1) + 8 * (kk >> 1);
+      ch[kk] = make_uint4(0u, 0u, 0u, 0u);
+      bt[kk] = 8;
+      w[kk] = s[kk] = z[kk] = 0.f;
+      drop[kk] = false;
       if (idx < n_cols) {
         const int c = cols[idx];
-        valid[u] = c <= t && c < n_tok;
-        if (valid[u]) {
-          wgt[u] = p[idx];
+        if (c <= t && c < n_tok) {
+          w[kk] = p[idx];
           const size_t bh = (size_t)c * H + h;
-          load_sz(kv.sz[1][1], bh * ngrp + gidx, &s[u], &z[u]);
-          load_raw<EL>(kv.codes[1][1] + bh * HD, 8, e0, raw[u]);
+          load_sz(kv.sz[1][1], bh * ngrp + vgrp, &s[kk], &z[kk]);
+          ch[kk] = load_chunk<CE>(kv.codes[1][1] + bh * HD, 8, cg);
+          drop[kk] = SHRINK && prune && !mark[idx];
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (!valid[u]) continue;
-      const float ws = wgt[u] * s[u];
-      axpy_raw<EL>(ws, raw[u], 8, o);
-      oz = fmaf(wgt[u], z[u], oz);
-      if (SHRINK && prune && !mark[i0 + 8 * u + cg]) {
-        axpy_raw<EL>(ws, raw[u], 8, ua);
-        uz = fmaf(wgt[u], z[u], uz);
-      }
-    }
+    v_batch(ch, bt, w, s, z, drop);
   }
   for (int r0 = 2; r0 <= loop; r0 += CL) {
     const int r1 = min(loop + 1, r0 + CL);
     if (!one_chunk) n_items = build_items(r0, r1);   // else still held from the K pass
     for (int i0 = 0; i0 < n_items; i0 += 16) {
-      Raw<EL> raw[2];
-      float s[2], z[2], wgt[2];
-      int bits[2], idx[2];
-      bool on[2];
+      uint4 ch[4];
+      int bt[4];
+      float w[4], s[4], z[4];
+      bool drop[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int it = i0 + 8 * u + cg;
-        on[u] = it < n_items;
-        bits[u] = 8;
-        idx[u] = 0;
-        if (on[u]) {
+      for (int kk = 0; kk < 4; ++kk) {
+        const int it = i0 + 2 * l4 + (kk & 1) + 8 * (kk >> 1);
+        ch[kk] = make_uint4(0u, 0u, 0u, 0u);
+        bt[kk] = 8;
+        w[kk] = s[kk] = z[kk] = 0.f;
+        drop[kk] = false;
+        if (it < n_items) {
           const int r = it_loop[it];
-          bits[u] = kv.res_bits[r];
-          idx[u] = it_idx[it];
-          wgt[u] = p[idx[u]];
+          const int idx = it_idx[it];
+          bt[kk] = kv.res_bits[r];
+          w[kk] = p[idx];
           const size_t rh = (size_t)it_row[it] * H + h;
-          load_sz(kv.sz[1][r], rh * ngrp + gidx, &s[u], &z[u]);
-          load_raw<EL>(kv.codes[1][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
+          load_sz(kv.sz[1][r], rh * ngrp + vgrp, &s[kk], &z[kk]);
+          ch[kk] = load_chunk<CE>(kv.codes[1][r] + rh * (HD * bt[kk] / 8), bt[kk], cg);
+          drop[kk] = SHRINK && prune && !mark[idx];
         }
       }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (!on[u]) continue;
-        const float ws = wgt[u] * s[u];
-        axpy_raw<EL>(ws, raw[u], bits[u], o);
-        oz = fmaf(wgt[u], z[u], oz);
-        if (SHRINK && prune && !mark[idx[u]]) {
-          axpy_raw<EL>(ws, raw[u], bits[u], ua);
-          uz = fmaf(wgt[u], z[u], uz);
-        }
-      }
+      v_batch(ch, bt, w, s, z, drop);
     }
     __syncwarp();
   }
-  // reduce the 8 column groups (lanes with the same part differ in bits 2..4)
-  const float2 oz2 = make_float2(oz, oz), uz2 = make_float2(uz, uz);
 #pragma unroll
-  for (int k = 0; k < EL / 2; ++k) {
-    o[k] = f2::add2(o[k], oz2);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      o[k].x += __shfl_xor_sync(0xffffffffu, o[k].x, off);
-      o[k].y += __shfl_xor_sync(0xffffffffu, o[k].y, off);
-    }
-    if (SHRINK) {
-      ua[k] = f2::add2(ua[k], uz2);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        ua[k].x += __shfl_xor_sync(0xffffffffu, ua[k].x, off);
-        ua[k].y += __shfl_xor_sync(0xffffffffu, ua[k].y, off);
-      }
-    }
+  for (int o = 1; o <= 2; o <<= 1) {
+    oz += __shfl_xor_sync(0xffffffffu, oz, o);
+    if (SHRINK) uz += __shfl_xor_sync(0xffffffffu, uz, o);
   }
 
-  // ---- outputs (lanes 0..3 hold the four parts)
-  if (cg == 0) {
-    const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD + e0;
-    const size_t ob = ((size_t)qi * H + h) * HD + e0;
-    float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + e0 : nullptr;
+  // ---- outputs: lane (g, g / 2) writes elements [CE g, CE g + CE)
+  if (l4 == (cg >> 1)) {
+    const int eb = CE * cg;
+    const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD + eb;
+    const size_t ob = ((size_t)qi * H + h) * HD + eb;
+    float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + eb : nullptr;
+    float val[CE], uo[CE];
 #pragma unroll
-    for (int j = 0; j < EL; ++j) {
-      const float ui = u_in[j];
-      const float val = ui + ((j & 1) ? o[j >> 1].y : o[j >> 1].x);
-      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(val);
-      else reinterpret_cast<float*>(P.out)[ob + j] = val;
-      if (want_stats) u_out[j] = prune ? ui + ((j & 1) ? ua[j >> 1].y : ua[j >> 1].x) : ui;
+    for (int q4 = 0; q4 < CE / 4; ++q4) {
+      const float4 ui = reinterpret_cast<const float4*>(u_in)[q4];
+      const float uiv[4] = {ui.x, ui.y, ui.z, ui.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = 4 * q4 + j, mt = e >> 1, r2 = 2 * (e & 1);
+        const float ov = (dv[mt][r2] + dv[mt][r2 + 1]) * o_unscale + oz;
+        val[e] = uiv[j] + ov;
+        uo[e] = uiv[j];
+        if (SHRINK && prune)
+          uo[e] = uiv[j] + ((du[SHRINK ? mt : 0][r2] + du[SHRINK ? mt : 0][r2 + 1]) * o_unscale + uz);
+      }
+    }
+    if (P.out_bf16) {
+      uint32_t pk[CE / 2];
+#pragma unroll
+      for (int j = 0; j < CE / 2; ++j) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(val[2 * j], val[2 * j + 1]);
+        pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) + ob);
+#pragma unroll
+      for (int j = 0; j < CE / 8; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + ob);
+#pragma unroll
+      for (int j = 0; j < CE / 4; ++j) dst[j] = make_float4(val[4 * j], val[4 * j + 1], val[4 * j + 2], val[4 * j + 3]);
+    }
+    if (want_stats) {
+#pragma unroll
+      for (int j = 0; j < CE / 4; ++j)
+        reinterpret_cast<float4*>(u_out)[j] = make_float4(uo[4 * j], uo[4 * j + 1], uo[4 * j + 2], uo[4 * j + 3]);
     }
   }
   if (!want_stats) return;

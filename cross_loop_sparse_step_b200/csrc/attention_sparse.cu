@@ -22,13 +22,17 @@
 //   softmax over the column set, p~ = m * softmax (m = cached mass).
 //   optional budget shrink: warp radix select over the binary32 bits of p~ * ||V^||
 //     (ties to the smaller column), ballot-ordered so the kept set stays ascending.
-//   V pass (rows = head elements, k = 16 stored rows, n = hi/lo of the weights of each
-//     quarter): o = sum (p~ s) codes + sum p~ z, and for dropped columns the same into
-//     the next loop's u'. Lane (g, g / 2) ends up with elements [g hd/8, (g+1) hd/8).
+//   V pass (binary32 pairs: the weights vary per stored row, so the sums are axpys):
+//     o += (p~ s) codes + p~ z over the chain's rows, and for dropped columns the same
+//     into the next loop's u'; lane (g, l) works on quarter l of rows g and g + 8 and the
+//     eight row groups are reduced by shuffles.
+//   A chunk of residual loops holds loops of one bit width, so each residual pass runs
+//   with the width as a compile-time constant and decodes in straight-line code.
 #include <float.h>
 
 #include "fl_internal.cuh"
 #include "attn_mma.cuh"
+#include "sm100_f32x2.cuh"
 
 namespace fl {
 namespace {
@@ -117,36 +121,40 @@ __device__ __forceinline__ void to_bytes(const Raw<EL>& r, int bits, uint32_t* w
   }
 }
 
-// Chunk [CE cg, CE cg + CE) of a stored row (CE = hd / 8 codes) as raw words.
-template <int CE>
-__device__ __forceinline__ uint4 load_chunk(const uint8_t* row, int bits, int cg) {
-  const uint8_t* src = row + (size_t)CE * cg * bits / 8;
-  const int bytes = CE * bits / 8;   // 16, 8, 4 or 2
-  if (bytes == 16) return *reinterpret_cast<const uint4*>(src);
-  if (bytes == 8) {
-    const uint2 u = *reinterpret_cast<const uint2*>(src);
-    return make_uint4(u.x, u.y, 0u, 0u);
+// o[j] += w * code[j]
+template <int EL>
+__device__ __forceinline__ void axpy_raw(float w, const Raw<EL>& r, int bits, float2* o) {
+  const float2 ww = make_float2(w, w);
+  float2 c[8];
+  if (bits == 8) {
+#pragma unroll
+    for (int i = 0; i < EL / 4; ++i) {
+      f2::dec8(raw_word(r, i), c);
+      o[2 * i] = f2::fma2(ww, c[0], o[2 * i]);
+      o[2 * i + 1] = f2::fma2(ww, c[1], o[2 * i + 1]);
+    }
+  } else if (bits == 4) {
+#pragma unroll
+    for (int i = 0; i < EL / 8; ++i) {
+      f2::dec4(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) o[4 * i + k] = f2::fma2(ww, c[k], o[4 * i + k]);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < EL / 16; ++i) {
+      f2::dec2(raw_word(r, i), c);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) o[8 * i + k] = f2::fma2(ww, c[k], o[8 * i + k]);
+    }
   }
-  if (bytes == 4) return make_uint4(*reinterpret_cast<const uint32_t*>(src), 0u, 0u, 0u);
-  return make_uint4((uint32_t)*reinterpret_cast<const uint16_t*>(src), 0u, 0u, 0u);
 }
 
-// The chunk as one code per byte: CE / 4 words.
-template <int CE>
-__device__ __forceinline__ void chunk_bytes(uint4 u, int bits, uint32_t* wb) {
-  if (bits == 8) {
-    wb[0] = u.x; wb[1] = u.y;
-    if (CE == 16) { wb[2] = u.z; wb[3] = u.w; }
-  } else if (bits == 4) {
-    mma::spread4(u.x, wb);
-    if (CE == 16) mma::spread4(u.y, wb + 2);
-  } else {
-    uint32_t t[4];
-    mma::spread2(u.x, t);
-#pragma unroll
-    for (int i = 0; i < CE / 4; ++i) wb[i] = t[i];
-  }
-}
+// A bit width as a type.
+template <int B>
+struct Width {
+  static constexpr int value = B;
+};
 
 // One warp's work: (query, head) number gw of the call described by P, with `base` the
 // warp's shared-memory slice. No CTA-wide barrier is used.
@@ -314,10 +322,15 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     }
     return total;
   };
-  const bool one_chunk = loop < 2 || CL >= loop - 1;
+  // a chunk: up to CL consecutive residual loops of one bit width
+  auto chunk_end = [&](int r0) -> int {
+    const int r1 = min(loop + 1, r0 + CL);
+    for (int r = r0 + 1; r < r1; ++r)
+      if (kv.res_bits[r] != kv.res_bits[r0]) return r;
+    return r1;
+  };
+  const bool one_chunk = loop < 2 || chunk_end(2) == loop + 1;
   int n_items = 0;   // items of the current chunk (all residual loops when one_chunk)
-
-  float smax_v = 0.f;   // largest V scale of the rows this lane touches (bounds the weights)
 
   // ---- K base pass: 16 columns per iteration; lane (g, l) loads quarter l of columns
   // i0 + g and i0 + 8 + g
@@ -341,9 +354,6 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
           if (P.bias && l4 == 0) bias_c[u] = P.bias[c];
           const size_t bh = (size_t)c * H + h;
           load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb[u], &zb[u]);
-          float sv, zv;
-          load_sz(kv.sz[1][1], bh * ngrp + gidx, &sv, &zv);
-          smax_v = fmaxf(smax_v, sv);
           load_raw<EL>(kv.codes[0][1] + bh * HD, 8, e0, raw[u]);
         }
       }
@@ -374,9 +384,9 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
   __syncwarp();
 
   // ---- K residual passes: items of a chunk as one stream, parts added in loop order
-  for (int r0 = 2; r0 <= loop; r0 += CL) {
-    const int r1 = min(loop + 1, r0 + CL);
-    n_items = build_items(r0, r1);
+  // (a chunk holds loops of one bit width, a compile-time constant in its pass)
+  auto k_res_pass = [&](auto width) {
+    constexpr int UB = decltype(width)::value;
     const float sc = P.scale;
     for (int i0 = 0; i0 < n_items; i0 += 16) {
       Raw<EL> raw[2];
@@ -387,18 +397,14 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
       for (int u = 0; u < 2; ++u) {
         const int it = i0 + 8 * u + cg;
         on[u] = it < n_items;
-        bits[u] = 8;
+        bits[u] = UB;
         sr[u] = zr[u] = 0.f;
 #pragma unroll
         for (int k = 0; k < EL / 16; ++k) raw[u].w[k] = make_uint4(0u, 0u, 0u, 0u);
         if (on[u]) {
           const int r = it_loop[it];
-          bits[u] = kv.res_bits[r];
           const size_t rh = (size_t)it_row[it] * H + h;
           load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr[u], &zr[u]);
-          float sv, zv;
-          load_sz(kv.sz[1][r], rh * ngrp + gidx, &sv, &zv);
-          smax_v = fmaxf(smax_v, sv);
           load_raw<EL>(kv.codes[0][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
         }
       }
@@ -420,6 +426,15 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         if (on[u] && l4 == 0) it_part[i0 + 8 * u + cg] = part * sc;
       }
+    }
+  };
+  for (int r0 = 2, r1; r0 <= loop; r0 = r1) {
+    r1 = chunk_end(r0);
+    n_items = build_items(r0, r1);
+    switch (kv.res_bits[r0]) {   // 2, 4 or 8 (checked at launch)
+      case 2: k_res_pass(Width<2>{}); break;
+      case 4: k_res_pass(Width<4>{}); break;
+      default: k_res_pass(Width<8>{}); break;
     }
     __syncwarp();
     for (int k = 0; k < r1 - r0; ++k) {   // loop order; a loop lists a column at most once
@@ -499,162 +514,120 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
 
 
 
-  // ---- V passes: rows = head elements (lane (g, l) holds elements CE g + 2 mt and
-  // CE g + 2 mt + 1 of tile mt), k = the 16 stored rows of an iteration (lane (g, l) loads
-  // rows 2l, 2l + 1, 2l + 8, 2l + 9), n = hi/lo weights of each quarter (lane (g, l)
-  // feeds n = g: quarter g / 2, hi for even g). D column pair (2l, 2l + 1) is quarter l's
-  // sum, kept by the lanes with l = g / 2, whose elements lie in that quarter.
-  constexpr int MT = HD / 16, CE = HD / 8;
-  const int vgrp = ((cg >> 1) * EL) / gs;   // group of the quarter this lane feeds
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) smax_v = fmaxf(smax_v, __shfl_xor_sync(0xffffffffu, smax_v, o));
-  // p~ <= m, so every weight p~ s stays below 2^14 after the scaling
-  const float wscale = mma::pow2_scale_for(fabsf(m_in) * smax_v, 14);
-  const float o_unscale = mma::kCodeUnscale / wscale;   // a power of two
-  float dv[MT][4], du[SHRINK ? MT : 1][4];
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dv[mt][j] = 0.f;
-#pragma unroll
-  for (int mt = 0; mt < (SHRINK ? MT : 1); ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) du[mt][j] = 0.f;
-  float oz = 0.f, uz = 0.f;   // sums of p~ z
 
-  auto v_batch = [&](const uint4* ch, const int* bt, const float* w, const float* s,
-                     const float* z, const bool* drop) {
-    uint32_t cw[4][CE / 4];
+  // ---- V passes: o part += (w s) codes + w z for every stored row of the chain
+  float2 o[EL / 2], ua[EL / 2];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) chunk_bytes<CE>(ch[kk], bt[kk], cw[kk]);
-    __half hv[4], hu[4];
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      __half lo;
-      const __half hi = mma::split_hi(w[kk] * s[kk] * wscale, &lo);
-      oz = fmaf(w[kk], z[kk], oz);
-      hv[kk] = (cg & 1) ? lo : hi;
-      hu[kk] = __float2half(0.f);
-      if (SHRINK && drop[kk]) {
-        hu[kk] = hv[kk];
-        uz = fmaf(w[kk], z[kk], uz);
-      }
-    }
-    const uint32_t b0 = mma::pack_h2(hv[0], hv[1]), b1 = mma::pack_h2(hv[2], hv[3]);
-    const uint32_t c0 = mma::pack_h2(hu[0], hu[1]), c1 = mma::pack_h2(hu[2], hu[3]);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const uint32_t sel = (mt & 1) ? 0x7632u : 0x5410u;
-      const uint32_t t1 = __byte_perm(cw[0][mt >> 1], cw[1][mt >> 1], sel);
-      const uint32_t t2 = __byte_perm(cw[2][mt >> 1], cw[3][mt >> 1], sel);
-      const uint32_t a0 = mma::code_pair(t1, 0, 2), a1 = mma::code_pair(t1, 1, 3);
-      const uint32_t a2 = mma::code_pair(t2, 0, 2), a3 = mma::code_pair(t2, 1, 3);
-      mma::m16n8k16(dv[mt], a0, a1, a2, a3, b0, b1);
-      if (SHRINK && prune) mma::m16n8k16(du[SHRINK ? mt : 0], a0, a1, a2, a3, c0, c1);
-    }
-  };
-
+  for (int k = 0; k < EL / 2; ++k) { o[k] = make_float2(0.f, 0.f); ua[k] = make_float2(0.f, 0.f); }
+  float oz = 0.f, uz = 0.f;   // the offsets' share, added to every element at the end
   for (int i0 = 0; i0 < n_cols; i0 += 16) {
-    uint4 ch[4];
-    int bt[4];
-    float w[4], s[4], z[4];
-    bool drop[4];
+    Raw<EL> raw[2];
+    float s[2], z[2], wgt[2];
+    bool valid[2];
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int idx = i0 + 2 * l4 + (kk & 1) + 8 * (kk >> 1);
-      ch[kk] = make_uint4(0u, 0u, 0u, 0u);
-      bt[kk] = 8;
-      w[kk] = s[kk] = z[kk] = 0.f;
-      drop[kk] = false;
+    for (int u = 0; u < 2; ++u) {
+      const int idx = i0 + 8 * u + cg;
+      valid[u] = false;
       if (idx < n_cols) {
         const int c = cols[idx];
-        if (c <= t && c < n_tok) {
-          w[kk] = p[idx];
+        valid[u] = c <= t && c < n_tok;
+        if (valid[u]) {
+          wgt[u] = p[idx];
           const size_t bh = (size_t)c * H + h;
-          load_sz(kv.sz[1][1], bh * ngrp + vgrp, &s[kk], &z[kk]);
-          ch[kk] = load_chunk<CE>(kv.codes[1][1] + bh * HD, 8, cg);
-          drop[kk] = SHRINK && prune && !mark[idx];
+          load_sz(kv.sz[1][1], bh * ngrp + gidx, &s[u], &z[u]);
+          load_raw<EL>(kv.codes[1][1] + bh * HD, 8, e0, raw[u]);
         }
       }
     }
-    v_batch(ch, bt, w, s, z, drop);
-  }
-  for (int r0 = 2; r0 <= loop; r0 += CL) {
-    const int r1 = min(loop + 1, r0 + CL);
-    if (!one_chunk) n_items = build_items(r0, r1);   // else still held from the K pass
-    for (int i0 = 0; i0 < n_items; i0 += 16) {
-      uint4 ch[4];
-      int bt[4];
-      float w[4], s[4], z[4];
-      bool drop[4];
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const int it = i0 + 2 * l4 + (kk & 1) + 8 * (kk >> 1);
-        ch[kk] = make_uint4(0u, 0u, 0u, 0u);
-        bt[kk] = 8;
-        w[kk] = s[kk] = z[kk] = 0.f;
-        drop[kk] = false;
-        if (it < n_items) {
+    for (int u = 0; u < 2; ++u) {
+      if (!valid[u]) continue;
+      const float ws = wgt[u] * s[u];
+      axpy_raw<EL>(ws, raw[u], 8, o);
+      oz = fmaf(wgt[u], z[u], oz);
+      if (SHRINK && prune && !mark[i0 + 8 * u + cg]) {
+        axpy_raw<EL>(ws, raw[u], 8, ua);
+        uz = fmaf(wgt[u], z[u], uz);
+      }
+    }
+  }
+  auto v_res_pass = [&](auto width) {
+    constexpr int UB = decltype(width)::value;
+    for (int i0 = 0; i0 < n_items; i0 += 16) {
+      Raw<EL> raw[2];
+      float s[2], z[2], wgt[2];
+      int bits[2], idx[2];
+      bool on[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = i0 + 8 * u + cg;
+        on[u] = it < n_items;
+        bits[u] = UB;
+        idx[u] = 0;
+        if (on[u]) {
           const int r = it_loop[it];
-          const int idx = it_idx[it];
-          bt[kk] = kv.res_bits[r];
-          w[kk] = p[idx];
+          idx[u] = it_idx[it];
+          wgt[u] = p[idx[u]];
           const size_t rh = (size_t)it_row[it] * H + h;
-          load_sz(kv.sz[1][r], rh * ngrp + vgrp, &s[kk], &z[kk]);
-          ch[kk] = load_chunk<CE>(kv.codes[1][r] + rh * (HD * bt[kk] / 8), bt[kk], cg);
-          drop[kk] = SHRINK && prune && !mark[idx];
+          load_sz(kv.sz[1][r], rh * ngrp + gidx, &s[u], &z[u]);
+          load_raw<EL>(kv.codes[1][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
         }
       }
-      v_batch(ch, bt, w, s, z, drop);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (!on[u]) continue;
+        const float ws = wgt[u] * s[u];
+        axpy_raw<EL>(ws, raw[u], bits[u], o);
+        oz = fmaf(wgt[u], z[u], oz);
+        if (SHRINK && prune && !mark[idx[u]]) {
+          axpy_raw<EL>(ws, raw[u], bits[u], ua);
+          uz = fmaf(wgt[u], z[u], uz);
+        }
+      }
+    }
+  };
+  for (int r0 = 2, r1; r0 <= loop; r0 = r1) {
+    r1 = chunk_end(r0);
+    if (!one_chunk) n_items = build_items(r0, r1);   // else still held from the K pass
+    switch (kv.res_bits[r0]) {
+      case 2: v_res_pass(Width<2>{}); break;
+      case 4: v_res_pass(Width<4>{}); break;
+      default: v_res_pass(Width<8>{}); break;
     }
     __syncwarp();
   }
+  // reduce the 8 column groups (lanes with the same part differ in bits 2..4)
+  const float2 oz2 = make_float2(oz, oz), uz2 = make_float2(uz, uz);
 #pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    oz += __shfl_xor_sync(0xffffffffu, oz, o);
-    if (SHRINK) uz += __shfl_xor_sync(0xffffffffu, uz, o);
+  for (int k = 0; k < EL / 2; ++k) {
+    o[k] = f2::add2(o[k], oz2);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      o[k].x += __shfl_xor_sync(0xffffffffu, o[k].x, off);
+      o[k].y += __shfl_xor_sync(0xffffffffu, o[k].y, off);
+    }
+    if (SHRINK) {
+      ua[k] = f2::add2(ua[k], uz2);
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        ua[k].x += __shfl_xor_sync(0xffffffffu, ua[k].x, off);
+        ua[k].y += __shfl_xor_sync(0xffffffffu, ua[k].y, off);
+      }
+    }
   }
 
-  // ---- outputs: lane (g, g / 2) writes elements [CE g, CE g + CE)
-  if (l4 == (cg >> 1)) {
-    const int eb = CE * cg;
-    const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD + eb;
-    const size_t ob = ((size_t)qi * H + h) * HD + eb;
-    float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + eb : nullptr;
-    float val[CE], uo[CE];
+  // ---- outputs (lanes 0..3 hold the four parts)
+  if (cg == 0) {
+    const float* u_in = P.unsel + ((size_t)h * P.stat_rows + srow) * HD + e0;
+    const size_t ob = ((size_t)qi * H + h) * HD + e0;
+    float* u_out = want_stats ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HD + e0 : nullptr;
 #pragma unroll
-    for (int q4 = 0; q4 < CE / 4; ++q4) {
-      const float4 ui = reinterpret_cast<const float4*>(u_in)[q4];
-      const float uiv[4] = {ui.x, ui.y, ui.z, ui.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = 4 * q4 + j, mt = e >> 1, r2 = 2 * (e & 1);
-        const float ov = (dv[mt][r2] + dv[mt][r2 + 1]) * o_unscale + oz;
-        val[e] = uiv[j] + ov;
-        uo[e] = uiv[j];
-        if (SHRINK && prune)
-          uo[e] = uiv[j] + ((du[SHRINK ? mt : 0][r2] + du[SHRINK ? mt : 0][r2 + 1]) * o_unscale + uz);
-      }
-    }
-    if (P.out_bf16) {
-      uint32_t pk[CE / 2];
-#pragma unroll
-      for (int j = 0; j < CE / 2; ++j) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(val[2 * j], val[2 * j + 1]);
-        pk[j] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(P.out) + ob);
-#pragma unroll
-      for (int j = 0; j < CE / 8; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-    } else {
-      float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + ob);
-#pragma unroll
-      for (int j = 0; j < CE / 4; ++j) dst[j] = make_float4(val[4 * j], val[4 * j + 1], val[4 * j + 2], val[4 * j + 3]);
-    }
-    if (want_stats) {
-#pragma unroll
-      for (int j = 0; j < CE / 4; ++j)
-        reinterpret_cast<float4*>(u_out)[j] = make_float4(uo[4 * j], uo[4 * j + 1], uo[4 * j + 2], uo[4 * j + 3]);
+    for (int j = 0; j < EL; ++j) {
+      const float ui = u_in[j];
+      const float val = ui + ((j & 1) ? o[j >> 1].y : o[j >> 1].x);
+      if (P.out_bf16) reinterpret_cast<__nv_bfloat16*>(P.out)[ob + j] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(P.out)[ob + j] = val;
+      if (want_stats) u_out[j] = prune ? ui + ((j & 1) ? ua[j >> 1].y : ua[j >> 1].x) : ui;
     }
   }
   if (!want_stats) return;

@@ -341,22 +341,15 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     bool valid[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
+      // rows past the set or outside [0, t] read column 0 (always stored) and are masked
       idx[u] = i0 + 8 * u + cg;
-      valid[u] = false;
-      bias_c[u] = 0.f;
-      sb[u] = zb[u] = 0.f;
-#pragma unroll
-      for (int k = 0; k < EL / 16; ++k) raw[u].w[k] = make_uint4(0u, 0u, 0u, 0u);
-      if (idx[u] < n_cols) {
-        const int c = cols[idx[u]];
-        valid[u] = c <= t && c < n_tok;
-        if (valid[u]) {
-          if (P.bias && l4 == 0) bias_c[u] = P.bias[c];
-          const size_t bh = (size_t)c * H + h;
-          load_sz(kv.sz[0][1], bh * ngrp + gidx, &sb[u], &zb[u]);
-          load_raw<EL>(kv.codes[0][1] + bh * HD, 8, e0, raw[u]);
-        }
-      }
+      const int ci = idx[u] < n_cols ? (int)cols[idx[u]] : 0;
+      valid[u] = idx[u] < n_cols && ci <= t && ci < n_tok;
+      const int c = valid[u] ? ci : 0;
+      bias_c[u] = (P.bias && l4 == 0) ? P.bias[c] : 0.f;
+      const uint32_t bh = (uint32_t)c * H + h;
+      load_sz(kv.sz[0][1], (size_t)bh * ngrp + gidx, &sb[u], &zb[u]);
+      load_raw<EL>(kv.codes[0][1] + (size_t)bh * HD, 8, e0, raw[u]);
     }
     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -395,18 +388,15 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
       bool on[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int it = i0 + 8 * u + cg;
-        on[u] = it < n_items;
+        // items past the chunk read item 0 (the chunk has one) and are masked
+        const int it0 = i0 + 8 * u + cg;
+        on[u] = it0 < n_items;
+        const int it = on[u] ? it0 : 0;
         bits[u] = UB;
-        sr[u] = zr[u] = 0.f;
-#pragma unroll
-        for (int k = 0; k < EL / 16; ++k) raw[u].w[k] = make_uint4(0u, 0u, 0u, 0u);
-        if (on[u]) {
-          const int r = it_loop[it];
-          const size_t rh = (size_t)it_row[it] * H + h;
-          load_sz(kv.sz[0][r], rh * ngrp + gidx, &sr[u], &zr[u]);
-          load_raw<EL>(kv.codes[0][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
-        }
+        const int r = it_loop[it];
+        const uint32_t rh = (uint32_t)it_row[it] * H + h;
+        load_sz(kv.sz[0][r], (size_t)rh * ngrp + gidx, &sr[u], &zr[u]);
+        load_raw<EL>(kv.codes[0][r] + (size_t)rh * (HD * UB / 8), UB, e0, raw[u]);
       }
       uint32_t wb0[EL / 4], wb1[EL / 4];
       to_bytes<EL>(raw[0], bits[0], wb0);
@@ -527,17 +517,13 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int idx = i0 + 8 * u + cg;
-      valid[u] = false;
-      if (idx < n_cols) {
-        const int c = cols[idx];
-        valid[u] = c <= t && c < n_tok;
-        if (valid[u]) {
-          wgt[u] = p[idx];
-          const size_t bh = (size_t)c * H + h;
-          load_sz(kv.sz[1][1], bh * ngrp + gidx, &s[u], &z[u]);
-          load_raw<EL>(kv.codes[1][1] + bh * HD, 8, e0, raw[u]);
-        }
-      }
+      const int ci = idx < n_cols ? (int)cols[idx] : 0;
+      valid[u] = idx < n_cols && ci <= t && ci < n_tok;
+      const int c = valid[u] ? ci : 0;   // masked rows read column 0
+      wgt[u] = valid[u] ? p[idx] : 0.f;
+      const uint32_t bh = (uint32_t)c * H + h;
+      load_sz(kv.sz[1][1], (size_t)bh * ngrp + gidx, &s[u], &z[u]);
+      load_raw<EL>(kv.codes[1][1] + (size_t)bh * HD, 8, e0, raw[u]);
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -560,18 +546,16 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
       bool on[2];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        const int it = i0 + 8 * u + cg;
-        on[u] = it < n_items;
+        const int it0 = i0 + 8 * u + cg;
+        on[u] = it0 < n_items;
+        const int it = on[u] ? it0 : 0;   // masked items read item 0
         bits[u] = UB;
-        idx[u] = 0;
-        if (on[u]) {
-          const int r = it_loop[it];
-          idx[u] = it_idx[it];
-          wgt[u] = p[idx[u]];
-          const size_t rh = (size_t)it_row[it] * H + h;
-          load_sz(kv.sz[1][r], rh * ngrp + gidx, &s[u], &z[u]);
-          load_raw<EL>(kv.codes[1][r] + rh * (HD * bits[u] / 8), bits[u], e0, raw[u]);
-        }
+        const int r = it_loop[it];
+        idx[u] = it_idx[it];
+        wgt[u] = p[idx[u]];
+        const uint32_t rh = (uint32_t)it_row[it] * H + h;
+        load_sz(kv.sz[1][r], (size_t)rh * ngrp + gidx, &s[u], &z[u]);
+        load_raw<EL>(kv.codes[1][r] + (size_t)rh * (HD * UB / 8), UB, e0, raw[u]);
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {

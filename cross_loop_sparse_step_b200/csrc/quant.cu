@@ -26,6 +26,31 @@ struct QuantOut {
   int row0;           // first residual row written (loop >= 2)
 };
 
+// K^ or V^ of token t at loop `upto` (t is the same for the whole warp, upto <= 31): lanes
+// 2..upto look up the slot rows of their loops at once, then the chain's rows are decoded
+// and added in loop order (a raw loop replaces the value).
+template <int N>
+__device__ __forceinline__ void reconstruct_warp(const KvView& kv, int which, int upto, int t,
+                                                 int h, int e0, int lane, float* acc) {
+  int my_row = -1;
+  if (lane >= 2 && lane <= upto) my_row = kv.slot[(size_t)lane * kv.n_tok + t];
+  decode_run<N>(kv, which, 1, kv.base_bits, t, h, e0, acc);
+  for (int r = 2; r <= upto; ++r) {
+    const int row = __shfl_sync(0xffffffffu, my_row, r);
+    if (row < 0) continue;
+    float d[N];
+    const int bits = kv.res_bits[r];
+    decode_run<N>(kv, which, r, bits, row, h, e0, d);
+    if (bits == 0) {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = d[i];
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = __fadd_rn(acc[i], d[i]);
+    }
+  }
+}
+
 template <int EPL, typename T>
 __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int loop,
                                                   const T* __restrict__ k_new,
@@ -54,7 +79,7 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
   float prev[EPL];
   float x[EPL];
   if (loop >= 2) {
-    reconstruct<EPL>(kv, which, loop - 1, t, h, e0, prev);
+    reconstruct_warp<EPL>(kv, which, loop - 1, t, h, e0, lane, prev);
 #pragma unroll
     for (int j = 0; j < EPL; ++j) x[j] = bits == 0 ? xin[j] : __fsub_rn(xin[j], prev[j]);
   } else {

@@ -373,21 +373,28 @@ def main():
         for kind in (0, 1):
             lib.fl_set_timing_events(kind, None, None, 0)
 
-    graph = None
-    kernels_per_step = None
+    graph = None        # the timed step
+    graph_h = None      # the same step with kernel events (per-kernel times, replayed apart:
+    kernels_per_step = None   # event nodes between kernels would hold back their overlap)
     if args.graph:
         restore(W)
         torch.cuda.synchronize()
-        arm_hooks()
         c0 = lib.fl_launch_count()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step_loops(W)
         kernels_per_step = lib.fl_launch_count() - c0
+        restore(W)
+        torch.cuda.synchronize()
+        arm_hooks()
+        graph_h = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_h):
+            step_loops(W)
         disarm_hooks()
-        for _ in range(2):
-            restore(W)
-            graph.replay()
+        for g in (graph, graph_h):
+            for _ in range(2):
+                restore(W)
+                g.replay()
         torch.cuda.synchronize()
         st = fl.check_device_status()
         if st != 0:
@@ -417,10 +424,6 @@ def main():
             step_loops(W)
         ends[i].record(stream)
         torch.cuda.nvtx.range_pop()
-        if graph is not None:   # the graph re-records one step's kernel events per replay
-            ends[i].synchronize()
-            for kind in (0, 1):
-                kern_ms[kind] += [x.elapsed_time(y) for x, y in zip(ev[kind][0], ev[kind][1])]
     torch.cuda.synchronize()
     if not args.graph:
         disarm_hooks()
@@ -428,6 +431,13 @@ def main():
             kern_ms[kind] = [x.elapsed_time(y) for x, y in zip(ev[kind][0], ev[kind][1])]
     launches = (lib.fl_launch_count() - launches0) if graph is None else kernels_per_step * args.steps
     clk = clocks.stop()
+    if graph_h is not None:   # per-kernel times: the instrumented step, replayed as often
+        for i in range(args.steps):
+            restore(W)
+            graph_h.replay()
+            torch.cuda.synchronize()
+            for kind in (0, 1):
+                kern_ms[kind] += [x.elapsed_time(y) for x, y in zip(ev[kind][0], ev[kind][1])]
     if world > 1:
         dist.barrier()
     st = fl.check_device_status()

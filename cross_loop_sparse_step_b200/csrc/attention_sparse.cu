@@ -638,6 +638,7 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
 template <int HD, bool SHRINK>
 __global__ void __launch_bounds__(NW * 32, min_ctas(SHRINK)) k_attn_sparse(const __grid_constant__ AttnParams P) {
   extern __shared__ __align__(16) uint8_t smem[];
+  griddep_wait();
   const int w = threadIdx.x >> 5;
   const int gw = blockIdx.x * NW + w;
   if (gw >= P.n_q * P.H) return;  // whole warp leaves
@@ -689,9 +690,9 @@ cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     have = (int)sm;
   }
-  kern<<<blocks, NW * 32, sm, s>>>(P);
+  const cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(NW * 32), sm, s, P);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Ps: device array of n AttnParams (already copied by the caller, same shapes; loops up

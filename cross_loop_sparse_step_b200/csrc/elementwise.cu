@@ -34,6 +34,7 @@ template <typename T>
 __global__ void __launch_bounds__(1024) k_rmsnorm_v8(const float* __restrict__ x,
                                                     const float* __restrict__ gamma, float eps,
                                                     T* __restrict__ out, int d) {
+  griddep_wait();
   const int row = blockIdx.x;
   const int e0 = threadIdx.x * 8;
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)row * d + e0);
@@ -139,8 +140,12 @@ cudaError_t launch_rmsnorm(const float* x, const float* gamma, float eps, void* 
   const bool v8 = d % 256 == 0 && d / 8 <= 1024 && (uintptr_t)x % 16 == 0 &&
                   (uintptr_t)gamma % 16 == 0 && (uintptr_t)out % 16 == 0;
   if (v8) {
-    if (dt == FL_F32) k_rmsnorm_v8<float><<<M, d / 8, 0, s>>>(x, gamma, eps, (float*)out, d);
-    else k_rmsnorm_v8<__nv_bfloat16><<<M, d / 8, 0, s>>>(x, gamma, eps, (__nv_bfloat16*)out, d);
+    const cudaError_t e =
+        dt == FL_F32 ? launch_pdl(k_rmsnorm_v8<float>, dim3(M), dim3(d / 8), 0, s, x, gamma, eps,
+                                  (float*)out, d)
+                     : launch_pdl(k_rmsnorm_v8<__nv_bfloat16>, dim3(M), dim3(d / 8), 0, s, x, gamma,
+                                  eps, (__nv_bfloat16*)out, d);
+    if (e != cudaSuccess) return e;
   } else if (dt == FL_F32) {
     k_rmsnorm<float><<<M, 256, 0, s>>>(x, gamma, eps, (float*)out, d);
   } else {

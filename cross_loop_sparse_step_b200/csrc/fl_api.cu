@@ -25,6 +25,15 @@ cudaError_t launch_gemm_qkv(const void* A, const void* W, float* q, float* k, fl
                             cudaStream_t s, const fl_kv_desc* fuse, int loop,
                             const GemmScratch* scr);
 
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("FL_PDL");
+    on = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return on == 1;
+}
+
 int* status_word() {
   static int* cache[128] = {nullptr};
   static std::mutex mu;

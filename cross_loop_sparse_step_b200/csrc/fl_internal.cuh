@@ -23,6 +23,28 @@ __device__ __forceinline__ void record_error(int* st, int code) {
 // Every kernel launch of the library bumps a process-wide counter (read through
 // fl_launch_count); GEMM and attention launches can be bracketed by caller events.
 void count_launch();
+
+// Programmatic dependent launch: a kernel launched this way may start (its CTAs placed,
+// its prologue run) while the previous kernel on the stream drains; it calls
+// griddep_wait() before it touches global memory that kernel writes or reads. FL_PDL=0
+// turns it off.
+bool pdl_enabled();
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 enum TimedKind { TIMED_GEMM = 0, TIMED_ATTN = 1, TIMED_KINDS = 2 };
 void timing_begin(int kind, cudaStream_t s);
 void timing_end(int kind, cudaStream_t s);

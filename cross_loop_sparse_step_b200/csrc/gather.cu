@@ -28,6 +28,7 @@ __global__ void __launch_bounds__(256) k_gather_scatter(int op, const uint8_t* _
 }
 
 __global__ void k_fill_i32(int32_t* p, int32_t v, size_t n) {
+  griddep_wait();
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x)
     p[i] = v;
@@ -62,8 +63,9 @@ cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const
 cudaError_t launch_fill_i32(int32_t* p, int32_t v, size_t n, cudaStream_t s) {
   if (n == 0) return cudaSuccess;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  k_fill_i32<<<blocks, 256, 0, s>>>(p, v, n);
+  const cudaError_t e = launch_pdl(k_fill_i32, dim3(blocks), dim3(256), 0, s, p, v, n);
   count_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

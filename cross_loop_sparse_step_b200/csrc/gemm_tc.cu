@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_slot;
+  griddep_wait();   // operands and C may still be in flight from the previous kernel
 
   if (warp == 0) {
     if (lane == 0) {
@@ -508,16 +509,19 @@ cudaError_t launch_bn(const void* A, const void* W, float* C, __nv_bfloat16* Y, 
   const int sms = sm_count();
   int grid = tiles < sms ? tiles : sms;
   SkPlan plan{0, nullptr, nullptr};
+  cudaError_t e;
   if (use_sk(tiles, K / BK, BN) && scr && scr->flag && scr->part && sms * 4 <= scr->n_flag &&
       (size_t)sms * BM * BN * 4 <= scr->part_bytes) {
     grid = sms;
     plan = SkPlan{1, scr->part, scr->flag};
-    kern_sk<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, plan, status_word());
+    e = launch_pdl(kern_sk, dim3(grid), dim3(192), smem, s, ma, mb, C, Y, M, N, K, ldc, N / 2, qo,
+                   plan, status_word());
   } else {
-    kern_dp<<<grid, 192, smem, s>>>(ma, mb, C, Y, M, N, K, ldc, N / 2, qo, plan, status_word());
+    e = launch_pdl(kern_dp, dim3(grid), dim3(192), smem, s, ma, mb, C, Y, M, N, K, ldc, N / 2, qo,
+                   plan, status_word());
   }
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
                                                   const T* __restrict__ v_new,
                                                   const int32_t* __restrict__ act_tok,
                                                   int n_act, int* st) {
+  griddep_wait();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int H = kv.H, hd = kv.hd, g = kv.g;
@@ -155,14 +156,14 @@ cudaError_t launch_epl(const KvView& v, const QuantOut& o, int loop, const void*
                        cudaStream_t s) {
   const size_t warps = (size_t)n_act * v.H * 2;
   const int blocks = (int)((warps * 32 + 255) / 256);
-  if (dt == FL_F32)
-    k_kv_quant<EPL, float><<<blocks, 256, 0, s>>>(v, o, loop, (const float*)k,
-                                                  (const float*)vv, act, n_act, st);
-  else
-    k_kv_quant<EPL, __nv_bfloat16><<<blocks, 256, 0, s>>>(
-        v, o, loop, (const __nv_bfloat16*)k, (const __nv_bfloat16*)vv, act, n_act, st);
+  const cudaError_t e =
+      dt == FL_F32
+          ? launch_pdl(k_kv_quant<EPL, float>, dim3(blocks), dim3(256), 0, s, v, o, loop,
+                       (const float*)k, (const float*)vv, act, n_act, st)
+          : launch_pdl(k_kv_quant<EPL, __nv_bfloat16>, dim3(blocks), dim3(256), 0, s, v, o, loop,
+                       (const __nv_bfloat16*)k, (const __nv_bfloat16*)vv, act, n_act, st);
   count_launch();
-  return cudaGetLastError();
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace

@@ -263,6 +263,10 @@ typedef struct {
   const float* col_bias;            /* device [n_tok] logit bias per column, nullable */
 } fl_model;
 
+/* Device workspace of the block calls: the RoPE table, the projection GEMMs' stream-K
+ * scratch (partial tiles and hand-over flags, cleared by every call) and the half-layer
+ * intermediates. One workspace serves one call at a time (calls on different streams
+ * need their own). Depends on the current device's SM count. */
 size_t fl_block_workspace_bytes(const fl_model* m, int32_t n_rows);
 /* RMSNorm + fused q/k/v projection + RoPE of n_rows rows x (device float [n][d])
  * at positions pos (device int32 [n]); writes q, k, v (device float [n][H][hd]). */

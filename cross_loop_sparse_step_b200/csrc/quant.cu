@@ -51,6 +51,69 @@ __device__ __forceinline__ void reconstruct_warp(const KvView& kv, int which, in
   }
 }
 
+// Quantises this lane's EPL values x of (row, head h, K|V) (group g = LPG lanes), stores
+// codes and (s, z); hat = the reconstruction (prev + deq, or deq at loop 1; raw values
+// when bits == 0).
+template <int EPL>
+__device__ __forceinline__ void quant_store(const KvView& kv, const QuantOut& out, int which,
+                                            int loop, int bits, size_t row, int h, int e0,
+                                            int lane, const float* xin, const float* x,
+                                            const float* prev, float* hat, int* st) {
+  const int H = kv.H, hd = kv.hd, g = kv.g;
+  if (bits == 0) {
+    float* dst = reinterpret_cast<float*>(out.codes[which]) + (row * H + h) * hd + e0;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) { dst[j] = xin[j]; hat[j] = xin[j]; }
+    return;
+  }
+  const int LPG = g / EPL;  // lanes per group
+  float mn = x[0], mx = x[0];
+#pragma unroll
+  for (int j = 1; j < EPL; ++j) { mn = fminf(mn, x[j]); mx = fmaxf(mx, x[j]); }
+  for (int o = 1; o < LPG; o <<= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const __half zh = __float2half_rd(mn);
+  const float zf = __half2float(zh);
+  const float qmax = (float)((1 << bits) - 1);
+  const float t1 = __fsub_ru(mx, zf);
+  const float t2 = __fdiv_ru(t1, qmax);
+  const __half sh = __float2half_ru(t2);
+  const float sf = __half2float(sh);
+  const bool bad = isinf(zf) || isinf(sf) || isnan(zf) || isnan(sf);
+  if (bad && (lane % LPG) == 0) record_error(st, FL_ERR_RANGE);
+  uint32_t word = 0;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    int code = 0;
+    if (!bad && sf != 0.f) {
+      const float w = __fdiv_rn(__fsub_rn(x[j], zf), sf);
+      code = (int)fminf(fmaxf(rintf(w), 0.f), qmax);
+    }
+    const float deq = __fmaf_rn((float)code, sf, zf);
+    hat[j] = loop == 1 ? deq : __fadd_rn(prev[j], deq);
+    word |= (uint32_t)code << (j * bits);
+  }
+  // combine the lanes that share one 32-bit output word
+  const int wbits = EPL * bits;
+  const int LPW = 32 / wbits;
+  word <<= (lane % LPW) * wbits;
+  for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
+  const size_t rowbytes = (size_t)hd * bits / 8;
+  if (lane % LPW == 0) {
+    uint32_t* cw = reinterpret_cast<uint32_t*>(out.codes[which] + (row * H + h) * rowbytes);
+    cw[lane / LPW] = word;
+  }
+  if (lane % LPG == 0) {
+    uint32_t* szw = reinterpret_cast<uint32_t*>(out.sz[which]);
+    const uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
+    szw[(row * H + h) * (hd / g) + e0 / g] = pair;
+  }
+}
+
+// One warp per (row, head): K and V together, so the loads of both (inputs, the slot rows
+// and the chain codes) are in flight at once.
 template <int EPL, typename T>
 __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int loop,
                                                   const T* __restrict__ k_new,
@@ -60,86 +123,43 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
   griddep_wait();
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int H = kv.H, hd = kv.hd, g = kv.g;
-  if (gw >= n_act * H * 2) return;
-  const int which = gw % 2;
-  const int h = (gw / 2) % H;
-  const int i = gw / (2 * H);
+  const int H = kv.H, hd = kv.hd;
+  if (gw >= n_act * H) return;
+  const int h = gw % H;
+  const int i = gw / H;
   const int t = act_tok ? act_tok[i] : i;
   if (t < 0 || t >= kv.n_tok) {
     if (lane == 0) record_error(st, FL_ERR_RANGE);
     return;
   }
   const int e0 = lane * EPL;
-  const T* src = (which == 0 ? k_new : v_new) + ((size_t)i * H + h) * hd + e0;
-  float xin[EPL];
+  const size_t off = ((size_t)i * H + h) * hd + e0;
+  float xin[2][EPL];
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) xin[j] = to_f32<T>(src[j]);
-
+  for (int j = 0; j < EPL; ++j) {
+    xin[0][j] = to_f32<T>(k_new[off + j]);
+    xin[1][j] = to_f32<T>(v_new[off + j]);
+  }
   const int bits = loop == 1 ? kv.base_bits : kv.res_bits[loop];
-  float prev[EPL];
-  float x[EPL];
+  float prev[2][EPL], x[2][EPL];
   if (loop >= 2) {
-    reconstruct_warp<EPL>(kv, which, loop - 1, t, h, e0, lane, prev);
+    reconstruct_warp<EPL>(kv, 0, loop - 1, t, h, e0, lane, prev[0]);
+    reconstruct_warp<EPL>(kv, 1, loop - 1, t, h, e0, lane, prev[1]);
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) x[j] = bits == 0 ? xin[j] : __fsub_rn(xin[j], prev[j]);
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) x[w][j] = bits == 0 ? xin[w][j] : __fsub_rn(xin[w][j], prev[w][j]);
   } else {
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) x[j] = xin[j];
+    for (int w = 0; w < 2; ++w)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) { x[w][j] = xin[w][j]; prev[w][j] = 0.f; }
   }
-  const int row = loop == 1 ? t : out.row0 + i;
+  const size_t row = loop == 1 ? (size_t)t : (size_t)out.row0 + i;
   float hat[EPL];
-  if (bits == 0) {
-    float* dst = reinterpret_cast<float*>(out.codes[which]) + ((size_t)row * H + h) * hd + e0;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) { dst[j] = xin[j]; hat[j] = xin[j]; }
-  } else {
-    const int LPG = g / EPL;  // lanes per group
-    float mn = x[0], mx = x[0];
-#pragma unroll
-    for (int j = 1; j < EPL; ++j) { mn = fminf(mn, x[j]); mx = fmaxf(mx, x[j]); }
-    for (int o = 1; o < LPG; o <<= 1) {
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    const __half zh = __float2half_rd(mn);
-    const float zf = __half2float(zh);
-    const float qmax = (float)((1 << bits) - 1);
-    const float t1 = __fsub_ru(mx, zf);
-    const float t2 = __fdiv_ru(t1, qmax);
-    const __half sh = __float2half_ru(t2);
-    const float sf = __half2float(sh);
-    const bool bad = isinf(zf) || isinf(sf) || isnan(zf) || isnan(sf);
-    if (bad && (lane % LPG) == 0) record_error(st, FL_ERR_RANGE);
-    uint32_t word = 0;
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      int code = 0;
-      if (!bad && sf != 0.f) {
-        const float w = __fdiv_rn(__fsub_rn(x[j], zf), sf);
-        code = (int)fminf(fmaxf(rintf(w), 0.f), qmax);
-      }
-      const float deq = __fmaf_rn((float)code, sf, zf);
-      hat[j] = loop == 1 ? deq : __fadd_rn(prev[j], deq);
-      word |= (uint32_t)code << (j * bits);
-    }
-    // combine the lanes that share one 32-bit output word
-    const int wbits = EPL * bits;
-    const int LPW = 32 / wbits;
-    word <<= (lane % LPW) * wbits;
-    for (int o = 1; o < LPW; o <<= 1) word |= __shfl_xor_sync(0xffffffffu, word, o);
-    const size_t rowbytes = (size_t)hd * bits / 8;
-    if (lane % LPW == 0) {
-      uint32_t* cw = reinterpret_cast<uint32_t*>(out.codes[which] + ((size_t)row * H + h) * rowbytes);
-      cw[lane / LPW] = word;
-    }
-    if (lane % LPG == 0) {
-      uint32_t* szw = reinterpret_cast<uint32_t*>(out.sz[which]);
-      const uint32_t pair = (uint32_t)__half_as_ushort(sh) | ((uint32_t)__half_as_ushort(zh) << 16);
-      szw[((size_t)row * H + h) * (hd / g) + e0 / g] = pair;
-    }
-  }
-  if (which == 1 && out.vnorm) {
+  quant_store<EPL>(kv, out, 0, loop, bits, row, h, e0, lane, xin[0], x[0], prev[0], hat, st);
+  quant_store<EPL>(kv, out, 1, loop, bits, row, h, e0, lane, xin[1], x[1], prev[1], hat, st);
+  if (out.vnorm) {   // ||V^|| from the V reconstruction (hat of the second call)
     float ss = 0.f;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) ss = fmaf(hat[j], hat[j], ss);
@@ -147,14 +167,14 @@ __global__ void __launch_bounds__(256) k_kv_quant(KvView kv, QuantOut out, int l
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if (lane == 0) out.vnorm[(size_t)t * H + h] = sqrtf(ss);
   }
-  if (loop >= 2 && which == 0 && h == 0 && lane == 0 && out.slot_row) out.slot_row[t] = row;
+  if (loop >= 2 && h == 0 && lane == 0 && out.slot_row) out.slot_row[t] = (int32_t)row;
 }
 
 template <int EPL>
 cudaError_t launch_epl(const KvView& v, const QuantOut& o, int loop, const void* k,
                        const void* vv, fl_dtype dt, const int32_t* act, int n_act, int* st,
                        cudaStream_t s) {
-  const size_t warps = (size_t)n_act * v.H * 2;
+  const size_t warps = (size_t)n_act * v.H;
   const int blocks = (int)((warps * 32 + 255) / 256);
   const cudaError_t e =
       dt == FL_F32

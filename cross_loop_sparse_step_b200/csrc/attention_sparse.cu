@@ -39,7 +39,7 @@ namespace {
 
 constexpr int NW = 4;              // warps per CTA
 // resident CTAs per SM the register budget is cut for (no spills at either setting)
-__host__ __device__ constexpr int min_ctas(bool shrink) { return shrink ? 3 : 5; }
+__host__ __device__ constexpr int min_ctas(bool shrink) { return shrink ? 3 : 6; }
 constexpr int ITEM_BYTES = 11;     // u16 column index + u8 loop + i32 row + f32 logit part
 constexpr int ITEM_BUDGET = 6144;  // per-warp bytes for residual items beyond one loop's
 

@@ -157,7 +157,13 @@ def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
     sched = fl.make_schedule(R, cfg["first_sparse"], n_active, col_k)
     run = fl.LoopRunner(model, sched, n_active, stores, max(col_k.values()) + 1)
     run.h.copy_(torch.from_numpy(synth.embeddings(g, N, d)).to(dev))
-    run.step(1)
+    torch.cuda.synchronize()
+    t1 = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+    t1[0].record()
+    run.step(1)   # the dense loop: the statistics producer for loop 2 (timed once, cold)
+    t1[1].record()
+    torch.cuda.synchronize()
+    loop1_ms = t1[0].elapsed_time(t1[1])
     cur, prev, _ = synth.pareto_delta_pair(g, N, d, 2)
     run.x_prev.copy_(run.h - torch.from_numpy((cur - prev).astype(np.float32)).to(dev))
     st = fl.check_device_status()
@@ -165,7 +171,7 @@ def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
         raise RuntimeError(f"loop 1 reported {fl.status_str(st)}")
     snap = (run.h.clone(), run.x_prev.clone())
     return dict(run=run, stores=stores, model=model, layers=layers, n_active=n_active, snap=snap,
-                L=L, R=R, N=N, d=d, H=H, hd=hd, F=F, col_k=col_k, res=res)
+                L=L, R=R, N=N, d=d, H=H, hd=hd, F=F, col_k=col_k, res=res, loop1_ms=loop1_ms)
 
 
 def step_loops(W):
@@ -536,6 +542,7 @@ def main():
             "gpu_launches": int(launches),
             "launch_mode": "cuda-graph replay" if graph is not None else "eager",
             "clocks": clk,
+            "loop1_ms": round(W["loop1_ms"], 3),   # dense loop 1 incl. statistics, one cold run
             "kv_bytes_per_token_per_layer": kvb,
             "kv_dense_bytes_per_token_per_layer": dense,
             "kv_reduction": dense / kvb,

@@ -5,7 +5,9 @@
 // Four lanes per column (a lane owns a quarter of the head slice, one quantisation group
 // at head_dim 128), sixteen columns in flight per warp (two per lane group per step):
 //   K pass   s_j = (sum over parts of s (q . codes) + z sum(q)) / sqrt(hd) + b_j for
-//            j = 0..t, kept in shared memory;
+//            j = 0..t, kept in shared memory; the q . codes dot products of 16 columns
+//            per step run as warp-level tensor-core MMAs with exact operands (codes as
+//            fp16 c * 2^-24, q as scaled hi + lo fp16; attn_mma.cuh);
 //   softmax  p_j;
 //   select   (when statistics are asked for and t > k) top-k of c_j = p_j ||V^_j||
 //            (or p_j) over j = 1..t by a warp radix select on the binary32 bits, equal
@@ -15,6 +17,7 @@
 // Used for loop 1 over an 8-bit base; other cases take the general kernel.
 #include <float.h>
 
+#include "attn_mma.cuh"
 #include "fl_internal.cuh"
 #include "sm100_f32x2.cuh"
 
@@ -26,6 +29,12 @@ __host__ __device__ inline size_t a16(size_t x) { return (x + 15) & ~size_t(15);
 // Per-warp shared memory: p [n_tok] f32 | mark [n_tok] u8 | hist [256] i32.
 __host__ __device__ inline size_t dense_warp_smem(int n_tok) {
   return a16((size_t)n_tok * 4) + a16((size_t)n_tok) + 256 * 4;
+}
+
+__device__ __forceinline__ void load_sz_pair(const uint16_t* sz, size_t idx, float* s, float* z) {
+  const uint32_t pair = reinterpret_cast<const uint32_t*>(sz)[idx];
+  *s = half_bits_to_float((uint16_t)(pair & 0xFFFFu));
+  *z = half_bits_to_float((uint16_t)(pair >> 16));
 }
 
 // 8-bit codes [e0, e0 + EL) of one base row as pairs, and the row's (s, z) for them.
@@ -65,9 +74,11 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
     return;
   }
   const int n_cols = t + 1;
-  float2 qv[EL / 2];
-  float qsum = 0.f;
+  constexpr int KS = HD / 16;
+  float qsum = 0.f, dot_unscale;
+  uint32_t bq[KS][2];
   {
+    float qx[EL];
     const size_t off = ((size_t)qi * H + h) * HD + e0;
 #pragma unroll
     for (int k = 0; k < EL / 2; ++k) {
@@ -81,24 +92,38 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
         a = v.x;
         b = v.y;
       }
-      qv[k] = make_float2(a, b);
+      qx[2 * k] = a;
+      qx[2 * k + 1] = b;
       qsum += a + b;
     }
+    dot_unscale = mma::q_fragments<HD>(qx, lane, bq);
   }
 
-  // ---- K pass
+  // ---- K pass: 16 columns per step; lane (g, l) loads quarter l of columns i0 + g and
+  // i0 + 8 + g (columns past t read column 0 and are masked)
   float lmax = -FLT_MAX;
   for (int i0 = 0; i0 < n_cols; i0 += 16) {
-    float part[2] = {0.f, 0.f};
+    Raw<EL> raw[2];
+    float sb[2], zb[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int c = i0 + 8 * u + cg;
-      if (c < n_cols) {
-        float2 cf[EL / 2];
-        float s, z;
-        base_part<EL>(kv, 0, (size_t)c * H + h, e0, gidx, ngrp, cf, &s, &z);
-        part[u] = fmaf(s, f2::dot_pairs<EL>(qv, cf), z * qsum);
-      }
+      const int col = i0 + 8 * u + cg;
+      const uint32_t bh = (uint32_t)(col < n_cols ? col : 0) * H + h;
+      load_sz_pair(kv.sz[0][1], (size_t)bh * ngrp + gidx, &sb[u], &zb[u]);
+      load_raw<EL>(kv.codes[0][1] + (size_t)bh * HD, 8, e0, raw[u]);
+    }
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const uint32_t w0 = raw_word(raw[0], ks), w1 = raw_word(raw[1], ks);
+      mma::m16n8k16(d, mma::code_pair(w0, 0, 1), mma::code_pair(w1, 0, 1),
+                    mma::code_pair(w0, 2, 3), mma::code_pair(w1, 2, 3), bq[ks][0], bq[ks][1]);
+    }
+    float part[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float dot = (d[2 * u] + d[2 * u + 1]) * dot_unscale;
+      part[u] = i0 + 8 * u + cg < n_cols ? fmaf(sb[u], dot, zb[u] * qsum) : 0.f;
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {

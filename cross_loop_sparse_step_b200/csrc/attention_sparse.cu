@@ -70,57 +70,6 @@ __device__ __forceinline__ void load_sz(const uint16_t* sz, size_t idx, float* s
   *z = half_bits_to_float((uint16_t)(pair >> 16));
 }
 
-// This lane's EL codes [e0, e0 + EL) of a stored row, as raw words (EL * bits / 8 bytes,
-// at most 32): loaded first, decoded later, so several rows' loads can be in flight.
-template <int EL>
-struct Raw {
-  uint4 w[EL / 16];
-};
-
-template <int EL>
-__device__ __forceinline__ void load_raw(const uint8_t* row, int bits, int e0, Raw<EL>& r) {
-  const uint8_t* src = row + (size_t)e0 * bits / 8;
-  if (bits == 8) {
-#pragma unroll
-    for (int k = 0; k < EL / 16; ++k) r.w[k] = reinterpret_cast<const uint4*>(src)[k];
-  } else if (bits == 4) {   // EL / 2 bytes
-    if constexpr (EL == 32) {
-      r.w[0] = *reinterpret_cast<const uint4*>(src);
-    } else {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
-    }
-  } else {                  // 2 bits: EL / 4 bytes
-    if constexpr (EL == 32) {
-      const uint2 u = *reinterpret_cast<const uint2*>(src);
-      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
-    } else {
-      r.w[0] = make_uint4(*reinterpret_cast<const uint32_t*>(src), 0u, 0u, 0u);
-    }
-  }
-}
-
-template <int EL>
-__device__ __forceinline__ uint32_t raw_word(const Raw<EL>& r, int i) {
-  const uint4 u = r.w[i >> 2];
-  return (i & 3) == 0 ? u.x : (i & 3) == 1 ? u.y : (i & 3) == 2 ? u.z : u.w;
-}
-
-// This lane's EL codes as one code per byte (EL / 4 words), from raw words of `bits` bits.
-template <int EL>
-__device__ __forceinline__ void to_bytes(const Raw<EL>& r, int bits, uint32_t* wb) {
-  if (bits == 8) {
-#pragma unroll
-    for (int i = 0; i < EL / 4; ++i) wb[i] = raw_word(r, i);
-  } else if (bits == 4) {
-#pragma unroll
-    for (int i = 0; i < EL / 8; ++i) mma::spread4(raw_word(r, i), wb + 2 * i);
-  } else {
-#pragma unroll
-    for (int i = 0; i < EL / 16; ++i) mma::spread2(raw_word(r, i), wb + 4 * i);
-  }
-}
-
 // o[j] += w * code[j]
 template <int EL>
 __device__ __forceinline__ void axpy_raw(float w, const Raw<EL>& r, int bits, float2* o) {
@@ -210,11 +159,9 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
     n_cols += __popc(__ballot_sync(0xffffffffu, c != FL_SENTINEL));
   }
   const float m_in = P.mass[(size_t)h * P.stat_rows + srow];
-  // this lane's quarter of q; the score MMAs take it as hi + lo fp16 parts scaled by
-  // qscale, lane (g, l) feeding column n = g of B (hi for even g, lo for odd g) with
-  // quarter g / 2 and zeros elsewhere, so column pair (2l, 2l + 1) of D is quarter l's dot
+  // this lane's quarter of q, and the score MMAs' B fragments made from it
   constexpr int KS = HD / 16;
-  float qsum = 0.f, qmax = 0.f;
+  float qsum = 0.f;
   uint32_t bq[KS][2];
   {
     float qx[EL];
@@ -235,25 +182,8 @@ __device__ __forceinline__ void attn_sparse_warp(const AttnParams& P, int gw, ui
       qx[2 * k] = a;
       qx[2 * k + 1] = b;
       qsum += a + b;
-      qmax = fmaxf(qmax, fmaxf(fabsf(a), fabsf(b)));
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
-    const float qscale = mma::pow2_scale_for(qmax, 14);
-    const bool feeds = l4 == (cg >> 1);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      __half part[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __half lo;
-        const __half hi = mma::split_hi(qx[4 * ks + j] * qscale, &lo);
-        part[j] = (cg & 1) ? lo : hi;
-      }
-      bq[ks][0] = feeds ? mma::pack_h2(part[0], part[1]) : 0u;
-      bq[ks][1] = feeds ? mma::pack_h2(part[2], part[3]) : 0u;
-    }
-    dot_unscale = mma::kCodeUnscale / qscale;   // a power of two
+    dot_unscale = mma::q_fragments<HD>(qx, lane, bq);
   }
   __syncwarp();
 

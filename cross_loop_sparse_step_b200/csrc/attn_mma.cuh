@@ -72,5 +72,89 @@ __device__ __forceinline__ void spread2(uint32_t w, uint32_t* out) {
   out[3] = __byte_perm(b01, b23, 0x7632);
 }
 
+// The score MMAs' B operand from this lane's quarter qx[HD / 4] of q (lane (g, l) of the
+// warp, g = lane / 4, l = lane % 4): q scaled by a power of two into [2^13, 2^14) and split
+// into hi + lo fp16; lane (g, l) feeds column n = g of B (hi for even g, lo for odd g)
+// with quarter g / 2 and zeros elsewhere, so D column pair (2l, 2l + 1) is quarter l's
+// dot. Over k-step ks a lane's logical k {2l, 2l+1, 2l+8, 2l+9} are its elements
+// 4 ks .. 4 ks + 3. Returns the factor that turns D back into dot products of codes.
+template <int HD>
+__device__ __forceinline__ float q_fragments(const float* qx, int lane, uint32_t (*bq)[2]) {
+  constexpr int KS = HD / 16;
+  float qmax = 0.f;
+#pragma unroll
+  for (int j = 0; j < HD / 4; ++j) qmax = fmaxf(qmax, fabsf(qx[j]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) qmax = fmaxf(qmax, __shfl_xor_sync(0xffffffffu, qmax, o));
+  const float qscale = pow2_scale_for(qmax, 14);
+  const int cg = lane >> 2, l4 = lane & 3;
+  const bool feeds = l4 == (cg >> 1);
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    __half part[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __half lo;
+      const __half hi = split_hi(qx[4 * ks + j] * qscale, &lo);
+      part[j] = (cg & 1) ? lo : hi;
+    }
+    bq[ks][0] = feeds ? pack_h2(part[0], part[1]) : 0u;
+    bq[ks][1] = feeds ? pack_h2(part[2], part[3]) : 0u;
+  }
+  return kCodeUnscale / qscale;   // a power of two
+}
+
 }  // namespace mma
+
+// This lane's EL codes [e0, e0 + EL) of a stored row, as raw words (EL * bits / 8 bytes,
+// at most 32): loaded first, decoded later, so several rows' loads can be in flight.
+template <int EL>
+struct Raw {
+  uint4 w[EL / 16];
+};
+
+template <int EL>
+__device__ __forceinline__ void load_raw(const uint8_t* row, int bits, int e0, Raw<EL>& r) {
+  const uint8_t* src = row + (size_t)e0 * bits / 8;
+  if (bits == 8) {
+#pragma unroll
+    for (int k = 0; k < EL / 16; ++k) r.w[k] = reinterpret_cast<const uint4*>(src)[k];
+  } else if (bits == 4) {   // EL / 2 bytes
+    if constexpr (EL == 32) {
+      r.w[0] = *reinterpret_cast<const uint4*>(src);
+    } else {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
+    }
+  } else {                  // 2 bits: EL / 4 bytes
+    if constexpr (EL == 32) {
+      const uint2 u = *reinterpret_cast<const uint2*>(src);
+      r.w[0] = make_uint4(u.x, u.y, 0u, 0u);
+    } else {
+      r.w[0] = make_uint4(*reinterpret_cast<const uint32_t*>(src), 0u, 0u, 0u);
+    }
+  }
+}
+
+template <int EL>
+__device__ __forceinline__ uint32_t raw_word(const Raw<EL>& r, int i) {
+  const uint4 u = r.w[i >> 2];
+  return (i & 3) == 0 ? u.x : (i & 3) == 1 ? u.y : (i & 3) == 2 ? u.z : u.w;
+}
+
+// This lane's EL codes as one code per byte (EL / 4 words), from raw words of `bits` bits.
+template <int EL>
+__device__ __forceinline__ void to_bytes(const Raw<EL>& r, int bits, uint32_t* wb) {
+  if (bits == 8) {
+#pragma unroll
+    for (int i = 0; i < EL / 4; ++i) wb[i] = raw_word(r, i);
+  } else if (bits == 4) {
+#pragma unroll
+    for (int i = 0; i < EL / 8; ++i) mma::spread4(raw_word(r, i), wb + 2 * i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < EL / 16; ++i) mma::spread2(raw_word(r, i), wb + 4 * i);
+  }
+}
+
 }  // namespace fl

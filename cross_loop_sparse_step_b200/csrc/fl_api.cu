@@ -399,6 +399,9 @@ fl_status fl_kv_append(const fl_kv_desc* kv, int32_t loop, const void* k_new, co
   FL_CHECK(valid_dt(dt), FL_ERR_UNSUPPORTED);
   FL_CHECK(loop >= 1 && loop <= kv->n_loops, FL_ERR_SHAPE);
   FL_CHECK(n_act >= 0 && n_act <= kv->n_tok && row0 >= 0, FL_ERR_SHAPE);
+  // a residual loop holds at most one row per token: rows row0 .. row0 + n_act - 1 must
+  // lie below n_tok (checked in 64 bits, before any launch)
+  if (loop >= 2) FL_CHECK((int64_t)row0 + n_act <= (int64_t)kv->n_tok, FL_ERR_SHAPE);
   if (n_act == 0) return FL_OK;
   const int bits = loop == 1 ? kv->base_bits : kv->res_bits[loop];
   FL_CHECK(kv->codes[0][loop] && kv->codes[1][loop], FL_ERR_INVALID_ARG);
@@ -564,6 +567,10 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
              st->kv[l].head_dim == m->head_dim && st->kv[l].n_loops >= R, FL_ERR_SHAPE);
   }
   if (loop >= 2) FL_CHECK(st->act[loop] && st->act_pos, FL_ERR_INVALID_ARG);
+  if (st->taps) {
+    FL_CHECK(st->taps->n >= 0, FL_ERR_SHAPE);
+    FL_CHECK(st->taps->n == 0 || st->taps->tok, FL_ERR_INVALID_ARG);
+  }
 
   cudaStream_t s = S(stream);
   int* sw = status_word();
@@ -608,14 +615,26 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
   }
   rc = prepare_rope(m, blk, s);
   if (rc != FL_OK) return rc;
+  // inspection taps: rows of the tapped tokens, per layer, into the caller's buffers
+  const fl_loop_taps* tp = st->taps;
+  const bool tap = tp && tp->n > 0;
+  auto tap_rows = [&](const void* src, void* base, size_t row_bytes, int l) -> cudaError_t {
+    if (!tap || !base) return cudaSuccess;
+    return launch_tap_rows(act, M, tp->tok, tp->n, src,
+                           static_cast<uint8_t*>(base) + (size_t)l * tp->n * row_bytes, row_bytes,
+                           s);
+  };
   for (int l = 0; l < L; ++l) {
+    FL_TRY(tap_rows(X, tap ? tp->x_in : nullptr, row_bytes, l));
     // Loop 1 writes the base codes in the projection epilogue. Later loops quantise the
     // residual against K^_{r-1}, whose chain decode is a string of dependent gathers; in
     // the four epilogue warps of the GEMM those stall the tensor pipe (measured: the fused
     // QKV launch took 2.1x the projection plus the separate quantiser), so they keep the
     // separate, wider quantiser launch.
     if (loop == 1 && kv_fusable(m, M, &st->kv[l], loop)) {
-      rc = run_qkv(m, l, X, M, act, q, nullptr, nullptr, blk, s, &st->kv[l], loop);
+      const bool keep_kv = tap && (tp->k || tp->v);   // a tapped step also stores k and v
+      rc = run_qkv(m, l, X, M, act, q, keep_kv ? k : nullptr, keep_kv ? v : nullptr, blk, s,
+                   &st->kv[l], loop);
       if (rc != FL_OK) return rc;
     } else {
       rc = run_qkv(m, l, X, M, act, q, k, v, blk, s);
@@ -637,9 +656,14 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
       a.stat_kind = sc->stat_kind;
     }
     a.out = attn; a.out_dt = m->dt;
+    FL_TRY(tap_rows(q, tap ? tp->q : nullptr, row_bytes, l));
+    FL_TRY(tap_rows(k, tap ? tp->k : nullptr, row_bytes, l));
+    FL_TRY(tap_rows(v, tap ? tp->v : nullptr, row_bytes, l));
     FL_TRY(launch_attention_timed(a, sw, s));
+    FL_TRY(tap_rows(attn, tap ? tp->attn : nullptr, (size_t)d * dt_size(m->dt), l));
     rc = run_out_ffn(m, l, X, M, attn, blk, s);
     if (rc != FL_OK) return rc;
+    FL_TRY(tap_rows(X, tap ? tp->x_out : nullptr, row_bytes, l));
   }
   if (loop >= 2)
     FL_TRY(launch_gather_scatter(FL_SCATTER, st->x_cur, st->h, act, M, N, row_bytes, sw, s));

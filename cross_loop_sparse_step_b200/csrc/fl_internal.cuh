@@ -212,6 +212,10 @@ cudaError_t launch_rope_table(float2* tab, int n_tok, int hd, float theta, cudaS
 cudaError_t launch_swiglu(const float* gu, int M, int F, void* out, fl_dtype dt,
                           cudaStream_t s);
 cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s);
+// Copies the rows of the tokens tok[0, n) found in the ascending list act[0, M) from src
+// (row p = act position p) to dst row i; tokens not in act are skipped.
+cudaError_t launch_tap_rows(const int32_t* act, int M, const int32_t* tok, int n,
+                            const void* src, void* dst, size_t row_bytes, cudaStream_t s);
 cudaError_t launch_fill_i32(int32_t* p, int32_t v, size_t n, cudaStream_t s);
 
 }  // namespace fl

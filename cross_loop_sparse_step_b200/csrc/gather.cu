@@ -34,6 +34,25 @@ __global__ void k_fill_i32(int32_t* p, int32_t v, size_t n) {
     p[i] = v;
 }
 
+// Tap copy: block i finds token tok[i] in the ascending row-token list act[0, M) by
+// binary search and copies that row of src to row i of dst; absent tokens are skipped.
+__global__ void __launch_bounds__(128) k_tap_rows(const int32_t* __restrict__ act, int M,
+                                                  const int32_t* __restrict__ tok,
+                                                  const uint8_t* __restrict__ src,
+                                                  uint8_t* __restrict__ dst, size_t row_bytes) {
+  const int t = tok[blockIdx.x];
+  int lo = 0, hi = M;   // first position with act[pos] >= t
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (act[mid] < t) lo = mid + 1;
+    else hi = mid;
+  }
+  if (lo >= M || act[lo] != t) return;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)lo * row_bytes);
+  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)blockIdx.x * row_bytes);
+  for (size_t e = threadIdx.x; e < row_bytes / 16; e += blockDim.x) d[e] = s[e];
+}
+
 __global__ void k_iota(int32_t* p, int n) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
     p[i] = i;
@@ -56,6 +75,15 @@ cudaError_t launch_gather_scatter(fl_gs_op op, const void* src, void* dst, const
   else
     k_gather_scatter<uint16_t><<<n_idx, 256, 0, s>>>(op, (const uint8_t*)src, (uint8_t*)dst,
                                                      idx, n_full, row_bytes, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tap_rows(const int32_t* act, int M, const int32_t* tok, int n,
+                            const void* src, void* dst, size_t row_bytes, cudaStream_t s) {
+  if (n <= 0 || M <= 0 || !dst) return cudaSuccess;
+  if (row_bytes % 16 || (uintptr_t)src % 16 || (uintptr_t)dst % 16) return cudaErrorInvalidValue;
+  k_tap_rows<<<n, 128, 0, s>>>(act, M, tok, (const uint8_t*)src, (uint8_t*)dst, row_bytes);
   count_launch();
   return cudaGetLastError();
 }

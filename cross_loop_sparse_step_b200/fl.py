@@ -73,6 +73,11 @@ class Schedule(ctypes.Structure):
                 ("stat_kind", c_i32)]
 
 
+class LoopTaps(ctypes.Structure):
+    _fields_ = [("n", c_i32), ("tok", vp), ("x_in", vp), ("q", vp), ("k", vp), ("v", vp),
+                ("attn", vp), ("x_out", vp)]
+
+
 class LoopState(ctypes.Structure):
     _fields_ = [
         ("h", vp), ("x_cur", vp), ("x_prev", vp),
@@ -80,6 +85,7 @@ class LoopState(ctypes.Structure):
         ("kv", ctypes.POINTER(KvDesc)),
         ("sel", ctypes.POINTER(vp)), ("mass", ctypes.POINTER(vp)), ("unsel", ctypes.POINTER(vp)),
         ("sel_stride", c_i32), ("ws", vp), ("ws_bytes", c_sz),
+        ("taps", ctypes.POINTER(LoopTaps)),
     ]
 
 
@@ -379,6 +385,31 @@ class LoopRunner:
         st.sel_stride = sel_stride
         st.ws, st.ws_bytes = self.ws.data_ptr(), nb
         self.c = st
+
+    def set_taps(self, tok):
+        """Inspection taps (fl_loop_taps) for the tokens ``tok`` (int32 device tensor):
+        every later step copies each layer's input, q, k, v, attention output and
+        output rows of those tokens into ``self.taps`` ([L, n, d] tensors). None turns
+        them off."""
+        if tok is None:
+            self.taps, self._taps = None, None
+            self.c.taps = ctypes.POINTER(LoopTaps)()
+            return None
+        c = self.model.c
+        L, n, d = c.n_layers, tok.numel(), c.d_model
+        dev = tok.device
+        adt = torch.bfloat16 if c.dt == BF16 else torch.float32
+        self.taps = {k: torch.full((L, n, d), float("nan"), dtype=torch.float32, device=dev)
+                     for k in ("x_in", "q", "k", "v", "x_out")}
+        self.taps["attn"] = torch.full((L, n, d), float("nan"), dtype=adt, device=dev)
+        self.taps["tok"] = tok
+        t = LoopTaps()
+        t.n, t.tok = n, tok.data_ptr()
+        for k in ("x_in", "q", "k", "v", "attn", "x_out"):
+            setattr(t, k, self.taps[k].data_ptr())
+        self._taps = t
+        self.c.taps = ctypes.pointer(t)
+        return self.taps
 
     def step(self, loop, stream=None):
         _ok(_loop(ctypes.byref(self.model.c), ctypes.byref(self.c), ctypes.byref(self.sched), loop,

@@ -105,7 +105,11 @@ fl_status fl_select_active(const void* h_cur, const void* h_prev, fl_dtype dt,
  * (256 KiB) built into the library, which every GPU that loads the library holds until
  * the process exits. n_rows above that maximum returns FL_ERR_SHAPE without launching.
  * The first call on a device looks up the scratch array's device address (with that
- * device current) and caches it: make that first call before any stream capture.
+ * device current) and caches it: make that first call before any stream capture. The
+ * cached address belongs to the device's primary context: after cudaDeviceReset (or
+ * anything else that destroys that context) it is stale, so do not call this entry point
+ * again in that process. The device status word of every entry point is cached the
+ * same way.
  * Every call on a device shares the one scratch array, so calls whose work overlaps on
  * the GPU (other streams or host threads) race; the caller must serialise them. No
  * scratch content has to survive between calls. Calls no allocator of any kind. */
@@ -306,6 +310,22 @@ typedef struct {
   int32_t stat_kind;                     /* fl_stat_kind */
 } fl_schedule;
 
+/* Inspection taps of fl_loop_step, for stage-by-stage checks of a loop against a
+ * reference on identical inputs (NULL in normal use; a tapped step launches extra
+ * copy kernels and, at loop 1, also stores the projection's k and v). For each of the
+ * n tokens tok[i] (device int32, any order) that the loop recomputes, row i of layer l
+ * (at offset (l * n + i) * d elements) receives, for every non-NULL buffer:
+ *   x_in   the layer's input row (float)        q, k, v  post-RoPE projections (float)
+ *   attn   the attention output (dtype m->dt)   x_out    the layer's output row (float)
+ * Rows of tokens the loop does not recompute are not written. */
+typedef struct {
+  int32_t n;
+  const int32_t* tok;
+  float* x_in; float* q; float* k; float* v;
+  void* attn;
+  float* x_out;
+} fl_loop_taps;
+
 typedef struct {
   float* h;            /* device [n_tok][d]: h_{r-1} on entry, h_r on return. Before
                           loop 1 the caller writes the embeddings h_0 here. */
@@ -322,6 +342,7 @@ typedef struct {
   float** unsel;       /* HOST array [n_layers] of device [H][n_tok][hd] */
   int32_t sel_stride;  /* >= max col_k + 1 */
   void* ws; size_t ws_bytes;
+  const fl_loop_taps* taps;  /* HOST pointer, nullable: inspection copies (see above) */
 } fl_loop_state;
 
 size_t fl_loop_step_workspace_bytes(const fl_model* m, const fl_schedule* s);

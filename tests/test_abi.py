@@ -51,7 +51,9 @@ int main(void) {
   F(fl_schedule, n_active) F(fl_schedule, col_k) F(fl_schedule, stat_kind)
   printf("fl_loop_state %zu\n", sizeof(fl_loop_state));
   F(fl_loop_state, act) F(fl_loop_state, act_pos) F(fl_loop_state, kv) F(fl_loop_state, sel_stride)
-  F(fl_loop_state, ws) F(fl_loop_state, ws_bytes)
+  F(fl_loop_state, ws) F(fl_loop_state, ws_bytes) F(fl_loop_state, taps)
+  printf("fl_loop_taps %zu\n", sizeof(fl_loop_taps));
+  F(fl_loop_taps, tok) F(fl_loop_taps, x_in) F(fl_loop_taps, attn) F(fl_loop_taps, x_out)
   return 0;
 }
 """
@@ -67,7 +69,8 @@ def test_struct_layouts_match_c():
         lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
     c = dict(l.rsplit(" ", 1) for l in lines if l.strip())
     py = {"fl_kv_desc": fl.KvDesc, "fl_attn_args": fl.AttnArgs, "fl_layer_weights": fl.LayerWeights,
-          "fl_model": fl.Model, "fl_schedule": fl.Schedule, "fl_loop_state": fl.LoopState}
+          "fl_model": fl.Model, "fl_schedule": fl.Schedule, "fl_loop_state": fl.LoopState,
+          "fl_loop_taps": fl.LoopTaps}
     for key, val in c.items():
         if "." in key:
             s, m = key.split(".")
@@ -101,5 +104,8 @@ def test_host_validation_without_gpu():
     assert fl._quant(ctypes.byref(kv), 1, p, p, 0, p, 8, None) == 2      # act_tok at loop 1
     assert fl._quant(ctypes.byref(kv), 3, p, p, 0, p, 8, None) == 2      # loop > n_loops
     assert fl._quant(ctypes.byref(kv), 1, p, p, 0, None, 8, None) == 1   # no code buffers
+    # decode append past the residual capacity (one row per token): rejected, no launch
+    assert fl._append(ctypes.byref(kv), 2, p, p, 0, p, 4, 5, None) == 2
+    assert fl._append(ctypes.byref(kv), 2, p, p, 0, p, 1, 2 ** 31 - 1, None) == 2
     a = fl.AttnArgs()
     assert fl._attn(ctypes.byref(a), None) == 1

@@ -3,9 +3,9 @@
 * the tiny fp32 looped block over R = 4 loops (and its shrinking-budget variant):
   active sets bit-exact, hidden states, carried statistics and the dequantised KV
   store within tolerance after every loop;
-* the 4K-token Ouro-1.4B shape (d 2048, 16 x 128 heads, FFN 5632, bf16) with two
-  layers over two loops: loop-2 selection bit-exact, sampled rows of h_2 within
-  tolerance;
+* the 4K-token Ouro-1.4B shape (d 2048, 16 x 128 heads, FFN 5632) in binary32 with
+  two layers over two loops, free-running: loop-2 selection bit-exact, sampled rows of
+  h_2 within tolerance;
 * the full 24-layer 4K workload in the configuration the benchmark times: the
   invariants of the method (nested sets of the scheduled size, inactive rows and
   their KV untouched, carried column sets valid, KV bytes equal to the closed form)."""
@@ -114,28 +114,17 @@ def _c2_like(n_layers):
     return cfg
 
 
-# Tolerance of a bf16 chain of layers against the fp64 oracle. Each stage matches on
-# identical inputs (relative L1 ~1e-5, see test_gpu_kernels); across layers a 1e-4
-# difference flips bf16 operand roundings (one ulp, 2^-8 relative) and int8 KV codes
-# (one step, range/255) in the next layer, so differences compound with the number of
-# layer applications on the path. Measured: two applications (h_1) relative L1 2.2e-3,
-# max-abs 2.2e-2; four (h_2 of the active rows) 3.3e-3, 5.3e-2. The chained bf16 check
-# keeps the spec relative L1 (5e-3) and allows max-abs 2.5e-2 per layer
-# application; the fp32 run of the same shape holds the benchmark spec's 2e-2 / 5e-3 exactly.
-CHAIN_BF16_MAX_ABS_PER_LAYER = 2.5e-2
-
-
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_4k_shape_two_layers_two_loops(dtype):
-    """Full 4K shape, two layers, loops 1 and 2: loop-2 selection bit-exact, sampled
-    rows of h_2 within tolerance."""
+def test_4k_shape_two_layers_two_loops_fp32():
+    """Full 4K shape in binary32, two layers, loops 1 and 2, free-running against the
+    oracle's own chain: loop-2 selection bit-exact, h_1 and sampled rows of h_2 within
+    the standard tolerance. (The bf16 workload is checked stage by stage on identical
+    inputs in test_gpu_teacher_forced.)"""
+    dtype = "f32"
     from cross_loop_sparse_step_b200 import fl
     cfg = _c2_like(2)
     cfg["n_loops"] = 2
     cfg["dtype"] = dtype
-    bf16 = dtype == "bf16"
-    tol1 = CHAIN_BF16_MAX_ABS_PER_LAYER * 2 if bf16 else 2e-2   # h_1: 2 layer applications
-    tol2 = CHAIN_BF16_MAX_ABS_PER_LAYER * 4 if bf16 else 2e-2   # h_2: 4 on the active rows
+    bf16 = False
     N, d, H, hd, F, L = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn",
                                           "n_layers"))
     g = synth.rng(0)
@@ -166,13 +155,13 @@ def test_4k_shape_two_layers_two_loops(dtype):
     want = oloop.run(layers, h0, sched_o, H, hd, bias,
                      select_prev={2: lambda rows: rows - delta.astype(np.float64)},
                      bf16_ops=bf16)
-    assert_close(h1_gpu, want["h"][1], max_abs=tol1, what="h_1")
+    assert_close(h1_gpu, want["h"][1], what="h_1")
     assert np.array_equal(host(run.act[2]), want["act"][2])
     h2 = host(run.h)
     rs = synth.rng(5)
     rows = np.concatenate([rs.choice(want["act"][2], 64, replace=False),
                            rs.choice(np.setdiff1d(np.arange(N), want["act"][2]), 16, replace=False)])
-    assert_close(h2[rows], want["h"][2][rows], max_abs=tol2, what="h_2 sampled rows")
+    assert_close(h2[rows], want["h"][2][rows], what="h_2 sampled rows")
 
 
 def test_4k_workload_24_layers_invariants():

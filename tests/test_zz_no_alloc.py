@@ -55,6 +55,30 @@ def test_noalloc_matches_workspace_entry_point(n, d, dt, k, use_tok):
         assert torch.equal(got_pos, want_pos)
 
 
+def test_noalloc_without_positions_and_with_k_zero():
+    """out_pos may be NULL (the kept tokens alone), and k = 0 runs only the change pass
+    into the shared scratch: both return what the workspace entry point returns."""
+    from cross_loop_sparse_step_b200 import fl
+    f = _noalloc(fl)
+    n, d, k = 3000, 256, 700
+    g = synth.rng(901)
+    cur, prev, _ = synth.pareto_delta_pair(g, n, d, 2)
+    hc, hp = torch.from_numpy(cur).cuda(), torch.from_numpy(prev).cuda()
+    want = fl.select_active(hc, hp, k)
+    got = torch.full((k,), -3, dtype=torch.int32, device="cuda")
+    rc = f(hc.data_ptr(), hp.data_ptr(), fl.F32, n, d, None, k, got.data_ptr(), None,
+           fl.stream_handle())
+    assert rc == 0, fl.status_str(rc)
+    assert fl.check_device_status() == 0
+    assert torch.equal(got, want)
+    untouched = torch.full((1,), -5, dtype=torch.int32, device="cuda")
+    rc = f(hc.data_ptr(), hp.data_ptr(), fl.F32, n, d, None, 0, untouched.data_ptr(), None,
+           fl.stream_handle())
+    assert rc == 0, fl.status_str(rc)
+    assert fl.check_device_status() == 0
+    assert int(untouched.item()) == -5
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     from cross_loop_sparse_step_b200 import fl
     f = _noalloc(fl)

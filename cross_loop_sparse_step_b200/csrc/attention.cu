@@ -359,6 +359,17 @@ cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, 
   return launch_attn_sparse_batched(host[0], static_cast<const AttnParams*>(ws), n, loop_max, s);
 }
 
+// The query-tile tensor-core form of the sparse attention unless FL_ATTN_TILE=0 (then
+// the warp-per-query kernel runs every sparse call).
+static bool attn_tile_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = getenv("FL_ATTN_TILE");
+    on = (e && atoi(e) == 0) ? 0 : 1;
+  }
+  return on == 1;
+}
+
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
   AttnParams P;
@@ -372,6 +383,7 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   P.out_stride = a.out_stride; P.stat_kind = a.stat_kind; P.vnorm = a.kv->vnorm;
   P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
   const bool sparse = a.sel != nullptr;
+  if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) return launch_attn_tile(P, s);
   if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);
   if (!sparse && dense_fast_eligible(P)) return launch_attn_dense_fast(P, s);
   const int max_cols = sparse ? a.sel_stride : a.kv->n_tok;

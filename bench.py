@@ -1,15 +1,18 @@
 #!/usr/bin/env python
 """Loop-step throughput of the FlashLoop lazy loop step on B200.
 
-Workload (default): the Ouro-1.4B-shaped 4K prefill - 4096 tokens, d_model 2048,
-16 x 128 heads, SwiGLU FFN 5632, 24 shared layers, R = 4 loops, bf16 GEMM operands,
-20% active tokens per sparse loop, 82 carried columns per query plus the sink,
-int8 base + 4-bit residual KV (group 32), a +4 logit bias on 2% of the columns and
-the sink, heavy-tailed (Pareto 1.5) hidden-state changes. Loop 1 (dense, every
-token, the producer of the carried statistics) runs once, untimed; one timed step
-is loops 2..R through fl_loop_step: selection, gather, 24 layers of the block on the
-active rows (QKV + RoPE, residual KV quantisation, sparse attention, O projection,
-FFN), scatter. value = N * (R - 1) / step time: loop-step tokens/s.
+Workload (default): the Ouro-2.6B-shaped 32K prefill - 32768 tokens, d_model 2048,
+16 x 128 heads, SwiGLU FFN 5632, 48 shared layers, R = 4 loops, bf16 GEMM operands,
+15% active tokens per sparse loop (4916), 2048 carried columns per query plus the
+sink, int8 base + 2-bit residual KV (group 32), a +4 logit bias on 2% of the columns
+and the sink, heavy-tailed (Pareto 1.5) hidden-state changes. Loop 1 (dense, every
+token, the producer of the carried statistics) runs before the timed region and is
+timed on its own; one timed step is loops 2..R through fl_loop_step: selection,
+gather, 48 layers of the block on the active rows (QKV + RoPE, residual KV
+quantisation, sparse attention, O projection, FFN), scatter.
+value = N * (R - 1) / step time: loop-step tokens/s. The line also reports the
+end-to-end prefill rate N / (t_1 + t_2 + ... + t_R) with the dense loop 1 included.
+Other workloads: --config (the 4K Ouro-1.4B shape, the 8K loop-depth sweep).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU: one process per GPU (torchrun); every rank runs an independent replica of
@@ -41,7 +44,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="ouro-1.4b-shape-prefill-4k")
+    ap.add_argument("--config", default="ouro-2.6b-shape-prefill-32k")
     ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -226,58 +229,82 @@ def kv_bytes(W):
 
 
 # ---------------------------------------------------------------- CPU baseline (oracle)
-def oracle_sample(cfg, n_layers=1, rows=256, seed=1):
-    """Times the oracle on a bounded sample of the loop-2 step: the token ranking over
-    all N rows, then for `n_layers` layers the block, residual quantisation and sparse
-    attention of `rows` active rows. Returns seconds extrapolated to one full sparse
-    loop (k_r rows x L layers), the measured seconds and the sample description."""
-    from cross_loop_sparse_step_b200 import configs, synth
-    from oracle import attention as oatt
-    from oracle import block as oblk
-    from oracle import kvstore as okv
-    from oracle import select as osel
-    N, d, H, hd, F, L = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn",
-                                          "n_layers"))
-    k_act = configs.active_counts(cfg)[2]
-    kcol = cfg["col_k"][2]
-    g = synth.rng(seed)
-    cur, prev, _ = synth.pareto_delta_pair(g, N, d, 2)
-    layers = synth.model_weights(g, n_layers, d, F, bf16=True)
-    bias = synth.col_bias(g, N, cfg["bias_frac"], cfg["bias_value"])
-    stores = []
-    for _ in range(n_layers):
-        st = okv.LayerKV(N, H, hd, cfg["group"], cfg["base_bits"], cfg["res_bits"], cfg["n_loops"])
-        st.write_base(synth.kv_values(g, N, H, hd), synth.kv_values(g, N, H, hd))
-        stores.append(st)
-    # carried statistics of the sampled queries: the sink, biased columns, then random
-    t0 = time.perf_counter()
-    act, _, _ = osel.select_active(cur, prev, None, k_act)
-    t_select = time.perf_counter() - t0
-    rs = synth.rng(seed + 1)
-    q_rows = np.sort(rs.choice(act, size=min(rows, len(act)), replace=False)).astype(np.int32)
-    X = synth.embeddings(g, len(q_rows), d).astype(np.float64)
-    S = np.full((H, N, kcol + 1), oatt.SENTINEL, np.uint16)
-    for t in q_rows:
-        for h in range(H):
-            n = min(kcol, int(t)) + 1
-            c = np.sort(np.concatenate([[0], rs.choice(np.arange(1, t + 1), n - 1, replace=False)])) \
-                if t > 0 else np.array([0])
-            S[h, t, :n] = c
-    m = np.full((H, N), 0.9)
-    u = np.zeros((H, N, hd))
-    t0 = time.perf_counter()
-    for li in range(n_layers):
-        q, k, v = oblk.qkv(X, q_rows, layers[li], H, hd)
-        stores[li].write_residual(2, q_rows, k.astype(np.float32), v.astype(np.float32))
-        Kh, Vh = stores[li].hat[2]
-        o = oatt.sparse_attention(q, q_rows, q_rows, Kh, Vh, S, m, u, bias)
-        X = oblk.out_ffn(X, o.reshape(len(q_rows), d), layers[li])
-    t_layers = time.perf_counter() - t0
-    per_loop = t_select + t_layers / n_layers * L * (k_act / len(q_rows))
-    desc = (f"loop-2 step sample: token ranking over all {N} rows, then {n_layers} layer(s) x "
-            f"{len(q_rows)} active rows (of {k_act}) x {H} heads; extrapolated x{L} layers, "
-            f"x{k_act}/{len(q_rows)} rows")
-    return per_loop, t_select + t_layers, desc
+class OracleSample:
+    """The oracle on a bounded sample of one sparse loop step of the workload.
+
+    Set-up (untimed): ``n_layers`` layers of random bf16 weights, their KV stores with
+    every token's base codes, the carried statistics of ``rows`` sampled active queries
+    (sink, biased columns, random others). ``run()`` (timed): the token ranking over all
+    N rows (h, previous state), then per layer the block, the residual quantisation and
+    the sparse attention of the sampled rows. Returns the seconds extrapolated to one
+    sparse loop step of the workload (k_r rows x L layers), the measured seconds and the
+    sample's description."""
+
+    def __init__(self, cfg, n_layers=1, rows=256, seed=1):
+        from cross_loop_sparse_step_b200 import configs, synth
+        from oracle import attention as oatt
+        from oracle import kvstore as okv
+        from oracle import select as osel
+        self.cfg = cfg
+        N, d, H, hd, F = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn"))
+        self.k_act = configs.active_counts(cfg)[2]
+        kcol = cfg["col_k"][2]
+        g = synth.rng(seed)
+        self.cur, self.prev, _ = synth.pareto_delta_pair(g, N, d, 2)
+        self.layers = synth.model_weights(g, n_layers, d, F, bf16=True)
+        self.bias = synth.col_bias(g, N, cfg["bias_frac"], cfg["bias_value"])
+        self.stores = []
+        for _ in range(n_layers):
+            st = okv.LayerKV(N, H, hd, cfg["group"], cfg["base_bits"], cfg["res_bits"],
+                             cfg["n_loops"])
+            st.write_base(synth.kv_values(g, N, H, hd), synth.kv_values(g, N, H, hd))
+            self.stores.append(st)
+        act, _, _ = osel.select_active(self.cur, self.prev, None, self.k_act)
+        rs = synth.rng(seed + 1)
+        self.q_rows = np.sort(rs.choice(act, size=min(rows, len(act)), replace=False)).astype(np.int32)
+        self.X = synth.embeddings(g, len(self.q_rows), d).astype(np.float64)
+        self.S = np.full((H, N, kcol + 1), oatt.SENTINEL, np.uint16)
+        for t in self.q_rows:
+            for h in range(H):
+                n = min(kcol, int(t)) + 1
+                c = np.sort(np.concatenate([[0], rs.choice(np.arange(1, t + 1), n - 1, replace=False)])) \
+                    if t > 0 else np.array([0])
+                self.S[h, t, :n] = c
+        self.m = np.full((H, N), 0.9)
+        self.u = np.zeros((H, N, hd))
+        self.n_layers = n_layers
+        self.desc = (f"loop-2 step sample: token ranking over all {N} rows, then {n_layers} "
+                     f"layer(s) x {len(self.q_rows)} active rows (of {self.k_act}) x {H} heads "
+                     f"with {kcol} carried columns; extrapolated x{cfg['n_layers']} layers, "
+                     f"x{self.k_act}/{len(self.q_rows)} rows")
+
+    def run(self):
+        from oracle import attention as oatt
+        from oracle import block as oblk
+        from oracle import select as osel
+        H, hd = self.cfg["n_heads"], self.cfg["head_dim"]
+        d = H * hd
+        t0 = time.perf_counter()
+        osel.select_active(self.cur, self.prev, None, self.k_act)
+        t_select = time.perf_counter() - t0
+        X = self.X
+        t0 = time.perf_counter()
+        for li in range(self.n_layers):
+            q, k, v = oblk.qkv(X, self.q_rows, self.layers[li], H, hd, bf16_ops=True)
+            self.stores[li].write_residual(2, self.q_rows, k.astype(np.float32), v.astype(np.float32))
+            Kh, Vh = self.stores[li].hat[2]
+            o = oatt.sparse_attention(q, self.q_rows, self.q_rows, Kh, Vh, self.S, self.m, self.u,
+                                      self.bias)
+            X = oblk.out_ffn(X, o.reshape(len(self.q_rows), d), self.layers[li], bf16_ops=True)
+        t_layers = time.perf_counter() - t0
+        per_loop = t_select + t_layers / self.n_layers * self.cfg["n_layers"] * (
+            self.k_act / len(self.q_rows))
+        return per_loop, t_select + t_layers, self.desc
+
+
+# bounded samples of the oracle per workload size: (layers, rows)
+def oracle_sample_size(cfg):
+    return (1, 128) if cfg["n_tok"] >= 16384 else (2, 256)
 
 
 def blas_threads():
@@ -296,12 +323,15 @@ def run_reference(args):
     from cross_loop_sparse_step_b200 import configs
     cfg = configs.CONFIGS[args.config]
     R = cfg["n_loops"]
-    times = []
-    desc = ""
+    n_layers, rows = oracle_sample_size(cfg)
+    sample = OracleSample(cfg, n_layers=n_layers, rows=rows, seed=1)
+    times, measured = [], []
+    desc = sample.desc
     for i in range(args.warmup + args.steps):
-        per_loop, _, desc = oracle_sample(cfg, n_layers=2, rows=512, seed=1 + i)
+        per_loop, meas, desc = sample.run()
         if i >= args.warmup:
             times.append(per_loop)
+            measured.append(meas)
     per_loop = float(np.mean(times))
     value = cfg["n_tok"] / per_loop
     cores = blas_threads()
@@ -310,6 +340,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_loop * (R - 1) * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "extrapolated": True,
+        "measured_s_per_step": round(float(np.mean(measured)), 3),
         "config": {"workload": cfg["name"], "n_tok": cfg["n_tok"], "layers": cfg["n_layers"],
                    "loops": R},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -508,9 +540,12 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        per_loop, measured, desc = oracle_sample(cfg, n_layers=8, rows=512)
+        n_layers, rows = oracle_sample_size(cfg)
+        sample = OracleSample(cfg, n_layers=n_layers, rows=rows, seed=1)
+        per_loop, measured, desc = sample.run()
         cpu = {"value": N / per_loop, "unit": "tokens/s", "cores": blas_threads(),
-               "kind": "oracle", "sample": desc, "measured_s": round(measured, 2)}
+               "kind": "oracle", "sample": desc, "measured_s": round(measured, 2),
+               "extrapolated": True}
 
     if rank == 0:
         line = {

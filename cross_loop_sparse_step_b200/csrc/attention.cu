@@ -325,9 +325,12 @@ cudaError_t launch_t(const AttnParams& P, int max_cols, cudaStream_t s) {
 
 }  // namespace
 
+static bool attn_tile_enabled();
+
 size_t attention_ws_bytes(const fl_attn_args& a) {
-  (void)a;
-  return 0;
+  if (a.sel || !a.kv) return 0;
+  const AttnParams P = make_attn_params(a, nullptr);
+  return attn_tile_enabled() && dense_tile_eligible(P) ? dense_tile_ws_bytes(P) : 0;
 }
 
 AttnParams make_attn_params(const fl_attn_args& a, int* st) {
@@ -384,6 +387,10 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
   const bool sparse = a.sel != nullptr;
   if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) return launch_attn_tile(P, s);
+  if (!sparse && attn_tile_enabled() && dense_tile_eligible(P)) {
+    if (P.sel_out && a.ws_bytes < dense_tile_ws_bytes(P)) return cudaErrorInvalidValue;
+    return launch_attn_dense_tile(P, a.ws, s);
+  }
   if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);
   if (!sparse && dense_fast_eligible(P)) return launch_attn_dense_fast(P, s);
   const int max_cols = sparse ? a.sel_stride : a.kv->n_tok;

@@ -47,21 +47,16 @@ __device__ __forceinline__ void base_part(const KvView& kv, int which, size_t bh
   f2::load_pairs<EL>(kv.codes[which][1] + bh * (size_t)(EL * 4), 8, e0, c);
 }
 
+// One warp's work: query qi, head h; `base` is the warp's shared-memory slice.
 template <int HD>
-__global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ AttnParams P) {
-  extern __shared__ __align__(16) uint8_t smem[];
+__device__ __forceinline__ void dense_warp(const AttnParams& P, int qi, int h, uint8_t* base) {
   constexpr int EL = HD / 4;
-  const int nw = blockDim.x >> 5;
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gw = blockIdx.x * nw + w;
-  if (gw >= P.n_q * P.H) return;  // whole warp leaves; no CTA-wide barrier below
-  const int qi = gw / P.H, h = gw % P.H;
+  const int lane = threadIdx.x & 31;
   const int H = P.H, n_tok = P.kv.n_tok, gs = P.kv.g;
   const KvView& kv = P.kv;
   const int l4 = lane & 3, cg = lane >> 2;
   const int e0 = l4 * EL, gidx = e0 / gs, ngrp = HD / gs;
 
-  uint8_t* base = smem + (size_t)w * dense_warp_smem(n_tok);
   float* p = reinterpret_cast<float*>(base);
   uint8_t* mark = base + a16((size_t)n_tok * 4);
   int* hist = reinterpret_cast<int*>(mark + a16((size_t)n_tok));
@@ -273,7 +268,59 @@ __global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ Attn
   if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = lm;
 }
 
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_dense(const __grid_constant__ AttnParams P) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nw = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int gw = blockIdx.x * nw + w;
+  if (gw >= P.n_q * P.H) return;  // whole warp leaves; no CTA-wide barrier below
+  dense_warp<HD>(P, gw / P.H, gw % P.H, smem + (size_t)w * dense_warp_smem(P.kv.n_tok));
+}
+
+// The (query, head) pairs list[0, *count) (entries h * n_q + query), warps striding over
+// the list: the exact finish of rows the tensor-core producer could not rank.
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_dense_list(const __grid_constant__ AttnParams P,
+                                                         const int* list, const int* count) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int nw = blockDim.x >> 5;
+  const int w = threadIdx.x >> 5;
+  const int n = *count;
+  for (int x = blockIdx.x * nw + w; x < n; x += gridDim.x * nw) {
+    const int rh = list[x];
+    dense_warp<HD>(P, rh % P.n_q, rh / P.n_q, smem + (size_t)w * dense_warp_smem(P.kv.n_tok));
+  }
+}
+
 }  // namespace
+
+bool dense_rows_supported(const AttnParams& P) {
+  return P.hd == 128 && P.kv.base_bits == 8 && dense_warp_smem(P.kv.n_tok) <= 200 * 1024;
+}
+
+cudaError_t launch_attn_dense_rows(const AttnParams& P, const int* list, const int* count,
+                                   cudaStream_t s) {
+  const size_t per = dense_warp_smem(P.kv.n_tok);
+  int nw = (int)((200 * 1024) / per);
+  nw = nw < 1 ? 1 : (nw > 4 ? 4 : nw);
+  const size_t sm = (size_t)nw * per;
+  static int attr_bytes[128] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if ((int)sm > attr_bytes[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_dense_list<128>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    attr_bytes[dev] = (int)sm;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  k_attn_dense_list<128><<<sms, nw * 32, sm, s>>>(P, list, count);
+  count_launch();
+  return cudaGetLastError();
+}
 
 bool dense_fast_eligible(const AttnParams& P) {
   if (P.sel != nullptr || P.loop != 1) return false;

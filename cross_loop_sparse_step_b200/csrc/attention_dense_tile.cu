@@ -1,0 +1,817 @@
+// Dense causal attention and the column statistics it hands to the next loop, on the
+// tensor cores, one CTA per (head, tile of 128 queries) (FlashLoop §4.2 "Loop-Aware
+// Sparse Attention": the sparse loops rank columns by statistics of the previous loop;
+// a dense loop is where they are produced).
+//
+// Statistics for query i (t = its position, k = the next loop's budget, t > k):
+//   S' = {0} U top-k over j in [1, t] of c_j = p_j ||V^_j|| (or p_j), ties to the smaller
+//   column; m' = sum over S' of p_j; u' = sum over the other columns of p_j V^_j.
+// The ranking of a row depends on s_j + log ||V^_j|| alone, so it is taken in four steps:
+//   kernel A, three passes over the tile's column chunks (the same producer / MMA / softmax
+//   pipeline as the sparse tile kernel; columns are the contiguous range [0, t_max]):
+//     flash  S = Q K^T (fp16 operands), online softmax with a causal mask, O += P V^
+//            -> o = O / sum, and the row's final maximum and sum;
+//     hist   S again (fp16): a 128-bin histogram per row of kappa_j = s_j + log2 ||V^_j||,
+//            1/8 log2 unit per bin below the row's upper bound (final maximum + the
+//            largest log2 ||V^|| the row saw) -> the bin holding the k-th largest, and a
+//            threshold one margin below it (the margin bounds the fp16 score error);
+//     cand   S with split operands (q = hi + lo, K^ = hi + lo, fp16 each; three MMAs,
+//            22 significant bits, binary32 sums): every column with kappa at or above the
+//            threshold is a candidate - written with its p_j to a per-row buffer;
+//   kernel B (one CTA per row and head): exact top-k of c_j = p_j ||V^_j|| among the
+//     candidates (radix select on the binary32 bits, equal values to the smaller column),
+//     S' written ascending, m' = p_0 + sum of the kept p_j;
+//   kernel C, one pass: S (fp16), p_j = 2^(s_j - max) / sum with the row's final maximum
+//     and sum, and u' = sum over the columns outside S' of p_j V^_j (P V^ on the tensor
+//     cores with the complement of S' as the mask).
+// A row whose candidates overflow its buffer (a near-uniform row of more than the buffer's
+// spare capacity in one histogram bin) is finished by the exact per-query kernel.
+// Every wait is bounded; a wait that runs out records FL_ERR_TIMEOUT, the CTA drains its
+// MMAs, frees TMEM and returns. Warp-collective TMEM accesses stay warp-uniform.
+#include <float.h>
+
+#include "attn_tile_common.cuh"
+
+namespace fl {
+namespace {
+
+using namespace sm100;
+using namespace tile;
+
+constexpr int NWARPS = 13;         // 0-3, 8-11 producers; 4-7 softmax; 12 MMA
+constexpr int NTHR = NWARPS * 32;
+constexpr int NBIN = 128;          // histogram bins per row
+constexpr float kBinsPerLog2 = 8.f;
+constexpr float kMargin = 1.f / 64;   // log2 units; fp16 scores differ by far less
+
+enum : int { PASS_FLASH = 0, PASS_HIST = 1, PASS_CAND = 2, PASS_UNSEL = 3 };
+
+// dynamic shared memory (1024-byte aligned base)
+constexpr uint32_t OFF_QHI = 0;
+constexpr uint32_t OFF_R1 = OFF_QHI + TILE;      // P | histogram [NBIN][TQ] u16 | Q lo
+constexpr uint32_t OFF_ST = OFF_R1 + TILE;       // stage s: tile A at OFF_ST + 2 s TILE, B after
+constexpr uint32_t OFF_META = OFF_ST + 4 * TILE; // [2][TC] bias (log2 units), [2][TC] log2 ||V^||
+constexpr uint32_t SMEM_BYTES = OFF_META + 4 * TC * 4 + 1024;
+static_assert(NBIN * TQ * 2 <= TILE, "histogram fits its region");
+
+struct DenseArgs {
+  AttnParams P;
+  int mode;          // 0: flash only, 1: flash + hist + cand, 2: unselected pass
+  int k;             // the next loop's budget
+  int cap;           // candidates per row
+  float2* m1l;       // [H][n_q] (final maximum, log2 units; sum)
+  int* cnt;          // [H][n_q] candidates written (> cap: overflow)
+  float* p0;         // [H][n_q] p of the sink column
+  uint16_t* ccol;    // [H][n_q][cap]
+  float* cp;         // [H][n_q][cap]
+};
+
+struct DenseShared {
+  uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full, pv_done, qlo_ready, hist_done,
+      fin;
+  uint32_t tmem;
+  int abort_flag;
+  int t_max;
+};
+
+__device__ __forceinline__ int pass_of(int mode, int G, int nc) {
+  if (mode == 2) return PASS_UNSEL;
+  if (mode == 0) return PASS_FLASH;
+  const int p = G / nc;
+  return p == 0 ? PASS_FLASH : (p == 1 ? PASS_HIST : PASS_CAND);
+}
+__device__ __forceinline__ bool has_pv(int pass) { return pass == PASS_FLASH || pass == PASS_UNSEL; }
+
+// the query row (fp32 or bf16) as 8 binary32 values from element e0
+__device__ __forceinline__ void load_q8(const AttnParams& P, int qi, int h, int e0, float* x) {
+  const size_t off = ((size_t)qi * P.H + h) * HDT + e0;
+  if (P.q_bf16) {
+    const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) { x[2 * k] = __low2float(b2[k]); x[2 * k + 1] = __high2float(b2[k]); }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off + 4);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+__global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
+  const AttnParams& P = A.P;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ DenseShared sh;
+  volatile int* abort = &sh.abort_flag;
+  float* meta = reinterpret_cast<float*>(smem + OFF_META);   // bias [2][TC], lvn [2][TC]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = P.H, n_tok = P.kv.n_tok;
+  const int n_tiles = (P.n_q + TQ - 1) / TQ;
+  const int h = blockIdx.x / n_tiles;
+  const int q0 = (blockIdx.x % n_tiles) * TQ;
+  const int mode = A.mode;
+  const bool stats = mode == 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sh.kv_full[s], 4); mbar_init(&sh.kv_empty[s], 1);
+      mbar_init(&sh.meta_full[s], 4); mbar_init(&sh.s_full[s], 1);
+    }
+    mbar_init(&sh.p_full, TQ);
+    mbar_init(&sh.pv_done, 1);
+    mbar_init(&sh.qlo_ready, TQ);
+    mbar_init(&sh.hist_done, TQ);
+    mbar_init(&sh.fin, 1);
+    sh.abort_flag = 0;
+    sh.t_max = -1;
+    fence_barrier_init();
+  }
+  if (warp == 12) tmem_alloc(&sh.tmem, 512);
+  griddep_wait();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sh.tmem;
+  if (threadIdx.x < TQ && q0 + (int)threadIdx.x < P.n_q) {
+    const int t = P.q_tok[q0 + threadIdx.x];
+    if (t >= 0 && t < n_tok) atomicMax(&sh.t_max, t);
+  }
+  __syncthreads();
+  const int t_max = sh.t_max;
+  const int nc = (t_max + TC) / TC;                  // chunks covering [0, t_max]
+  const int n_pass = stats ? 3 : 1;
+  const int total = t_max < 0 ? 0 : nc * n_pass;
+  const float scale2 = P.scale * kLog2e;
+  const uint32_t idesc = idesc_f16_f32(TQ, TC);
+
+  if (warp >= 4 && warp < 8) {
+    // ================================================================ softmax warps
+    const int i = (warp - 4) * 32 + lane;
+    const int qi = q0 + i;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    bool valid = qi < P.n_q;
+    int t = -1, srow = 0;
+    if (valid) {
+      t = P.q_tok[qi];
+      srow = P.q_row ? P.q_row[qi] : t;
+      const bool row_ok = mode == 2 ? (srow >= 0 && srow < P.stat_rows) : true;
+      if (t < 0 || t >= n_tok || !row_ok) {
+        record_error(P.st, FL_ERR_RANGE);
+        valid = false;
+        t = -1;
+      }
+    }
+    const size_t rh = (size_t)h * P.n_q + (valid ? qi : 0);
+    // Q (hi part: fp16 of q) for every pass
+    {
+      uint8_t* qt = smem + OFF_QHI;
+      for (int e0 = 0; e0 < HDT; e0 += 8) {
+        float x[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x[k] = 0.f;
+        if (valid) load_q8(P, qi, h, e0, x);
+        *reinterpret_cast<uint4*>(qt + sw128_offset(i, e0, TQ)) =
+            make_uint4(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]), pack_h2(x[6], x[7]));
+      }
+      fence_proxy_async_smem();
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");
+
+    // unselected pass: the row's maximum and sum, and its S' walked in step with the chunks
+    float m_used = -INFINITY, lsum = 0.f;
+    const uint16_t* sel_row = nullptr;
+    int ent = 0;
+    bool ended = true;
+    uint32_t nx[8];
+    int gr[8], gmax = -1;
+    auto load_next = [&]() {
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        nx[k] = (!ended && ent + k < P.out_stride) ? (uint32_t)sel_row[ent + k] : (uint32_t)FL_SENTINEL;
+      ent += 8;
+    };
+    auto take_next = [&]() {
+      gmax = -1;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = (int)nx[k];
+        gr[k] = -1;
+        if (ended || c == (int)FL_SENTINEL) { ended = true; continue; }
+        if (c > t) continue;
+        gr[k] = c;
+        gmax = c;
+      }
+      if (ent >= P.out_stride) ended = true;
+      load_next();
+    };
+#pragma unroll
+    for (int k = 0; k < 8; ++k) gr[k] = -1;
+    if (mode == 2 && valid) {
+      const float2 ml = A.m1l[rh];
+      m_used = ml.x;
+      lsum = ml.y;
+      sel_row = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
+      ended = false;
+      load_next();
+      take_next();
+    }
+    const bool sel_row_stats = stats && valid && t > A.k;   // rows that rank columns
+    // m_used: the reference of P and the sum (raised only by more than 2^8); m_true: the
+    // exact running maximum, which anchors the histogram
+    float m_true = -INFINITY, lvmax = -INFINITY, ktop = 0.f, thr = -INFINITY, p0 = 0.f;
+    int cand = 0;
+    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + OFF_R1);
+    uint8_t* pt = smem + OFF_R1;
+    const bool pv_stat = P.stat_kind == FL_STAT_PV;
+
+    for (int G = 0; G < total; ++G) {
+      const int pass = pass_of(mode, G, nc);
+      const int c = G % nc;
+      const int sb = G & 1;
+      if (!warp_wait(&sh.s_full[sb], (G >> 1) & 1, abort)) break;
+      if (!warp_wait(&sh.meta_full[sb], (G >> 1) & 1, abort)) break;
+      tc_fence_after();
+      const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
+      const float* bias = meta + sb * TC;
+      const float* lvn = meta + 2 * TC + sb * TC;
+      const int nin = t < 0 ? 0 : min(max(t - c * TC + 1, 0), TC);   // causal columns
+      if (pass == PASS_FLASH) {
+        float cmax = -INFINITY;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float v[32];
+          tmem_ld32(s_addr + g4 * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int jj = g4 * 32 + j;
+            if (jj < nin) {
+              cmax = fmaxf(cmax, fmaf(v[j], scale2, bias[jj]));
+              lvmax = fmaxf(lvmax, lvn[jj]);
+            }
+          }
+        }
+        m_true = fmaxf(m_true, cmax);
+        float alpha = 1.f;
+        bool rescale = false;
+        if (cmax > m_used + kRescale) {
+          if (m_used != -INFINITY && lsum > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
+          m_used = cmax;
+        }
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+        tc_fence_after();
+        if (rescale) lsum *= alpha;
+        if (__any_sync(0xffffffffu, rescale)) {
+          const uint32_t o_addr = tmem + lane_base + 2u * TC;
+#pragma unroll 1
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float v[32];
+            tmem_ld32(o_addr + g4 * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= alpha;
+            tmem_st32(o_addr + g4 * 32, v);
+          }
+        }
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float v[32];
+          tmem_ld32(s_addr + g4 * 32, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int jj = g4 * 32 + j;
+            const float a = jj < nin ? exp2f(fmaf(v[j], scale2, bias[jj]) - m_used) : 0.f;
+            const float b = jj + 1 < nin ? exp2f(fmaf(v[j + 1], scale2, bias[jj + 1]) - m_used) : 0.f;
+            const __half2 hv = __floats2half2_rn(a, b);
+            const float2 back = __half22float2(hv);
+            lsum += back.x + back.y;
+            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(pt + sw128_offset(i, g4 * 32 + q * 8, TQ)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        if (c == nc - 1) {
+          // ---- end of the flash pass: o = O / sum; the row's maximum and sum
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort)) break;
+          tc_fence_after();
+          const uint32_t o_addr = tmem + lane_base + 2u * TC;
+          const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
+          const size_t ob = ((size_t)qi * H + h) * HDT;
+#pragma unroll 1
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float v[32];
+            tmem_ld32(o_addr + g4 * 32, v);
+            if (!valid) continue;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              const float o0 = v[j] * f, o1 = v[j + 1] * f, o2 = v[j + 2] * f, o3 = v[j + 3] * f;
+              if (P.out_bf16) {
+                __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(P.out) + ob + g4 * 32 + j;
+                const __nv_bfloat162 a = __floats2bfloat162_rn(o0, o1), b = __floats2bfloat162_rn(o2, o3);
+                *reinterpret_cast<uint2*>(o) = make_uint2(*reinterpret_cast<const uint32_t*>(&a),
+                                                          *reinterpret_cast<const uint32_t*>(&b));
+              } else {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(P.out) + ob + g4 * 32 + j) =
+                    make_float4(o0, o1, o2, o3);
+              }
+            }
+          }
+          if (stats) {
+            if (valid) A.m1l[rh] = make_float2(m_used, lsum);
+            ktop = m_true + (pv_stat ? lvmax : 0.f);
+            // the histogram takes the P region over (every thread saw the last P V^ finish)
+            for (int b = 0; b < NBIN; ++b) hist[b * TQ + i] = 0;
+          }
+        }
+      } else if (pass == PASS_HIST) {
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float v[32];
+          tmem_ld32(s_addr + g4 * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int jj = g4 * 32 + j;
+            if (sel_row_stats && jj < nin && (c > 0 || jj > 0)) {
+              const float kap = fmaf(v[j], scale2, bias[jj]) + (pv_stat ? lvn[jj] : 0.f);
+              float bf = (ktop - kap) * kBinsPerLog2;
+              bf = fminf(fmaxf(bf, 0.f), (float)(NBIN - 1));   // NaN-free: kap finite or -inf
+              const int b = (int)bf;
+              hist[b * TQ + i] += 1;
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        if (c == nc - 1) {
+          // ---- the bin of the k-th largest; the candidate threshold one margin below it
+          if (sel_row_stats) {
+            int acc = 0, b = 0;
+            for (; b < NBIN - 1; ++b) {
+              acc += hist[b * TQ + i];
+              if (acc >= A.k) break;
+            }
+            thr = b >= NBIN - 1 ? -INFINITY : ktop - (float)(b + 1) / kBinsPerLog2 - kMargin;
+          }
+          // every row's histogram read: the region becomes Q lo (a bounded wait, not a
+          // named barrier, so an aborted warp cannot hold the others)
+          mbar_arrive(&sh.hist_done);
+          if (!warp_wait(&sh.hist_done, 0, abort)) break;
+          uint8_t* ql = smem + OFF_R1;
+          for (int e0 = 0; e0 < HDT; e0 += 8) {
+            float x[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) x[k] = 0.f;
+            if (valid) load_q8(P, qi, h, e0, x);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) x[k] = x[k] - __half2float(__float2half_rn(x[k]));
+            *reinterpret_cast<uint4*>(ql + sw128_offset(i, e0, TQ)) =
+                make_uint4(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]), pack_h2(x[6], x[7]));
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(&sh.qlo_ready);
+        }
+      } else if (pass == PASS_CAND) {
+        const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
+        uint16_t* ccol = A.ccol + rh * A.cap;
+        float* cpr = A.cp + rh * A.cap;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float v[32];
+          tmem_ld32(s_addr + g4 * 32, v);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int jj = g4 * 32 + j;
+            if (sel_row_stats && jj < nin) {
+              const float s2 = fmaf(v[j], scale2, bias[jj]);
+              if (c == 0 && jj == 0) {
+                p0 = exp2f(s2 - m_used) * inv_l;
+              } else if (s2 + (pv_stat ? lvn[jj] : 0.f) >= thr) {
+                if (cand < A.cap) {
+                  ccol[cand] = (uint16_t)(c * TC + jj);
+                  cpr[cand] = exp2f(s2 - m_used) * inv_l;
+                }
+                ++cand;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        if (c == nc - 1 && sel_row_stats) {
+          A.cnt[rh] = cand;
+          A.p0[rh] = p0;
+        }
+      } else {   // PASS_UNSEL: u' over the columns outside S'
+        uint32_t mask[4] = {0u, 0u, 0u, 0u};   // columns of S' in this chunk
+        const int lo = c * TC, hi = lo + TC;
+        while (true) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int pos = gr[k] - lo;
+            const uint32_t bit = (pos >= 0 && pos < TC) ? 1u << (pos & 31) : 0u;
+            const int w = pos >> 5;
+            mask[0] |= w == 0 ? bit : 0u;
+            mask[1] |= w == 1 ? bit : 0u;
+            mask[2] |= w == 2 ? bit : 0u;
+            mask[3] |= w == 3 ? bit : 0u;
+          }
+          if (gmax < hi && !ended) take_next();
+          else break;
+        }
+        __syncwarp();   // reconverge before the warp-collective TMEM accesses
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          float v[32];
+          tmem_ld32(s_addr + g4 * 32, v);
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const int jj = g4 * 32 + j;
+            const bool ina = jj < nin && !(mask[g4] & (1u << j));
+            const bool inb = jj + 1 < nin && !(mask[g4] & (1u << (j + 1)));
+            const float a = ina ? exp2f(fmaf(v[j], scale2, bias[jj]) - m_used) : 0.f;
+            const float b = inb ? exp2f(fmaf(v[j + 1], scale2, bias[jj + 1]) - m_used) : 0.f;
+            const __half2 hv = __floats2half2_rn(a, b);
+            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(pt + sw128_offset(i, g4 * 32 + q * 8, TQ)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&sh.p_full);
+        if (c == nc - 1) {
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort)) break;
+          tc_fence_after();
+          const uint32_t o_addr = tmem + lane_base + 2u * TC;
+          const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
+          float* u = valid ? P.unsel_out + ((size_t)h * P.stat_rows + srow) * HDT : nullptr;
+#pragma unroll 1
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float v[32];
+            tmem_ld32(o_addr + g4 * 32, v);
+            if (!valid) continue;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              *reinterpret_cast<float4*>(u + g4 * 32 + j) =
+                  make_float4(v[j] * f, v[j + 1] * f, v[j + 2] * f, v[j + 3] * f);
+          }
+        }
+      }
+    }
+  } else if (warp == 12) {
+    // ================================================================ MMA warp
+    asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");
+    if (lane == 0 && total > 0) {
+      const uint32_t qh = smem_u32(smem + OFF_QHI);
+      const uint32_t r1 = smem_u32(smem + OFF_R1);
+      bool qlo_seen = false;
+      auto issue_qk = [&](int G) -> bool {
+        const int pass = pass_of(mode, G, nc);
+        const int st = G & 1;
+        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort)) return false;
+        if (pass == PASS_CAND && !qlo_seen) {
+          if (!mbar_wait(&sh.qlo_ready, 0, abort)) return false;
+          qlo_seen = true;
+        }
+        tc_fence_after();
+        const uint32_t a_t = smem_u32(smem + OFF_ST + 2 * st * TILE);
+        const uint32_t b_t = a_t + TILE;
+        const uint32_t d = tmem + (uint32_t)(st * TC);
+#pragma unroll
+        for (int kk = 0; kk < HDT / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+          mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(a_t + off), idesc,
+                   kk > 0 ? 1u : 0u);
+          if (pass == PASS_CAND) {   // q_hi K_lo + q_lo K_hi
+            mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(b_t + off), idesc, 1u);
+            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_kmajor(a_t + off), idesc, 1u);
+          }
+        }
+        mma_commit(&sh.s_full[st]);
+        if (!has_pv(pass)) mma_commit(&sh.kv_empty[st]);
+        return true;
+      };
+      bool ok = issue_qk(0);
+      for (int G = 0; ok && G < total; ++G) {
+        if (G + 1 < total && !issue_qk(G + 1)) break;
+        if (!mbar_wait(&sh.p_full, G & 1, abort)) break;
+        tc_fence_after();
+        const int pass = pass_of(mode, G, nc);
+        if (has_pv(pass)) {
+          const int st = G & 1, c = G % nc;
+          const uint32_t v_t = smem_u32(smem + OFF_ST + (2 * st + 1) * TILE);
+          const uint32_t d = tmem + 2u * TC;
+#pragma unroll
+          for (int kk = 0; kk < TC / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_kmajor(v_t + off), idesc,
+                     (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.pv_done);
+          mma_commit(&sh.kv_empty[st]);
+        }
+      }
+    }
+    if (lane == 0) mma_commit(&sh.fin);
+  } else {
+    // ================================================================ producer warps
+    const int grp = warp < 4 ? 0 : 1;
+    const int jj = (warp & 3) * 32 + lane;
+    uint8_t* a_tile = smem + OFF_ST + 2 * grp * TILE;
+    uint8_t* b_tile = a_tile + TILE;
+    const bool pv_stat = P.stat_kind == FL_STAT_PV && P.vnorm;
+    for (int G = grp; G < total; G += 2) {
+      if (__any_sync(0xffffffffu, *abort != 0)) break;
+      if (G >= 2 && !warp_wait(&sh.kv_empty[grp], ((G >> 1) - 1) & 1, abort)) break;
+      const int pass = pass_of(mode, G, nc);
+      const int c = G % nc;
+      const int colv = c * TC + jj;
+      const int col = colv <= t_max ? colv : -1;
+      meta[grp * TC + jj] = (col >= 0 && P.bias) ? __ldg(P.bias + col) * kLog2e : 0.f;
+      meta[2 * TC + grp * TC + jj] =
+          (col >= 0 && pv_stat) ? log2f(__ldg(P.vnorm + (size_t)col * H + h)) : 0.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
+      uint32_t chain = 0;
+      BaseRow brow[2];
+      const bool need_v = has_pv(pass);
+      if (col >= 0) {
+        load_base(P, 0, col, h, brow[0]);
+        if (need_v) load_base(P, 1, col, h, brow[1]);
+        for (int r = 2; r <= P.loop; ++r)
+          if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
+      }
+#pragma unroll
+      for (int e0 = 0; e0 < HDT; e0 += 16) {   // K^ (pass cand: hi and lo parts)
+        float x[16];
+        if (col >= 0) reconstruct16(P, 0, col, h, brow[0], chain, e0, x);
+        else {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) x[k] = 0.f;
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const float* y = x + 8 * half;
+          *reinterpret_cast<uint4*>(a_tile + sw128_offset(jj, e0 + 8 * half, TC)) =
+              make_uint4(pack_h2(y[0], y[1]), pack_h2(y[2], y[3]), pack_h2(y[4], y[5]), pack_h2(y[6], y[7]));
+          if (pass == PASS_CAND) {
+            float lo[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) lo[k] = y[k] - __half2float(__float2half_rn(y[k]));
+            *reinterpret_cast<uint4*>(b_tile + sw128_offset(jj, e0 + 8 * half, TC)) =
+                make_uint4(pack_h2(lo[0], lo[1]), pack_h2(lo[2], lo[3]), pack_h2(lo[4], lo[5]),
+                           pack_h2(lo[6], lo[7]));
+          }
+        }
+      }
+      if (need_v) {
+#pragma unroll
+        for (int e0 = 0; e0 < HDT; e0 += 16) {   // V^ transposed: row e, column jj
+          float x[16];
+          if (col >= 0) reconstruct16(P, 1, col, h, brow[1], chain, e0, x);
+          else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) x[k] = 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            *reinterpret_cast<__half*>(b_tile + sw128_offset(e0 + k, jj, HDT)) = __float2half_rn(x[k]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
+    }
+  }
+
+  // ---- teardown: every MMA done before TMEM is released
+  __syncthreads();
+  if (warp == 12) {
+    if (lane == 0) {
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(&sh.fin, 0))
+        if (globaltimer() - t0 > kWaitLimitNs) { sh.abort_flag = 1; break; }
+    }
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, FL_ERR_TIMEOUT);
+}
+
+// ---------------------------------------------------------------- kernel B: selection
+constexpr int SEL_THREADS = 256;
+
+// Exact top-k of c_j = p_j ||V^_j|| (or p_j) among a row's candidates, equal values to
+// the smaller column: S' = {0} U kept (ascending - candidates are stored in column order),
+// m' = p_0 + sum of kept p_j. Rows at positions t <= k keep every column [0, t] (m' = 1).
+// A row whose candidates overflowed is listed for the exact per-query kernel.
+__global__ void __launch_bounds__(SEL_THREADS) k_dense_select(const __grid_constant__ DenseArgs A,
+                                                              int* ovf_n, int* ovf_list) {
+  const AttnParams& P = A.P;
+  extern __shared__ uint8_t sm[];
+  const int qi = blockIdx.x % P.n_q, h = blockIdx.x / P.n_q;
+  const int t = P.q_tok[qi];
+  const int srow = P.q_row ? P.q_row[qi] : t;
+  if (t < 0 || t >= P.kv.n_tok || srow < 0 || srow >= P.stat_rows) return;   // recorded in A
+  uint16_t* so = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
+  const size_t rh = (size_t)h * P.n_q + qi;
+  const int k = A.k;
+  if (t <= k) {
+    for (int j = threadIdx.x; j < P.out_stride; j += SEL_THREADS)
+      so[j] = j <= t ? (uint16_t)j : (uint16_t)FL_SENTINEL;
+    if (threadIdx.x == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = 1.f;
+    return;
+  }
+  const int n = A.cnt[rh];
+  if (n > A.cap || n < k) {   // overflow (or a count that cannot hold k): exact fallback
+    if (threadIdx.x == 0) {
+      const int slot = atomicAdd(ovf_n, 1);
+      ovf_list[slot] = (int)rh;
+    }
+    return;
+  }
+  uint32_t* key = reinterpret_cast<uint32_t*>(sm);                 // [cap] c as bits
+  uint16_t* col = reinterpret_cast<uint16_t*>(key + A.cap);        // [cap]
+  float* pv = reinterpret_cast<float*>(col + ((A.cap + 1) & ~1));  // [cap]
+  __shared__ int hist[256];
+  __shared__ int s_dig, s_above, s_wsum[SEL_THREADS / 32], s_eqb[SEL_THREADS / 32];
+  __shared__ float s_mass[SEL_THREADS / 32];
+  const bool pv_stat = P.stat_kind == FL_STAT_PV;
+  const uint16_t* cc = A.ccol + rh * A.cap;
+  const float* cp = A.cp + rh * A.cap;
+  for (int x = threadIdx.x; x < n; x += SEL_THREADS) {
+    const int cidx = cc[x];
+    const float p = cp[x];
+    const float cv = pv_stat ? p * P.vnorm[(size_t)cidx * P.H + h] : p;
+    key[x] = __float_as_uint(fmaxf(cv, 0.f));
+    col[x] = (uint16_t)cidx;
+    pv[x] = p;
+  }
+  __syncthreads();
+  // radix select of the k-th largest key, 8 bits at a time
+  uint32_t prefix = 0, pmask = 0;
+  int need = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = threadIdx.x; b < 256; b += SEL_THREADS) hist[b] = 0;
+    __syncthreads();
+    for (int x = threadIdx.x; x < n; x += SEL_THREADS)
+      if ((key[x] & pmask) == prefix) atomicAdd(&hist[(key[x] >> shift) & 255u], 1);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int above = 0, d = 255;
+      for (; d > 0; --d) {
+        if (above + hist[d] >= need) break;
+        above += hist[d];
+      }
+      s_dig = d;
+      s_above = above;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)s_dig << shift;
+    pmask |= 255u << shift;
+    need -= s_above;
+    __syncthreads();
+  }
+  // keep key > prefix, and the first `need` entries (smallest columns) with key == prefix;
+  // the candidates are in ascending column order, so a stable compaction keeps S' ascending
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  int written = 0, eq_seen = 0;
+  float mass = 0.f;
+  for (int base = 0; base < n; base += SEL_THREADS) {
+    const int x = base + threadIdx.x;
+    const bool in = x < n;
+    const uint32_t kv = in ? key[x] : 0u;
+    const bool eq = in && kv == prefix;
+    const uint32_t eb = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) s_eqb[w] = __popc(eb);
+    __syncthreads();
+    int eq_before = eq_seen + __popc(eb & lt), eq_tot = 0;
+    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) {
+      if (ww < w) eq_before += s_eqb[ww];
+      eq_tot += s_eqb[ww];
+    }
+    const bool keep = in && (kv > prefix || (eq && eq_before < need));
+    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) s_wsum[w] = __popc(kb);
+    __syncthreads();
+    int pos = written + __popc(kb & lt), tot = 0;
+    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) {
+      if (ww < w) pos += s_wsum[ww];
+      tot += s_wsum[ww];
+    }
+    if (keep && pos < k) {
+      so[1 + pos] = col[x];
+      mass += pv[x];
+    }
+    written += tot;
+    eq_seen += eq_tot;
+    __syncthreads();
+  }
+  written = min(written, k);
+  for (int j = 1 + written + threadIdx.x; j < P.out_stride; j += SEL_THREADS) so[j] = (uint16_t)FL_SENTINEL;
+  if (threadIdx.x == 0) so[0] = 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
+  if (lane == 0) s_mass[w] = mass;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = A.p0[rh];
+    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) m += s_mass[ww];
+    P.mass_out[(size_t)h * P.stat_rows + srow] = m;
+  }
+}
+
+}  // namespace
+
+size_t dense_tile_ws_bytes(const AttnParams& P) {
+  if (!P.sel_out) return 0;
+  const int cap = P.k_next + 1024;
+  const size_t rows = (size_t)P.H * P.n_q;
+  return align_up(rows * sizeof(float2)) + 2 * align_up(rows * 4) + align_up(rows * cap * 2) +
+         align_up(rows * cap * 4) + align_up(4) + align_up(rows * 4);
+}
+
+bool dense_tile_eligible(const AttnParams& P) {
+  if (P.sel || P.hd != HDT || P.kv.hd != HDT) return false;
+  if (P.kv.base_bits != 8 || (P.kv.g != 32 && P.kv.g != 64)) return false;
+  if (P.kv.n_tok > 65535 || P.loop > 31) return false;
+  for (int r = 2; r <= P.loop; ++r) {
+    const int b = P.kv.res_bits[r];
+    if (b != 2 && b != 4 && b != 8) return false;
+  }
+  if (P.sel_out && P.stat_kind == FL_STAT_PV && !P.vnorm) return false;
+  if (P.sel_out && (P.k_next < 1 || P.k_next + 1 > P.out_stride)) return false;
+  // rows the candidates cannot rank are finished by the per-query kernel
+  if (P.sel_out && !dense_rows_supported(P)) return false;
+  return true;
+}
+
+cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s) {
+  static bool attr_set[128] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_attn_dense_tile,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  DenseArgs A{};
+  A.P = P;
+  A.k = P.k_next;
+  A.cap = P.k_next + 1024;
+  const size_t rows = (size_t)P.H * P.n_q;
+  int* ovf_n = nullptr;
+  int* ovf_list = nullptr;
+  if (P.sel_out) {
+    uint8_t* p = static_cast<uint8_t*>(ws);
+    A.m1l = reinterpret_cast<float2*>(p); p += align_up(rows * sizeof(float2));
+    A.cnt = reinterpret_cast<int*>(p); p += align_up(rows * 4);
+    A.p0 = reinterpret_cast<float*>(p); p += align_up(rows * 4);
+    A.ccol = reinterpret_cast<uint16_t*>(p); p += align_up(rows * A.cap * 2);
+    A.cp = reinterpret_cast<float*>(p); p += align_up(rows * A.cap * 4);
+    ovf_n = reinterpret_cast<int*>(p); p += align_up(4);
+    ovf_list = reinterpret_cast<int*>(p);
+    cudaError_t e = cudaMemsetAsync(ovf_n, 0, sizeof(int), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int n_tiles = (P.n_q + TQ - 1) / TQ;
+  A.mode = P.sel_out ? 1 : 0;
+  cudaError_t e = launch_pdl(k_attn_dense_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  if (!P.sel_out) return cudaGetLastError();
+  const size_t sel_smem = (size_t)A.cap * 10 + 16;
+  static int sel_attr[128] = {0};
+  if ((int)sel_smem > sel_attr[dev]) {
+    e = cudaFuncSetAttribute(k_dense_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem);
+    if (e != cudaSuccess) return e;
+    sel_attr[dev] = (int)sel_smem;
+  }
+  k_dense_select<<<(unsigned)rows, SEL_THREADS, sel_smem, s>>>(A, ovf_n, ovf_list);
+  count_launch();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  A.mode = 2;
+  e = launch_pdl(k_attn_dense_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return launch_attn_dense_rows(P, ovf_list, ovf_n, s);
+}
+
+}  // namespace fl

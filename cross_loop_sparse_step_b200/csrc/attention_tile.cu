@@ -30,23 +30,17 @@
 // the call writes no statistics (none requested, or in place with an unchanged budget).
 #include <float.h>
 
-#include "fl_internal.cuh"
-#include "sm100_ptx.cuh"
+#include "attn_tile_common.cuh"
 
 namespace fl {
 namespace {
 
 using namespace sm100;
+using namespace tile;
 
-constexpr int TQ = 128;            // queries per tile = TMEM lanes = MMA M
-constexpr int TC = 128;            // union columns per chunk
-constexpr int HDT = 128;           // head_dim
 constexpr int NWARPS = 13;         // 0-3, 8-11 producers; 4-7 softmax; 12 MMA
 constexpr int NTHR = NWARPS * 32;
-constexpr uint32_t TILE = TQ * HDT * 2;          // one fp16 128 x 128 operand tile
 constexpr int MAX_WORDS = 2048;                  // bitmap words for n_tok <= 65535
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescale = 8.f;                  // log2 growth of the maximum that rescales O
 
 // dynamic shared memory (1024-byte aligned base)
 constexpr uint32_t OFF_Q = 0;
@@ -64,85 +58,6 @@ struct TileShared {
   int n_union;
   int scan[NWARPS];
 };
-
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
-  const __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Dequantised residual codes of `BITS` bits for elements [e0, e0 + 16) of a stored row,
-// added to acc in binary32: acc += fmaf(code, s, z).
-template <int BITS>
-__device__ __forceinline__ void add_residual16(const uint8_t* row_codes, uint32_t szw, int e0,
-                                               float* acc) {
-  const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
-  const float z = half_bits_to_float((uint16_t)(szw >> 16));
-  uint32_t w[BITS / 2];
-  if constexpr (BITS == 8) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row_codes + e0));
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  } else if constexpr (BITS == 4) {
-    const uint2 v = __ldg(reinterpret_cast<const uint2*>(row_codes + e0 / 2));
-    w[0] = v.x; w[1] = v.y;
-  } else {
-    w[0] = __ldg(reinterpret_cast<const uint32_t*>(row_codes + e0 / 4));
-  }
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int bit = i * BITS;
-    const uint32_t c = (w[bit >> 5] >> (bit & 31)) & ((1u << BITS) - 1u);
-    acc[i] = __fadd_rn(acc[i], __fmaf_rn((float)c, s, z));
-  }
-}
-
-// The base row of K or V (which = 0 / 1) of token `col`, head h: 128 int8 codes and the
-// (s, z) pairs of its groups, loaded together so one round of memory latency covers them.
-struct BaseRow {
-  uint4 raw[8];
-  uint32_t sz[4];
-};
-
-__device__ __forceinline__ void load_base(const AttnParams& P, int which, int col, int h,
-                                          BaseRow& b) {
-  const KvView& kv = P.kv;
-  const size_t bh = (size_t)col * P.H + h;
-  const uint4* cp = reinterpret_cast<const uint4*>(kv.codes[which][1] + bh * HDT);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) b.raw[k] = __ldg(cp + k);
-  const int ng = HDT / kv.g;
-  const uint32_t* sp = reinterpret_cast<const uint32_t*>(kv.sz[which][1]) + bh * ng;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) b.sz[k] = k < ng ? __ldg(sp + k) : 0u;
-}
-
-// K^ or V^ elements [e0, e0 + 16) of token `col`: the base (already loaded), then the
-// residual rows of the loops in `chain` (bit r set: loop r rewrote the token), added in
-// loop order - the store's reconstruction.
-__device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, int col, int h,
-                                              const BaseRow& b, uint32_t chain, int e0,
-                                              float* acc) {
-  const KvView& kv = P.kv;
-  const int g = kv.g, ng = HDT / g;
-  const uint32_t szw = g == 32 ? b.sz[e0 / 32] : b.sz[e0 / 64];
-  const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
-  const float z = half_bits_to_float((uint16_t)(szw >> 16));
-  const uint32_t w[4] = {b.raw[e0 / 16].x, b.raw[e0 / 16].y, b.raw[e0 / 16].z, b.raw[e0 / 16].w};
-#pragma unroll
-  for (int i = 0; i < 16; ++i)
-    acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
-  while (chain) {
-    const int r = __ffs(chain) - 1;
-    chain &= chain - 1;
-    const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
-    const size_t rh = (size_t)row * P.H + h;
-    const int bits = kv.res_bits[r];
-    const uint32_t rsz =
-        __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g);
-    if (bits == 2) add_residual16<2>(kv.codes[which][r] + rh * (HDT / 4), rsz, e0, acc);
-    else if (bits == 4) add_residual16<4>(kv.codes[which][r] + rh * (HDT / 2), rsz, e0, acc);
-    else add_residual16<8>(kv.codes[which][r] + rh * HDT, rsz, e0, acc);
-  }
-}
 
 // rank of token `col` among the union's columns (col must be in the union)
 __device__ __forceinline__ int union_rank(const uint32_t* bits, const uint16_t* pre, int col) {
@@ -315,7 +230,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
     float m_used = -INFINITY, lsum = 0.f;
     const float m_in = valid ? P.mass[(size_t)h * P.stat_rows + srow] : 0.f;
     uint8_t* pt = smem + OFF_P;
-    for (int c = 0; c < n_chunks && !*abort; ++c) {
+    for (int c = 0; c < n_chunks; ++c) {   // leaves only through warp-uniform waits
       uint32_t mask[4] = {0u, 0u, 0u, 0u};
       const int lo = c * TC, hi = lo + TC;
       while (true) {
@@ -332,9 +247,11 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
         if (gmax < hi && !ended) take_next();
         else break;
       }
+      __syncwarp();   // reconverge before the warp-collective TMEM accesses
       const int sb = c & 1;
-      if (!mbar_wait(&sh.s_full[sb], (c >> 1) & 1, abort)) break;
-      if (!mbar_wait(&sh.meta_full[sb], (c >> 1) & 1, abort)) break;
+      // waits agree across the warp: the TMEM loads below are warp-collective
+      if (!warp_wait(&sh.s_full[sb], (c >> 1) & 1, abort)) break;
+      if (!warp_wait(&sh.meta_full[sb], (c >> 1) & 1, abort)) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = biasbuf + sb * TC;
@@ -355,10 +272,10 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       }
       // P of the previous chunk must have been consumed (and O completed) before P is
       // rewritten or O rescaled
-      if (c > 0 && !mbar_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+      if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
       tc_fence_after();
-      if (rescale) {
-        lsum *= alpha;
+      if (rescale) lsum *= alpha;
+      if (__any_sync(0xffffffffu, rescale)) {   // warp-collective; alpha = 1 elsewhere
         const uint32_t o_addr = tmem + lane_base + 2u * TC;
 #pragma unroll 1
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -394,9 +311,10 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       mbar_arrive(&sh.p_full);
     }
     // ---- output: o = u + m * O / sum
-    if (n_chunks > 0 && !*abort) mbar_wait(&sh.pv_done, (n_chunks - 1) & 1, abort);
+    bool done_ok = !*abort;
+    if (n_chunks > 0 && done_ok) done_ok = mbar_wait(&sh.pv_done, (n_chunks - 1) & 1, abort);
     tc_fence_after();
-    if (!*abort) {
+    if (__all_sync(0xffffffffu, done_ok)) {
       const uint32_t o_addr = tmem + lane_base + 2u * TC;
       const float f = (valid && lsum > 0.f) ? m_in / lsum : 0.f;
       const float* u = valid ? P.unsel + ((size_t)h * P.stat_rows + srow) * HDT : nullptr;
@@ -474,8 +392,9 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
     const float* bias_g = P.bias;
     uint8_t* k_tile = smem + OFF_K0 + 2 * grp * TILE;
     uint8_t* v_tile = k_tile + TILE;
-    for (int c = grp; c < n_chunks && !*abort; c += 2) {
-      if (c >= 2 && !mbar_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort)) break;
+    for (int c = grp; c < n_chunks; c += 2) {
+      if (__any_sync(0xffffffffu, *abort != 0)) break;   // warp-uniform exit
+      if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort)) break;
       // column of rank c * TC + jj: the last word whose prefix <= rank, then the bit
       const int R = c * TC + jj;
       int col = -1;

@@ -423,6 +423,8 @@ fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream) {
   fl_status st = check_attn(a);
   if (st != FL_OK) return st;
   if (a->n_q == 0) return FL_OK;
+  const size_t need = attention_ws_bytes(*a);
+  if (need) FL_CHECK(a->ws && a->ws_bytes >= need, FL_ERR_WORKSPACE);
   return cuda_st(launch_attention_timed(*a, status_word(), S(stream)));
 }
 
@@ -510,8 +512,23 @@ fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n
 }
 
 // ---------------------------------------------------------------- loop step
-static size_t loop_ws_layout(const fl_model* m, Carver* c, int32_t** iota, float** delta,
-                             float** q, float** k, float** v, void** attn, void** blk) {
+// Workspace of the dense attention calls of a schedule that hand statistics to a sparse
+// successor: every token queries, with the largest such budget (an upper bound).
+static size_t loop_attn_ws(const fl_model* m, const fl_schedule* s) {
+  if (!s) return 0;
+  int kmax = 0;
+  for (int r = 1; r < s->n_loops && r < FL_MAX_LOOPS; ++r)
+    if ((r == 1 || s->col_k[r] == 0) && s->col_k[r + 1] > kmax) kmax = s->col_k[r + 1];
+  if (kmax == 0) return 0;
+  AttnParams P{};
+  P.H = m->n_heads; P.hd = m->head_dim; P.n_q = m->n_tok; P.k_next = kmax;
+  P.sel_out = reinterpret_cast<uint16_t*>(1);
+  return dense_tile_ws_bytes(P);
+}
+
+static size_t loop_ws_layout(const fl_model* m, const fl_schedule* sc, Carver* c, int32_t** iota,
+                             float** delta, float** q, float** k, float** v, void** attn,
+                             void** blk, void** att_ws, size_t* att_bytes) {
   const size_t N = m->n_tok, d = m->d_model;
   *iota = (int32_t*)c->take(N * 4);
   *delta = (float*)c->take(N * 4);
@@ -520,15 +537,16 @@ static size_t loop_ws_layout(const fl_model* m, Carver* c, int32_t** iota, float
   *v = (float*)c->take(N * d * 4);
   *attn = c->take(N * d * dt_size(m->dt));
   *blk = c->take(block_ws(m, (int)N));
+  *att_bytes = loop_attn_ws(m, sc);
+  *att_ws = *att_bytes ? c->take(*att_bytes) : nullptr;
   return c->off;
 }
 
 size_t fl_loop_step_workspace_bytes(const fl_model* m, const fl_schedule* s) {
-  (void)s;
   if (!m || m->n_tok <= 0) return 0;
   Carver c(nullptr);
-  int32_t* i; float *dl, *q, *k, *v; void *a, *b;
-  return loop_ws_layout(m, &c, &i, &dl, &q, &k, &v, &a, &b);
+  int32_t* i; float *dl, *q, *k, *v; void *a, *b, *aw; size_t ab;
+  return loop_ws_layout(m, s, &c, &i, &dl, &q, &k, &v, &a, &b, &aw, &ab);
 }
 
 fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* sc, int32_t loop,
@@ -575,8 +593,8 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
   cudaStream_t s = S(stream);
   int* sw = status_word();
   Carver c(st->ws);
-  int32_t* iota; float *delta, *q, *k, *v; void *attn, *blk;
-  loop_ws_layout(m, &c, &iota, &delta, &q, &k, &v, &attn, &blk);
+  int32_t* iota; float *delta, *q, *k, *v; void *attn, *blk, *att_ws; size_t att_bytes;
+  loop_ws_layout(m, sc, &c, &iota, &delta, &q, &k, &v, &attn, &blk, &att_ws, &att_bytes);
   if (st->delta) delta = st->delta;
   FL_TRY(launch_iota(iota, N, s));
 
@@ -656,6 +674,7 @@ fl_status fl_loop_step(const fl_model* m, fl_loop_state* st, const fl_schedule* 
       a.stat_kind = sc->stat_kind;
     }
     a.out = attn; a.out_dt = m->dt;
+    a.ws = att_ws; a.ws_bytes = att_bytes;
     FL_TRY(tap_rows(q, tap ? tp->q : nullptr, row_bytes, l));
     FL_TRY(tap_rows(k, tap ? tp->k : nullptr, row_bytes, l));
     FL_TRY(tap_rows(v, tap ? tp->v : nullptr, row_bytes, l));

@@ -158,6 +158,14 @@ size_t attention_batched_ws_bytes(int n);
 cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, int* st,
                                      cudaStream_t s);
 bool dense_fast_eligible(const AttnParams& P);
+// The tensor-core dense producer (query tiles; statistics by candidates and an exact
+// selection), its workspace, and the per-query exact finish of listed rows.
+bool dense_tile_eligible(const AttnParams& P);
+size_t dense_tile_ws_bytes(const AttnParams& P);
+cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s);
+bool dense_rows_supported(const AttnParams& P);
+cudaError_t launch_attn_dense_rows(const AttnParams& P, const int* list, const int* count,
+                                   cudaStream_t s);
 cudaError_t launch_attn_dense_fast(const AttnParams& P, cudaStream_t s);
 
 template <typename T> __device__ __forceinline__ float to_f32(T x);

@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const int pass = pass_of(mode, G, nc);
       const int c = G % nc;
       const int sb = G & 1;
-      if (!warp_wait(&sh.s_full[sb], (G >> 1) & 1, abort)) break;
-      if (!warp_wait(&sh.meta_full[sb], (G >> 1) & 1, abort)) break;
+      if (!warp_wait(&sh.s_full[sb], (G >> 1) & 1, abort, 1 + 16 * mode)) break;
+      if (!warp_wait(&sh.meta_full[sb], (G >> 1) & 1, abort, 2 + 16 * mode)) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = meta + sb * TC;
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           if (m_used != -INFINITY && lsum > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
           m_used = cmax;
         }
-        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 3 + 16 * mode)) break;
         tc_fence_after();
         if (rescale) lsum *= alpha;
         if (__any_sync(0xffffffffu, rescale)) {
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         mbar_arrive(&sh.p_full);
         if (c == nc - 1) {
           // ---- end of the flash pass: o = O / sum; the row's maximum and sum
-          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort)) break;
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, 4 + 16 * mode)) break;
           tc_fence_after();
           const uint32_t o_addr = tmem + lane_base + 2u * TC;
           const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           // every row's histogram read: the region becomes Q lo (a bounded wait, not a
           // named barrier, so an aborted warp cannot hold the others)
           mbar_arrive(&sh.hist_done);
-          if (!warp_wait(&sh.hist_done, 0, abort)) break;
+          if (!warp_wait(&sh.hist_done, 0, abort, 5 + 16 * mode)) break;
           uint8_t* ql = smem + OFF_R1;
           for (int e0 = 0; e0 < HDT; e0 += 8) {
             float x[8];
@@ -425,7 +425,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           else break;
         }
         __syncwarp();   // reconverge before the warp-collective TMEM accesses
-        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 11 + 16 * mode)) break;
         tc_fence_after();
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -451,7 +451,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         tc_fence_before();
         mbar_arrive(&sh.p_full);
         if (c == nc - 1) {
-          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort)) break;
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, 12 + 16 * mode)) break;
           tc_fence_after();
           const uint32_t o_addr = tmem + lane_base + 2u * TC;
           const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
@@ -479,9 +479,9 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       auto issue_qk = [&](int G) -> bool {
         const int pass = pass_of(mode, G, nc);
         const int st = G & 1;
-        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort, 6 + 16 * mode)) return false;
         if (pass == PASS_CAND && !qlo_seen) {
-          if (!mbar_wait(&sh.qlo_ready, 0, abort)) return false;
+          if (!mbar_wait(&sh.qlo_ready, 0, abort, 7 + 16 * mode)) return false;
           qlo_seen = true;
         }
         tc_fence_after();
@@ -499,13 +499,12 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           }
         }
         mma_commit(&sh.s_full[st]);
-        if (!has_pv(pass)) mma_commit(&sh.kv_empty[st]);
         return true;
       };
       bool ok = issue_qk(0);
       for (int G = 0; ok && G < total; ++G) {
         if (G + 1 < total && !issue_qk(G + 1)) break;
-        if (!mbar_wait(&sh.p_full, G & 1, abort)) break;
+        if (!mbar_wait(&sh.p_full, G & 1, abort, 8 + 16 * mode)) break;
         tc_fence_after();
         const int pass = pass_of(mode, G, nc);
         if (has_pv(pass)) {
@@ -519,8 +518,10 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
                      (c > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&sh.pv_done);
-          mma_commit(&sh.kv_empty[st]);
         }
+        // the stage (operand tiles and its column metadata) is free once the softmax has
+        // handed the chunk back - also in passes without P V^, whose metadata it reads
+        mma_commit(&sh.kv_empty[G & 1]);
       }
     }
     if (lane == 0) mma_commit(&sh.fin);
@@ -533,7 +534,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     const bool pv_stat = P.stat_kind == FL_STAT_PV && P.vnorm;
     for (int G = grp; G < total; G += 2) {
       if (__any_sync(0xffffffffu, *abort != 0)) break;
-      if (G >= 2 && !warp_wait(&sh.kv_empty[grp], ((G >> 1) - 1) & 1, abort)) break;
+      if (G >= 2 && !warp_wait(&sh.kv_empty[grp], ((G >> 1) - 1) & 1, abort, 9 + 16 * mode)) break;
       const int pass = pass_of(mode, G, nc);
       const int c = G % nc;
       const int colv = c * TC + jj;
@@ -601,13 +602,13 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     if (lane == 0) {
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(&sh.fin, 0))
-        if (globaltimer() - t0 > kWaitLimitNs) { sh.abort_flag = 1; break; }
+        if (globaltimer() - t0 > kWaitLimitNs) { atomicCAS(&sh.abort_flag, 0, 10 + 16 * mode); break; }
     }
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, FL_ERR_TIMEOUT);
+  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
 // ---------------------------------------------------------------- kernel B: selection

@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       __syncwarp();   // reconverge before the warp-collective TMEM accesses
       const int sb = c & 1;
       // waits agree across the warp: the TMEM loads below are warp-collective
-      if (!warp_wait(&sh.s_full[sb], (c >> 1) & 1, abort)) break;
-      if (!warp_wait(&sh.meta_full[sb], (c >> 1) & 1, abort)) break;
+      if (!warp_wait(&sh.s_full[sb], (c >> 1) & 1, abort, 101)) break;
+      if (!warp_wait(&sh.meta_full[sb], (c >> 1) & 1, abort, 102)) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = biasbuf + sb * TC;
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       }
       // P of the previous chunk must have been consumed (and O completed) before P is
       // rewritten or O rescaled
-      if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort)) break;
+      if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 103)) break;
       tc_fence_after();
       if (rescale) lsum *= alpha;
       if (__any_sync(0xffffffffu, rescale)) {   // warp-collective; alpha = 1 elsewhere
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
     }
     // ---- output: o = u + m * O / sum
     bool done_ok = !*abort;
-    if (n_chunks > 0 && done_ok) done_ok = mbar_wait(&sh.pv_done, (n_chunks - 1) & 1, abort);
+    if (n_chunks > 0 && done_ok) done_ok = mbar_wait(&sh.pv_done, (n_chunks - 1) & 1, abort, 104);
     tc_fence_after();
     if (__all_sync(0xffffffffu, done_ok)) {
       const uint32_t o_addr = tmem + lane_base + 2u * TC;
@@ -353,7 +353,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       const uint32_t p_base = smem_u32(smem + OFF_P);
       auto issue_qk = [&](int c) -> bool {
         const int st = c & 1;
-        if (!mbar_wait(&sh.kv_full[st], (c >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&sh.kv_full[st], (c >> 1) & 1, abort, 106)) return false;
         tc_fence_after();
         const uint32_t k_base = smem_u32(smem + OFF_K0 + 2 * st * TILE);
         const uint32_t d = tmem + (uint32_t)(st * TC);
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       bool ok = issue_qk(0);
       for (int c = 0; ok && c < n_chunks; ++c) {
         if (c + 1 < n_chunks && !issue_qk(c + 1)) break;
-        if (!mbar_wait(&sh.p_full, c & 1, abort)) break;
+        if (!mbar_wait(&sh.p_full, c & 1, abort, 108)) break;
         tc_fence_after();
         const int st = c & 1;
         const uint32_t v_base = smem_u32(smem + OFF_K0 + (2 * st + 1) * TILE);
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
     uint8_t* v_tile = k_tile + TILE;
     for (int c = grp; c < n_chunks; c += 2) {
       if (__any_sync(0xffffffffu, *abort != 0)) break;   // warp-uniform exit
-      if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort)) break;
+      if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort, 109)) break;
       // column of rank c * TC + jj: the last word whose prefix <= rank, then the bit
       const int R = c * TC + jj;
       int col = -1;
@@ -459,13 +459,13 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
     if (lane == 0) {
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(&sh.fin, 0))
-        if (globaltimer() - t0 > kWaitLimitNs) { sh.abort_flag = 1; break; }
+        if (globaltimer() - t0 > kWaitLimitNs) { atomicCAS(&sh.abort_flag, 0, 110); break; }
     }
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, FL_ERR_TIMEOUT);
+  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
 }  // namespace

@@ -19,8 +19,9 @@ constexpr float kRescale = 8.f;    // log2 growth of the maximum that rescales O
 
 // mbar_wait whose outcome agrees across the (converged) warp: false on every lane if it
 // failed on any, so warp-collective TMEM accesses that follow stay aligned.
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int site = 1) {
+  const bool ok = mbar_wait(bar, parity, abort, site);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -103,6 +104,11 @@ __device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, in
   }
 }
 
+
+// Status word value of a bounded wait that ran out: FL_ERR_TIMEOUT in the low byte, the
+// wait's site code above it (fl_check_device_status returns the low byte and keeps the
+// site for fl_last_error_detail).
+__device__ __forceinline__ int timeout_code(int site) { return FL_ERR_TIMEOUT | (site << 8); }
 
 }  // namespace tile
 }  // namespace fl

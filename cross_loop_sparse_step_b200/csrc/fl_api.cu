@@ -75,14 +75,20 @@ void timing_end(int kind, cudaStream_t s) {
   if (h.next < (int)h.end.size()) record_event(h.end[h.next++], s);
 }
 
+static std::atomic<long long> g_bf16_simt{0};
+
 cudaError_t launch_gemm(fl_dtype dt, const void* A, const void* W, float* C, int M, int N,
                         int K, int ldc, GemmEpi epi, cudaStream_t s, const GemmScratch* scr) {
   timing_begin(TIMED_GEMM, s);
   cudaError_t e;
-  if (dt == FL_BF16 && gemm_tc_supported(M, N, K))
+  if (dt == FL_BF16 && gemm_tc_supported(M, N, K)) {
     e = launch_gemm_tc(A, W, C, M, N, K, ldc, epi, s, scr);
-  else
+  } else {
+    // binary32 projections always run here; a bf16 one only when its shape cannot be
+    // tiled for the tensor cores - counted, so that a caller can see it happened
+    if (dt == FL_BF16) g_bf16_simt.fetch_add(1, std::memory_order_relaxed);
     e = launch_gemm_simt(dt, A, W, C, M, N, K, ldc, epi, s);
+  }
   timing_end(TIMED_GEMM, s);
   return e;
 }
@@ -301,6 +307,8 @@ const char* fl_version(void) { return "0.1.0"; }
 
 int64_t fl_launch_count(void) { return (int64_t)g_launches.load(); }
 
+int64_t fl_gemm_bf16_cuda_core_count(void) { return (int64_t)g_bf16_simt.load(); }
+
 fl_status fl_set_timing_events(int32_t kind, void* const* begin, void* const* end, int32_t n) {
   FL_CHECK(kind >= 0 && kind < TIMED_KINDS && n >= 0, FL_ERR_INVALID_ARG);
   FL_CHECK(n == 0 || (begin && end), FL_ERR_INVALID_ARG);
@@ -318,14 +326,19 @@ int32_t fl_timing_recorded(int32_t kind) {
   return g_hooks[kind].next;
 }
 
+static std::atomic<int> g_last_detail{0};
+
 fl_status fl_check_device_status(void* stream) {
   if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return FL_ERR_CUDA;
   int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_fl_status, sizeof(int)) != cudaSuccess) return FL_ERR_CUDA;
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_fl_status, &zero, sizeof(int)) != cudaSuccess) return FL_ERR_CUDA;
-  return (fl_status)v;
+  g_last_detail.store(v >> 8);
+  return (fl_status)(v & 0xFF);
 }
+
+int32_t fl_last_error_detail(void) { return g_last_detail.load(); }
 
 size_t fl_select_active_workspace_bytes(int32_t n_rows) {
   return n_rows > 0 ? align_up((size_t)n_rows * 4) : 0;

@@ -53,15 +53,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity; false if the CTA aborted or the wait ran
-// out (then the abort flag is set).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// out. The first wait of a CTA that runs out writes its `site` (a nonzero code naming
+// the wait) into the abort flag, so the CTA can report where it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int site = 1) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > kWaitLimitNs) {
-      *abort = 1;
+      atomicCAS(const_cast<int*>(abort), 0, site);
       return false;
     }
   }

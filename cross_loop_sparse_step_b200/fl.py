@@ -99,6 +99,7 @@ def _sig(name, res, args):
 _status_str = _sig("fl_status_str", ctypes.c_char_p, [c_i32])
 _version = _sig("fl_version", ctypes.c_char_p, [])
 _check = _sig("fl_check_device_status", c_i32, [vp])
+_detail = _sig("fl_last_error_detail", c_i32, [])
 _sel_ws = _sig("fl_select_active_workspace_bytes", c_sz, [c_i32])
 _select = _sig("fl_select_active", c_i32,
                [vp, vp, c_i32, c_i32, c_i32, vp, c_i32, vp, vp, vp, vp, c_sz, vp])
@@ -168,6 +169,11 @@ def stream_handle(stream=None):
 def check_device_status(stream=None):
     """Synchronise and return (and clear) the device status word (0 = ok)."""
     return _check(stream_handle(stream))
+
+
+def last_error_detail():
+    """Detail of the last status returned (for a timed-out wait: the wait's site code)."""
+    return _detail()
 
 
 # ---------------------------------------------------------------- entry points

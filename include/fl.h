@@ -61,6 +61,12 @@ const char* fl_version(void);
 /* Number of kernel launches the library has issued in this process. */
 int64_t fl_launch_count(void);
 
+/* Number of bf16 projection GEMMs that ran on the CUDA-core kernel instead of the
+ * tensor cores because their shape cannot be tiled (K not a multiple of 64 or N not a
+ * multiple of 128), in this process. Binary32 projections always use the CUDA cores
+ * and are not counted. */
+int64_t fl_gemm_bf16_cuda_core_count(void);
+
 /* Measurement hook. With n > 0 the library records the caller's events begin[i] and
  * end[i] (each a cudaEvent_t passed as void*) on the launch stream around its next n
  * launches of one kind (0: the projection GEMMs, 1: the attention kernel);
@@ -73,6 +79,10 @@ int32_t fl_timing_recorded(int32_t kind);
 /* Synchronises `stream`, returns the first error a kernel recorded on the current
  * device since the last call (FL_OK if none) and clears it. */
 fl_status fl_check_device_status(void* stream);
+/* Detail of the error the last fl_check_device_status returned: for FL_ERR_TIMEOUT from
+ * a tensor-core attention kernel, the code of the wait that ran out (which kernel, role
+ * and barrier; listed beside the kernels' sources); 0 when there is none. */
+int32_t fl_last_error_detail(void);
 
 /* ------------------------------------------------------------------------- *
  * Active-token selection (§4.1): rank the rows updated in the previous loop by

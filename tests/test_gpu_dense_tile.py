@@ -87,7 +87,7 @@ def test_dense_tile_matches_oracle(name, n, H, g, loop, k, nq, use_bias, sample,
                         col_bias=dev(bias) if bias is not None else None, k_next=k, sel_out=S,
                         mass_out=m, unsel_out=u, stat_kind=kind)
     st = fl.check_device_status()
-    assert st == 0, fl.status_str(st)
+    assert st == 0, (fl.status_str(st), fl.last_error_detail())
     pick = np.sort(rs.choice(len(q_tok), size=min(sample, len(q_tok)), replace=False))
     pick = np.unique(np.concatenate([pick, [0, len(q_tok) - 1]]))
     qt = q_tok[pick]

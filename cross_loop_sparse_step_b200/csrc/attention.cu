@@ -62,8 +62,9 @@ __device__ __forceinline__ int col_of(const uint16_t* cols, int idx) {
   return cols ? (int)cols[idx] : idx;
 }
 
+// One CTA's work: query qi, head h (every early return is CTA-uniform).
 template <int NT, int EPL>
-__global__ void __launch_bounds__(NT) k_attention(AttnParams P, int max_cols) {
+__device__ __forceinline__ void attention_cta(const AttnParams& P, int max_cols, int qi, int h) {
   extern __shared__ __align__(16) uint8_t smem[];
   constexpr int NG = NT / 8;                    // column groups
   float* p = reinterpret_cast<float*>(smem);    // [max_cols] scores, then probabilities
@@ -74,8 +75,6 @@ __global__ void __launch_bounds__(NT) k_attention(AttnParams P, int max_cols) {
   uint16_t* cols = P.sel ? reinterpret_cast<uint16_t*>(mark + ((max_cols + 15) & ~15)) : nullptr;
   __shared__ float s_red[32];
 
-  const int qi = blockIdx.x / P.H;
-  const int h = blockIdx.x % P.H;
   const int tid = threadIdx.x;
   const int grp = tid >> 3, li = tid & 7;
   const int hd = P.hd;
@@ -296,6 +295,24 @@ __global__ void __launch_bounds__(NT) k_attention(AttnParams P, int max_cols) {
   (void)n_keep;
 }
 
+template <int NT, int EPL>
+__global__ void __launch_bounds__(NT) k_attention(AttnParams P, int max_cols) {
+  attention_cta<NT, EPL>(P, max_cols, blockIdx.x / P.H, blockIdx.x % P.H);
+}
+
+// The (query, head) pairs list[0, *count) (entries h * n_q + query), CTAs striding over
+// the list: the exact finish of rows the tensor-core dense producer could not rank.
+template <int NT, int EPL>
+__global__ void __launch_bounds__(NT) k_attention_list(AttnParams P, int max_cols,
+                                                       const int* list, const int* count) {
+  const int n = *count;
+  for (int x = blockIdx.x; x < n; x += gridDim.x) {
+    __syncthreads();   // the previous row's shared-memory reads are done
+    const int rh = list[x];
+    attention_cta<NT, EPL>(P, max_cols, rh % P.n_q, rh / P.n_q);
+  }
+}
+
 size_t smem_bytes(int nt, int hd, int max_cols, bool sparse) {
   const int NG = nt / 8;
   size_t b = (size_t)max_cols * 4 + 2 * (size_t)NG * hd * 4 + 320 * 4;
@@ -324,6 +341,34 @@ cudaError_t launch_t(const AttnParams& P, int max_cols, cudaStream_t s) {
 }
 
 }  // namespace
+
+// Listed rows of a dense call with statistics, by the general kernel (any store).
+bool dense_list_supported(const AttnParams& P) {
+  return smem_bytes(256, P.hd, P.kv.n_tok, false) <= 227 * 1024;
+}
+
+cudaError_t launch_attention_list(const AttnParams& P, const int* list, const int* count,
+                                  cudaStream_t s) {
+  const int max_cols = P.kv.n_tok;
+  const size_t sm = smem_bytes(256, P.hd, max_cols, false);
+  if (sm > 227 * 1024) return cudaErrorInvalidValue;
+  auto kern = P.hd == 128 ? k_attention_list<256, 16> : k_attention_list<256, 8>;
+  static int attr_bytes[2][128] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  int& have = attr_bytes[P.hd == 128 ? 1 : 0][dev];
+  if ((int)sm > have) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    have = (int)sm;
+  }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  kern<<<sms, 256, sm, s>>>(P, max_cols, list, count);
+  count_launch();
+  return cudaGetLastError();
+}
 
 static bool attn_tile_enabled();
 

@@ -295,8 +295,10 @@ __global__ void __launch_bounds__(128) k_attn_dense_list(const __grid_constant__
 
 }  // namespace
 
+// The warp-per-query kernel reads the 8-bit base alone: loop 1 of a quantised store.
 bool dense_rows_supported(const AttnParams& P) {
-  return P.hd == 128 && P.kv.base_bits == 8 && dense_warp_smem(P.kv.n_tok) <= 200 * 1024;
+  return P.hd == 128 && P.loop == 1 && P.kv.base_bits == 8 &&
+         dense_warp_smem(P.kv.n_tok) <= 200 * 1024;
 }
 
 cudaError_t launch_attn_dense_rows(const AttnParams& P, const int* list, const int* count,

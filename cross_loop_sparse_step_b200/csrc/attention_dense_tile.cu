@@ -74,6 +74,11 @@ struct DenseShared {
   int t_max;
 };
 
+// code of a wait for the timeout report: the site, the chunk step and the warp
+__device__ __forceinline__ int site_of(int site, int G, int warp) {
+  return site | (min(G, 4095) << 8) | ((warp & 15) << 20);
+}
+
 __device__ __forceinline__ int pass_of(int mode, int G, int nc) {
   if (mode == 2) return PASS_UNSEL;
   if (mode == 0) return PASS_FLASH;
@@ -230,8 +235,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const int pass = pass_of(mode, G, nc);
       const int c = G % nc;
       const int sb = G & 1;
-      if (!warp_wait(&sh.s_full[sb], (G >> 1) & 1, abort, 1 + 16 * mode)) break;
-      if (!warp_wait(&sh.meta_full[sb], (G >> 1) & 1, abort, 2 + 16 * mode)) break;
+      if (!warp_wait(&sh.s_full[sb], (G >> 1) & 1, abort, site_of(1 + 16 * mode, G, warp))) break;
+      if (!warp_wait(&sh.meta_full[sb], (G >> 1) & 1, abort, site_of(2 + 16 * mode, G, warp))) break;
       tc_fence_after();
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = meta + sb * TC;
@@ -259,7 +264,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           if (m_used != -INFINITY && lsum > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
           m_used = cmax;
         }
-        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 3 + 16 * mode)) break;
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, site_of(3 + 16 * mode, G, warp))) break;
         tc_fence_after();
         if (rescale) lsum *= alpha;
         if (__any_sync(0xffffffffu, rescale)) {
@@ -298,7 +303,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         mbar_arrive(&sh.p_full);
         if (c == nc - 1) {
           // ---- end of the flash pass: o = O / sum; the row's maximum and sum
-          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, 4 + 16 * mode)) break;
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, site_of(4 + 16 * mode, G, warp))) break;
           tc_fence_after();
           const uint32_t o_addr = tmem + lane_base + 2u * TC;
           const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
@@ -361,7 +366,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           // every row's histogram read: the region becomes Q lo (a bounded wait, not a
           // named barrier, so an aborted warp cannot hold the others)
           mbar_arrive(&sh.hist_done);
-          if (!warp_wait(&sh.hist_done, 0, abort, 5 + 16 * mode)) break;
+          if (!warp_wait(&sh.hist_done, 0, abort, site_of(5 + 16 * mode, G, warp))) break;
           uint8_t* ql = smem + OFF_R1;
           for (int e0 = 0; e0 < HDT; e0 += 8) {
             float x[8];
@@ -425,7 +430,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           else break;
         }
         __syncwarp();   // reconverge before the warp-collective TMEM accesses
-        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 11 + 16 * mode)) break;
+        if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, site_of(11 + 16 * mode, G, warp))) break;
         tc_fence_after();
 #pragma unroll
         for (int g4 = 0; g4 < 4; ++g4) {
@@ -451,7 +456,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         tc_fence_before();
         mbar_arrive(&sh.p_full);
         if (c == nc - 1) {
-          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, 12 + 16 * mode)) break;
+          if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, site_of(12 + 16 * mode, G, warp))) break;
           tc_fence_after();
           const uint32_t o_addr = tmem + lane_base + 2u * TC;
           const float f = (valid && lsum > 0.f) ? 1.f / lsum : 0.f;
@@ -479,9 +484,9 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       auto issue_qk = [&](int G) -> bool {
         const int pass = pass_of(mode, G, nc);
         const int st = G & 1;
-        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort, 6 + 16 * mode)) return false;
+        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort, site_of(6 + 16 * mode, G, warp))) return false;
         if (pass == PASS_CAND && !qlo_seen) {
-          if (!mbar_wait(&sh.qlo_ready, 0, abort, 7 + 16 * mode)) return false;
+          if (!mbar_wait(&sh.qlo_ready, 0, abort, site_of(7 + 16 * mode, G, warp))) return false;
           qlo_seen = true;
         }
         tc_fence_after();
@@ -504,7 +509,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       bool ok = issue_qk(0);
       for (int G = 0; ok && G < total; ++G) {
         if (G + 1 < total && !issue_qk(G + 1)) break;
-        if (!mbar_wait(&sh.p_full, G & 1, abort, 8 + 16 * mode)) break;
+        if (!mbar_wait(&sh.p_full, G & 1, abort, site_of(8 + 16 * mode, G, warp))) break;
         tc_fence_after();
         const int pass = pass_of(mode, G, nc);
         if (has_pv(pass)) {
@@ -534,7 +539,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     const bool pv_stat = P.stat_kind == FL_STAT_PV && P.vnorm;
     for (int G = grp; G < total; G += 2) {
       if (__any_sync(0xffffffffu, *abort != 0)) break;
-      if (G >= 2 && !warp_wait(&sh.kv_empty[grp], ((G >> 1) - 1) & 1, abort, 9 + 16 * mode)) break;
+      if (G >= 2 && !warp_wait(&sh.kv_empty[grp], ((G >> 1) - 1) & 1, abort, site_of(9 + 16 * mode, G, warp))) break;
       const int pass = pass_of(mode, G, nc);
       const int c = G % nc;
       const int colv = c * TC + jj;
@@ -747,16 +752,16 @@ size_t dense_tile_ws_bytes(const AttnParams& P) {
 
 bool dense_tile_eligible(const AttnParams& P) {
   if (P.sel || P.hd != HDT || P.kv.hd != HDT) return false;
-  if (P.kv.base_bits != 8 || (P.kv.g != 32 && P.kv.g != 64)) return false;
+  if ((P.kv.base_bits != 8 && P.kv.base_bits != 0) || (P.kv.g != 32 && P.kv.g != 64)) return false;
   if (P.kv.n_tok > 65535 || P.loop > 31) return false;
   for (int r = 2; r <= P.loop; ++r) {
     const int b = P.kv.res_bits[r];
-    if (b != 2 && b != 4 && b != 8) return false;
+    if (b != 0 && b != 2 && b != 4 && b != 8) return false;
   }
   if (P.sel_out && P.stat_kind == FL_STAT_PV && !P.vnorm) return false;
   if (P.sel_out && (P.k_next < 1 || P.k_next + 1 > P.out_stride)) return false;
-  // rows the candidates cannot rank are finished by the per-query kernel
-  if (P.sel_out && !dense_rows_supported(P)) return false;
+  // rows the candidates cannot rank are finished by a per-query kernel
+  if (P.sel_out && !dense_rows_supported(P) && !dense_list_supported(P)) return false;
   return true;
 }
 
@@ -812,7 +817,10 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   e = launch_pdl(k_attn_dense_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
   count_launch();
   if (e != cudaSuccess) return e;
-  return launch_attn_dense_rows(P, ovf_list, ovf_n, s);
+  // rows whose candidates overflowed: the warp-per-query kernel (loop 1, 8-bit base) or
+  // the general CTA-per-query kernel (any store)
+  if (dense_rows_supported(P)) return launch_attn_dense_rows(P, ovf_list, ovf_n, s);
+  return launch_attention_list(P, ovf_list, ovf_n, s);
 }
 
 }  // namespace fl

@@ -472,11 +472,11 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
 
 bool sparse_tile_eligible(const AttnParams& P) {
   if (P.hd != HDT || P.kv.hd != HDT || !P.sel) return false;
-  if (P.kv.base_bits != 8 || (P.kv.g != 32 && P.kv.g != 64)) return false;
+  if ((P.kv.base_bits != 8 && P.kv.base_bits != 0) || (P.kv.g != 32 && P.kv.g != 64)) return false;
   if (P.kv.n_tok > 65535 || P.loop > 31) return false;
   for (int r = 2; r <= P.loop; ++r) {
     const int b = P.kv.res_bits[r];
-    if (b != 2 && b != 4 && b != 8) return false;
+    if (b != 0 && b != 2 && b != 4 && b != 8) return false;
   }
   // statistics: none requested, or updated in place with an unchanged budget
   if (P.sel_out) {

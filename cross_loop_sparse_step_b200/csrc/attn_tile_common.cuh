@@ -65,6 +65,7 @@ struct BaseRow {
 __device__ __forceinline__ void load_base(const AttnParams& P, int which, int col, int h,
                                           BaseRow& b) {
   const KvView& kv = P.kv;
+  if (kv.base_bits == 0) return;   // binary32 rows are read run by run
   const size_t bh = (size_t)col * P.H + h;
   const uint4* cp = reinterpret_cast<const uint4*>(kv.codes[which][1] + bh * HDT);
 #pragma unroll
@@ -83,19 +84,38 @@ __device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, in
                                               float* acc) {
   const KvView& kv = P.kv;
   const int g = kv.g, ng = HDT / g;
-  const uint32_t szw = g == 32 ? b.sz[e0 / 32] : b.sz[e0 / 64];
-  const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
-  const float z = half_bits_to_float((uint16_t)(szw >> 16));
-  const uint32_t w[4] = {b.raw[e0 / 16].x, b.raw[e0 / 16].y, b.raw[e0 / 16].z, b.raw[e0 / 16].w};
+  if (kv.base_bits == 0) {   // unquantised store: the binary32 values themselves
+    const float4* rp = reinterpret_cast<const float4*>(kv.codes[which][1]) +
+                       ((size_t)col * P.H + h) * (HDT / 4) + e0 / 4;
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
-    acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = __ldg(rp + k);
+      acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
+    }
+  } else {
+    const uint32_t szw = g == 32 ? b.sz[e0 / 32] : b.sz[e0 / 64];
+    const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
+    const float z = half_bits_to_float((uint16_t)(szw >> 16));
+    const uint32_t w[4] = {b.raw[e0 / 16].x, b.raw[e0 / 16].y, b.raw[e0 / 16].z, b.raw[e0 / 16].w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
+  }
   while (chain) {
     const int r = __ffs(chain) - 1;
     chain &= chain - 1;
     const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
     const size_t rh = (size_t)row * P.H + h;
     const int bits = kv.res_bits[r];
+    if (bits == 0) {   // an unquantised loop stores the new value itself
+      const float4* rp = reinterpret_cast<const float4*>(kv.codes[which][r]) + rh * (HDT / 4) + e0 / 4;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 v = __ldg(rp + k);
+        acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
+      }
+      continue;
+    }
     const uint32_t rsz =
         __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g);
     if (bits == 2) add_residual16<2>(kv.codes[which][r] + rh * (HDT / 4), rsz, e0, acc);
@@ -108,7 +128,9 @@ __device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, in
 // Status word value of a bounded wait that ran out: FL_ERR_TIMEOUT in the low byte, the
 // wait's site code above it (fl_check_device_status returns the low byte and keeps the
 // site for fl_last_error_detail).
-__device__ __forceinline__ int timeout_code(int site) { return FL_ERR_TIMEOUT | (site << 8); }
+__device__ __forceinline__ int timeout_code(int site) {
+  return FL_ERR_TIMEOUT | ((site & 0xFFFFFF) << 8);
+}
 
 }  // namespace tile
 }  // namespace fl

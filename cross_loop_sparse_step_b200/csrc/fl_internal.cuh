@@ -164,6 +164,9 @@ bool dense_tile_eligible(const AttnParams& P);
 size_t dense_tile_ws_bytes(const AttnParams& P);
 cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s);
 bool dense_rows_supported(const AttnParams& P);
+bool dense_list_supported(const AttnParams& P);
+cudaError_t launch_attention_list(const AttnParams& P, const int* list, const int* count,
+                                  cudaStream_t s);
 cudaError_t launch_attn_dense_rows(const AttnParams& P, const int* list, const int* count,
                                    cudaStream_t s);
 cudaError_t launch_attn_dense_fast(const AttnParams& P, cudaStream_t s);

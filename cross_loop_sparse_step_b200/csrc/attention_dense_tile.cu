@@ -27,7 +27,10 @@
 // A row whose candidates overflow its buffer (a near-uniform row of more than the buffer's
 // spare capacity in one histogram bin) is finished by the exact per-query kernel.
 // Every wait is bounded; a wait that runs out records FL_ERR_TIMEOUT, the CTA drains its
-// MMAs, frees TMEM and returns. Warp-collective TMEM accesses stay warp-uniform.
+// MMAs, frees TMEM and returns. Warp-collective TMEM accesses stay warp-uniform. The
+// softmax hands each score buffer back on a barrier of its own: in the passes without
+// P V^ nothing else keeps the four softmax warps in step, and with one shared barrier a
+// warp running a chunk ahead would complete the previous chunk's phase early.
 #include <float.h>
 
 #include "attn_tile_common.cuh"
@@ -60,6 +63,7 @@ struct DenseArgs {
   int k;             // the next loop's budget
   int cap;           // candidates per row
   float2* m1l;       // [H][n_q] (final maximum, log2 units; sum)
+  int* dbg;          // [grid][12] a CTA whose wait ran out: site, chunks, t_max, progress
   int* cnt;          // [H][n_q] candidates written (> cap: overflow)
   float* p0;         // [H][n_q] p of the sink column
   uint16_t* ccol;    // [H][n_q][cap]
@@ -67,11 +71,12 @@ struct DenseArgs {
 };
 
 struct DenseShared {
-  uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full, pv_done, qlo_ready, hist_done,
+  uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full[2], pv_done, qlo_ready, hist_done,
       fin;
   uint32_t tmem;
   int abort_flag;
   int t_max;
+  int prog[8];   // progress: softmax warps' last chunk step, MMA's, producer groups', hist arrivals
 };
 
 // code of a wait for the timeout report: the site, the chunk step and the warp
@@ -124,13 +129,16 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       mbar_init(&sh.kv_full[s], 4); mbar_init(&sh.kv_empty[s], 1);
       mbar_init(&sh.meta_full[s], 4); mbar_init(&sh.s_full[s], 1);
     }
-    mbar_init(&sh.p_full, TQ);
+    mbar_init(&sh.p_full[0], TQ);
+    mbar_init(&sh.p_full[1], TQ);
     mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.qlo_ready, TQ);
     mbar_init(&sh.hist_done, TQ);
     mbar_init(&sh.fin, 1);
     sh.abort_flag = 0;
     sh.t_max = -1;
+    for (int k = 0; k < 8; ++k) sh.prog[k] = -1;
+    sh.prog[7] = 0;
     fence_barrier_init();
   }
   if (warp == 12) tmem_alloc(&sh.tmem, 512);
@@ -300,7 +308,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
+        if (lane == 0) sh.prog[warp - 4] = G;
         if (c == nc - 1) {
           // ---- end of the flash pass: o = O / sum; the row's maximum and sum
           if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, site_of(4 + 16 * mode, G, warp))) break;
@@ -352,7 +361,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           }
         }
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
+        if (lane == 0) sh.prog[warp - 4] = G;
         if (c == nc - 1) {
           // ---- the bin of the k-th largest; the candidate threshold one margin below it
           if (sel_row_stats) {
@@ -366,6 +376,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           // every row's histogram read: the region becomes Q lo (a bounded wait, not a
           // named barrier, so an aborted warp cannot hold the others)
           mbar_arrive(&sh.hist_done);
+          atomicAdd(&sh.prog[7], 1);
           if (!warp_wait(&sh.hist_done, 0, abort, site_of(5 + 16 * mode, G, warp))) break;
           uint8_t* ql = smem + OFF_R1;
           for (int e0 = 0; e0 < HDT; e0 += 8) {
@@ -407,7 +418,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           }
         }
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
+        if (lane == 0) sh.prog[warp - 4] = G;
         if (c == nc - 1 && sel_row_stats) {
           A.cnt[rh] = cand;
           A.p0[rh] = p0;
@@ -454,7 +466,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(&sh.p_full);
+        mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
+        if (lane == 0) sh.prog[warp - 4] = G;
         if (c == nc - 1) {
           if (!warp_wait(&sh.pv_done, (nc - 1) & 1, abort, site_of(12 + 16 * mode, G, warp))) break;
           tc_fence_after();
@@ -509,7 +522,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       bool ok = issue_qk(0);
       for (int G = 0; ok && G < total; ++G) {
         if (G + 1 < total && !issue_qk(G + 1)) break;
-        if (!mbar_wait(&sh.p_full, G & 1, abort, site_of(8 + 16 * mode, G, warp))) break;
+        if (!mbar_wait(&sh.p_full[G & 1], (G >> 1) & 1, abort, site_of(8 + 16 * mode, G, warp))) break;
         tc_fence_after();
         const int pass = pass_of(mode, G, nc);
         if (has_pv(pass)) {
@@ -527,6 +540,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         // the stage (operand tiles and its column metadata) is free once the softmax has
         // handed the chunk back - also in passes without P V^, whose metadata it reads
         mma_commit(&sh.kv_empty[G & 1]);
+        sh.prog[4] = G;
       }
     }
     if (lane == 0) mma_commit(&sh.fin);
@@ -598,6 +612,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
+      if (lane == 0 && (warp & 3) == 0) sh.prog[5 + grp] = G;
     }
   }
 
@@ -613,7 +628,14 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
+  if (threadIdx.x == 0 && sh.abort_flag) {
+    record_error(P.st, timeout_code(sh.abort_flag));
+    if (A.dbg) {
+      int* d = A.dbg + (size_t)blockIdx.x * 12;
+      d[0] = sh.abort_flag; d[1] = nc; d[2] = t_max; d[3] = mode;
+      for (int k = 0; k < 8; ++k) d[4 + k] = sh.prog[k];
+    }
+  }
 }
 
 // ---------------------------------------------------------------- kernel B: selection
@@ -747,7 +769,8 @@ size_t dense_tile_ws_bytes(const AttnParams& P) {
   const int cap = P.k_next + 1024;
   const size_t rows = (size_t)P.H * P.n_q;
   return align_up(rows * sizeof(float2)) + 2 * align_up(rows * 4) + align_up(rows * cap * 2) +
-         align_up(rows * cap * 4) + align_up(4) + align_up(rows * 4);
+         align_up(rows * cap * 4) + align_up(4) + align_up(rows * 4) +
+         align_up((size_t)((P.n_q + TQ - 1) / TQ) * P.H * 12 * 4);
 }
 
 bool dense_tile_eligible(const AttnParams& P) {
@@ -792,7 +815,8 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
     A.ccol = reinterpret_cast<uint16_t*>(p); p += align_up(rows * A.cap * 2);
     A.cp = reinterpret_cast<float*>(p); p += align_up(rows * A.cap * 4);
     ovf_n = reinterpret_cast<int*>(p); p += align_up(4);
-    ovf_list = reinterpret_cast<int*>(p);
+    ovf_list = reinterpret_cast<int*>(p); p += align_up(rows * 4);
+    A.dbg = reinterpret_cast<int*>(p);
     cudaError_t e = cudaMemsetAsync(ovf_n, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
   }

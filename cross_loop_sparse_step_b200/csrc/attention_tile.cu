@@ -52,7 +52,7 @@ constexpr uint32_t OFF_BIAS = OFF_PRE + MAX_WORDS * 2;   // [2][TC] float (log2 
 constexpr uint32_t SMEM_BYTES = OFF_BIAS + 2 * TC * 4 + 1024;
 
 struct TileShared {
-  uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full, pv_done, fin;
+  uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full[2], pv_done, fin;
   uint32_t tmem;
   int abort_flag;
   int n_union;
@@ -87,7 +87,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       mbar_init(&sh.kv_full[s], 4); mbar_init(&sh.kv_empty[s], 1);
       mbar_init(&sh.meta_full[s], 4); mbar_init(&sh.s_full[s], 1);
     }
-    mbar_init(&sh.p_full, TQ);
+    mbar_init(&sh.p_full[0], TQ);
+    mbar_init(&sh.p_full[1], TQ);
     mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.fin, 1);
     sh.abort_flag = 0;
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&sh.p_full);
+      mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer
     }
     // ---- output: o = u + m * O / sum
     bool done_ok = !*abort;
@@ -369,7 +370,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
       bool ok = issue_qk(0);
       for (int c = 0; ok && c < n_chunks; ++c) {
         if (c + 1 < n_chunks && !issue_qk(c + 1)) break;
-        if (!mbar_wait(&sh.p_full, c & 1, abort, 108)) break;
+        if (!mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1, abort, 108)) break;
         tc_fence_after();
         const int st = c & 1;
         const uint32_t v_base = smem_u32(smem + OFF_K0 + (2 * st + 1) * TILE);

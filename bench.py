@@ -38,6 +38,42 @@ METRIC = "loop-step tokens/s at R loops + % of HBM/tensor roofline; KV bytes/tok
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# Component toggles and loop schedules (paper §5.3 Figure 4: the contribution of each
+# lazy update; §4.1: dense early loops; §4.2: progressive pruning with smaller budgets).
+VARIANTS = {
+    "flashloop": "all three lazy updates as configured",
+    "dense": "no lazy update: every token, dense attention, unquantised KV in every loop",
+    "token-sparse": "token-sparse updates only: dense attention, unquantised KV",
+    "token+attn": "token-sparse updates and sparse attention, unquantised KV",
+    "dense-early": "loop 2 dense (every token, dense attention), the lazy updates from loop 3",
+    "shrink": "carried column budget halved loop after loop (k, k/2, k/4, ...)",
+}
+
+
+def apply_variant(cfg, variant):
+    """The workload with one of VARIANTS applied (a copy)."""
+    c = dict(cfg)
+    R = c["n_loops"]
+    loops = range(2, R + 1)
+    if variant in ("dense", "token-sparse", "token+attn"):
+        c["base_bits"] = 0
+        c["res_bits"] = {r: 0 for r in loops}
+    if variant in ("dense", "token-sparse"):
+        c["col_k"] = {r: 0 for r in loops}
+    if variant == "dense":
+        c["first_sparse"] = R + 1
+        c["tok_frac"] = {r: 1.0 for r in loops}
+    if variant == "dense-early":
+        c["first_sparse"] = 3
+        c["col_k"] = dict(c["col_k"], **{2: 0})
+        c["tok_frac"] = dict(c["tok_frac"], **{2: 1.0})
+    if variant == "shrink":
+        k0 = c["col_k"][2]
+        c["col_k"] = {r: max(1, k0 >> (r - 2)) for r in loops}
+    c["variant"] = variant
+    return c
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -46,6 +82,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="ouro-2.6b-shape-prefill-32k")
     ap.add_argument("--layers", type=int, default=None, help="override layer count (profiling)")
+    ap.add_argument("--variant", default="flashloop", choices=sorted(VARIANTS),
+                    help="component toggle or loop schedule (see VARIANTS)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
@@ -158,7 +196,8 @@ def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
               for _ in range(L)]
     col_k = {r: cfg["col_k"][r] for r in range(2, R + 1)}
     sched = fl.make_schedule(R, cfg["first_sparse"], n_active, col_k)
-    run = fl.LoopRunner(model, sched, n_active, stores, max(col_k.values()) + 1)
+    kmax = max(col_k.values())
+    run = fl.LoopRunner(model, sched, n_active, stores, kmax + 1 if kmax > 0 else 0)
     h0 = torch.from_numpy(synth.embeddings(g, N, d)).to(dev)
     # the dense loop 1 (the producer of loop 2's statistics): once cold, then timed warm
     # from the same embeddings (it rewrites the same base KV and statistics)
@@ -201,38 +240,53 @@ def gemm_flops_per_step(W):
 
 
 def attention_bytes_per_launch(W, torch):
-    """Algorithmic bytes of one sparse-attention launch (one layer of one loop), from
-    the carried column sets: q (fp32), S, m, u read; o (bf16), S', m', u' written;
-    and the compressed KV of the distinct columns each head reads (base K and V plus
-    the residual rows of every loop up to r in which the column was active)."""
+    """Algorithmic work of one attention launch (one layer of one loop) per loop r:
+    (bytes, algorithmic FLOP, executed tensor FLOP, sparse?).
+
+    Sparse loops, from the carried column sets: q (fp32), S, m, u read; o (bf16) written;
+    the compressed KV of the distinct columns each head reads (base K and V plus the
+    residual rows of every loop up to r in which the column was active); FLOP 4 hd |S|;
+    the query-tile form executes QK^T and PV on 128-column chunks of each tile's union.
+    Dense loops: every active query over its causal prefix, FLOP 4 hd (t + 1), the whole
+    store read once per head."""
     H, hd, N = W["H"], W["hd"], W["N"]
     g = W["stores"][0].g
+    st0 = W["stores"][0]
+    slot = st0.slot.cpu().numpy()
     out = {}
     for r in range(2, W["R"] + 1):
         act = W["run"].act[r][: W["n_active"][r]].long()
         nq = act.numel()
-        k1 = W["col_k"][r] + 1
-        sel = W["run"].sel[0][:, act].cpu().numpy().view(np.uint16)
-        slot = W["stores"][0].slot.cpu().numpy()
-        kv = 0
-        for h in range(H):
-            cols = np.unique(sel[h][sel[h] != 0xFFFF]).astype(np.int64)
-            kv += len(cols) * 2 * (hd + hd // g * 4)   # base codes + (s, z) for K and V
+        base_row = 2 * (hd + hd // g * 4) if st0.base_bits else 2 * hd * 4
+        if W["col_k"][r] > 0:
+            k1 = W["run"].sel[0].shape[2]
+            sel = W["run"].sel[0][:, act].cpu().numpy().view(np.uint16)
+            kv = 0
+            for h in range(H):
+                cols = np.unique(sel[h][sel[h] != 0xFFFF]).astype(np.int64)
+                kv += len(cols) * base_row
+                for rr in range(2, r + 1):
+                    b = W["res"][rr]
+                    nrow = int((slot[rr][cols] >= 0).sum())
+                    kv += nrow * (2 * (hd * b // 8 + hd // g * 4) if b else 2 * hd * 4)
+            fixed = nq * H * hd * 4 + H * nq * k1 * 2 + H * nq * 4 + H * nq * hd * 4 + nq * H * hd * 2
+            flops = 4 * hd * int((sel != 0xFFFF).sum())
+            chunks = 0
+            for h in range(H):
+                for t0 in range(0, nq, 128):
+                    blk = sel[h, t0:t0 + 128]
+                    u = np.unique(blk[blk != 0xFFFF]).size
+                    chunks += -(-u // 128)
+            out[r] = (fixed + kv, flops, chunks * 4 * 128 * 128 * hd, True)
+        else:
+            pos = act.cpu().numpy().astype(np.int64)
+            kv = N * H * base_row
             for rr in range(2, r + 1):
                 b = W["res"][rr]
-                nrow = int((slot[rr][cols] >= 0).sum())
-                kv += nrow * 2 * (hd * b // 8 + hd // g * 4)
-        fixed = nq * H * hd * 4 + 2 * (H * nq * k1 * 2 + H * nq * 4 + H * nq * hd * 4) + nq * H * hd * 2
-        flops = 4 * hd * int((sel != 0xFFFF).sum())
-        # the query-tile form runs QK^T and PV on 128-column chunks of each tile's union
-        chunks = 0
-        for h in range(H):
-            for t0 in range(0, nq, 128):
-                blk = sel[h, t0:t0 + 128]
-                u = np.unique(blk[blk != 0xFFFF]).size
-                chunks += -(-u // 128)
-        executed = chunks * 4 * 128 * 128 * hd
-        out[r] = (fixed + kv, flops, executed)
+                nrow = int((slot[rr] >= 0).sum())
+                kv += nrow * H * (2 * (hd * b // 8 + hd // g * 4) if b else 2 * hd * 4)
+            flops = 4 * hd * H * int((pos + 1).sum())
+            out[r] = (kv + nq * H * hd * 6, flops, flops, False)
     return out
 
 
@@ -385,7 +439,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
-    cfg = configs.CONFIGS[args.config]
+    cfg = apply_variant(configs.CONFIGS[args.config], args.variant)
     W = build_workload(cfg, fl, torch, synth, configs, seed=rank, n_layers=args.layers)
     R, N = W["R"], W["N"]
     stream = torch.cuda.current_stream()
@@ -548,17 +602,26 @@ def main():
                  "traffic": None, "peak_source": f"{pk_kind} bf16 sustained",
                  "share_of_step": gemm_s * 1e3 / step_total_ms, "per_gemm": per_gemm,
                  "timing": timing_note}
-    attn_line = {"bound": "hbm", "kernel": "k_attn_tile (sparse, carried mass, tcgen05)",
-                 "achieved": attn_gbs, "peak": peak_h, "unit": "GB/s",
-                 "frac": attn_gbs / peak_h, "traffic": None,
-                 "peak_source": f"{pk_kind} HBM copy",
-                 "bytes_per_launch": {str(r): abytes[r][0] for r in abytes},
-                 "avg_launch_us": attn_s / len(attn_ms) * 1e6,
-                 "share_of_step": attn_s * 1e3 / step_total_ms,
-                 "algorithmic_tflops": attn_alg_flops / attn_s / 1e12,
-                 "executed_tflops": attn_exec_total / attn_s / 1e12,
-                 "executed_over_algorithmic_flops": attn_exec_total / max(attn_alg_flops, 1),
-                 "timing": timing_note}
+    all_sparse = all(abytes[r][3] for r in abytes)
+    if all_sparse:
+        attn_line = {"bound": "hbm", "kernel": "k_attn_tile (sparse, carried mass, tcgen05)",
+                     "achieved": attn_gbs, "peak": peak_h, "unit": "GB/s",
+                     "frac": attn_gbs / peak_h, "traffic": None,
+                     "peak_source": f"{pk_kind} HBM copy"}
+    else:   # dense attention in some timed loop: tensor-bound on its algorithmic FLOP
+        attn_line = {"bound": "tensor", "kernel": "k_attn_tile / k_attn_dense_tile (tcgen05)",
+                     "achieved": attn_alg_flops / attn_s / 1e12, "peak": peak_t,
+                     "unit": "TFLOP/s", "frac": attn_alg_flops / attn_s / 1e12 / peak_t,
+                     "traffic": None, "peak_source": f"{pk_kind} bf16 sustained (fp16 same rate)",
+                     "hbm_gbs": attn_gbs}
+    attn_line.update({
+        "bytes_per_launch": {str(r): abytes[r][0] for r in abytes},
+        "avg_launch_us": attn_s / len(attn_ms) * 1e6,
+        "share_of_step": attn_s * 1e3 / step_total_ms,
+        "algorithmic_tflops": attn_alg_flops / attn_s / 1e12,
+        "executed_tflops": attn_exec_total / attn_s / 1e12,
+        "executed_over_algorithmic_flops": attn_exec_total / max(attn_alg_flops, 1),
+        "timing": timing_note})
     attn_dominant = attn_s > gemm_s
     loop_ms = step_total_ms / args.steps
     prefill = {"tokens_per_s": N / ((W["loop1_ms"] + loop_ms) / 1e3),
@@ -614,6 +677,7 @@ def main():
                        "loops": R, "timed_loops": list(range(2, R + 1)),
                        "active_tokens": W["n_active"][2], "col_k": cfg["col_k"][2],
                        "res_bits": cfg["res_bits"][2], "group": cfg["group"],
+                       "variant": cfg.get("variant", "flashloop"),
                        "parallelism": f"replicas x{world}",
                        "l2": f"inputs larger than L2 ({weights_gb:.2f} GB of bf16 weights "
                              "read per loop step)"},

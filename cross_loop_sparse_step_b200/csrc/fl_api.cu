@@ -428,6 +428,21 @@ fl_status fl_kv_append(const fl_kv_desc* kv, int32_t loop, const void* k_new, co
                                  S(stream), loop == 1 ? 0 : row0, true));
 }
 
+fl_status fl_kv_reconstruct(const fl_kv_desc* kv, int32_t loop, const int32_t* tok, int32_t n,
+                            float* out_k, float* out_v, void* stream) {
+  fl_status st = check_kv(kv);
+  if (st != FL_OK) return st;
+  FL_CHECK(loop >= 1 && loop <= kv->n_loops && n >= 0, FL_ERR_SHAPE);
+  if (n == 0) return FL_OK;
+  FL_CHECK(tok && out_k && out_v, FL_ERR_INVALID_ARG);
+  for (int r = 1; r <= loop; ++r) {
+    FL_CHECK(kv->codes[0][r] && kv->codes[1][r], FL_ERR_INVALID_ARG);
+    const int b = r == 1 ? kv->base_bits : kv->res_bits[r];
+    if (b != 0) FL_CHECK(kv->sz[0][r] && kv->sz[1][r], FL_ERR_INVALID_ARG);
+  }
+  return cuda_st(launch_kv_reconstruct(*kv, loop, tok, n, out_k, out_v, status_word(), S(stream)));
+}
+
 size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a) {
   return a ? attention_ws_bytes(*a) : 0;
 }

@@ -200,6 +200,8 @@ cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
                             const void* v_new, fl_dtype dt, const int32_t* act_tok, int n_act,
                             int* st, cudaStream_t s, int row0 = 0, bool append = false);
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s);
+cudaError_t launch_kv_reconstruct(const fl_kv_desc& kv, int loop, const int32_t* tok, int n,
+                                  float* out_k, float* out_v, int* st, cudaStream_t s);
 size_t attention_ws_bytes(const fl_attn_args& a);
 
 // Scratch of the tensor-core GEMM's stream-K split: hand-over flags (zero before the first

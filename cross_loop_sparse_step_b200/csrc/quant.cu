@@ -213,4 +213,40 @@ cudaError_t launch_kv_quant(const fl_kv_desc& kv, int loop, const void* k_new,
   return launch_epl<2>(v, o, loop, k_new, v_new, dt, act_tok, n_act, st, s);
 }
 
+// K^_loop and V^_loop of the listed tokens, rebuilt from the store: the base, then the
+// residual row of every loop 2..loop that lists the token, added in loop order (the
+// store's own reconstruction, bit for bit). One thread per 8 elements of a (token, head).
+__global__ void k_kv_reconstruct(const KvView kv, int loop, const int32_t* __restrict__ tok,
+                                 int n, float* __restrict__ out_k, float* __restrict__ out_v,
+                                 int* st) {
+  const int per_row = kv.H * (kv.hd / 8);
+  const long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+  if (i >= (long long)n * per_row) return;
+  const int row = (int)(i / per_row), rem = (int)(i % per_row);
+  const int h = rem / (kv.hd / 8), e0 = (rem % (kv.hd / 8)) * 8;
+  const int t = tok[row];
+  if (t < 0 || t >= kv.n_tok) {
+    record_error(st, FL_ERR_RANGE);
+    return;
+  }
+  const size_t o = ((size_t)row * kv.H + h) * kv.hd + e0;
+  float acc[8];
+  reconstruct<8>(kv, 0, loop, t, h, e0, acc);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out_k[o + k] = acc[k];
+  reconstruct<8>(kv, 1, loop, t, h, e0, acc);
+#pragma unroll
+  for (int k = 0; k < 8; ++k) out_v[o + k] = acc[k];
+}
+
+cudaError_t launch_kv_reconstruct(const fl_kv_desc& kv, int loop, const int32_t* tok, int n,
+                                  float* out_k, float* out_v, int* st, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const long long threads = (long long)n * kv.n_heads * (kv.head_dim / 8);
+  const int blocks = (int)((threads + 255) / 256);
+  k_kv_reconstruct<<<blocks, 256, 0, s>>>(make_view(kv), loop, tok, n, out_k, out_v, st);
+  count_launch();
+  return cudaGetLastError();
+}
+
 }  // namespace fl

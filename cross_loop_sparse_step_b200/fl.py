@@ -108,6 +108,8 @@ _quant = _sig("fl_kv_residual_quant", c_i32,
               [ctypes.POINTER(KvDesc), c_i32, vp, vp, c_i32, vp, c_i32, vp])
 _append = _sig("fl_kv_append", c_i32,
                [ctypes.POINTER(KvDesc), c_i32, vp, vp, c_i32, vp, c_i32, c_i32, vp])
+_recon = _sig("fl_kv_reconstruct", c_i32,
+               [ctypes.POINTER(KvDesc), c_i32, vp, c_i32, vp, vp, vp])
 _attn_b_ws = _sig("fl_sparse_loop_attn_batched_workspace_bytes", c_sz, [c_i32])
 _attn_b = _sig("fl_sparse_loop_attn_batched", c_i32, [ctypes.POINTER(AttnArgs), c_i32, vp, c_sz, vp])
 _attn_ws = _sig("fl_sparse_loop_attn_workspace_bytes", c_sz, [ctypes.POINTER(AttnArgs)])
@@ -258,6 +260,16 @@ def kv_append(store, loop, k_new, v_new, act_tok, row0=0, stream=None):
     """Decode: add the tokens act_tok to loop `loop` (rows row0.. for loop >= 2)."""
     _ok(_append(ctypes.byref(store.desc), loop, ptr(k_new), ptr(v_new), dtype_code(k_new),
                 ptr(act_tok), act_tok.numel(), row0, stream_handle(stream)), "fl_kv_append")
+
+
+def kv_reconstruct(store, loop, tok, stream=None):
+    """K^_loop, V^_loop of the tokens `tok` (int32 device tensor) as float [n, H, hd]."""
+    n = tok.numel()
+    k = torch.empty(n, store.H, store.hd, dtype=torch.float32, device=tok.device)
+    v = torch.empty_like(k)
+    _ok(_recon(ctypes.byref(store.desc), loop, ptr(tok), n, ptr(k), ptr(v),
+               stream_handle(stream)), "fl_kv_reconstruct")
+    return k, v
 
 
 def make_attn_args(q, q_tok, store, loop, out, col_bias=None, sel=None, mass=None, unsel=None,

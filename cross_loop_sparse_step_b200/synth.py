@@ -97,3 +97,14 @@ def query_values(g, n_q, n_heads, head_dim, scale=1.0):
 def sorted_subset(g, n, k):
     """k distinct integers from [0, n), ascending."""
     return np.sort(g.choice(n, size=k, replace=False)).astype(np.int32)
+
+
+def kv_loop_sequence(g, n, H, hd, R, scale=1.0, decay=0.5, delta=0.25):
+    """Per-loop K (or V) of n tokens over R loops: K_1 ~ N(0, scale^2) and
+    K_r = K_{r-1} + D_r with D_r ~ N(0, (scale * delta * decay^(r-2))^2) - a change that
+    shrinks loop after loop (§3.3: cross-loop KV updates are small). float32 arrays."""
+    K = [(g.standard_normal((n, H, hd)) * scale).astype(np.float32)]
+    for r in range(2, R + 1):
+        d = g.standard_normal((n, H, hd)) * scale * delta * decay ** (r - 2)
+        K.append((K[-1] + d).astype(np.float32))
+    return K

@@ -199,6 +199,14 @@ fl_status fl_kv_append(const fl_kv_desc* kv, int32_t loop, const void* k_new, co
                        fl_dtype dt, const int32_t* act_tok, int32_t n_act, int32_t row0,
                        void* stream);
 
+/* The reconstruction K^_loop, V^_loop of the n tokens tok[i] (device int32), as the
+ * attention reads it: the base, then the residual row of every loop 2..loop whose slot
+ * lists the token, added in binary32 in loop order (a raw loop replaces the value).
+ * out_k, out_v: device float [n][H][hd]. For inspection and for the residual-vs-full
+ * quantisation diagnostic (§3.3); a token outside [0, n_tok) records FL_ERR_RANGE. */
+fl_status fl_kv_reconstruct(const fl_kv_desc* kv, int32_t loop, const int32_t* tok, int32_t n,
+                            float* out_k, float* out_v, void* stream);
+
 /* ------------------------------------------------------------------------- *
  * Loop-aware sparse attention (§4.2), and the dense causal attention of a loop
  * whose successor is sparse (the producer of the statistics).

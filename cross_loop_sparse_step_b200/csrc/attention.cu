@@ -378,6 +378,7 @@ size_t attention_ws_bytes(const fl_attn_args& a) {
   return attn_tile_enabled() && dense_tile_eligible(P) ? dense_tile_ws_bytes(P) : 0;
 }
 
+
 AttnParams make_attn_params(const fl_attn_args& a, int* st) {
   AttnParams P;
   P.q = a.q; P.q_bf16 = a.q_dt == FL_BF16;
@@ -402,6 +403,9 @@ cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, 
   // pageable source: the copy is staged before this call returns
   cudaError_t e = cudaMemcpyAsync(ws, host.data(), n * sizeof(AttnParams), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return e;
+  bool tile = attn_tile_enabled();
+  for (int i = 0; tile && i < n; ++i) tile = sparse_tile_eligible(host[i]);
+  if (tile) return launch_attn_tile_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
   int loop_max = 1;   // shared-memory slices sized for the deepest call
   for (int i = 0; i < n; ++i) loop_max = host[i].loop > loop_max ? host[i].loop : loop_max;
   return launch_attn_sparse_batched(host[0], static_cast<const AttnParams*>(ws), n, loop_max, s);

@@ -65,7 +65,8 @@ __device__ __forceinline__ int union_rank(const uint32_t* bits, const uint16_t* 
   return (int)pre[w] + __popc(bits[w] & ((1u << (col & 31)) - 1u));
 }
 
-__global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
+// One CTA: head h, the tile of queries starting at q0 of the call described by P.
+__device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -77,9 +78,6 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = P.H, n_tok = P.kv.n_tok, stride = P.sel_stride;
-  const int n_tiles = (P.n_q + TQ - 1) / TQ;
-  const int h = blockIdx.x / n_tiles;
-  const int q0 = (blockIdx.x % n_tiles) * TQ;
   const int n_words = (n_tok + 31) >> 5;
 
   if (threadIdx.x == 0) {
@@ -469,6 +467,28 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
   if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
+__global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
+  const int n_tiles = (P.n_q + TQ - 1) / TQ;
+  attn_tile_cta(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
+}
+
+// Many calls in one launch (batched decode: one store per sequence): CTA b works on call
+// b / per, per = tiles x heads of a call; the call's arguments are copied from global
+// memory into shared memory first.
+__global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams* __restrict__ Ps,
+                                                                 int per) {
+  __shared__ AttnParams sP;
+  const int call = blockIdx.x / per, b = blockIdx.x % per;
+  {
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(Ps + call);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(&sP);
+    for (int i = threadIdx.x; i < (int)(sizeof(AttnParams) / 4); i += blockDim.x) dst[i] = src[i];
+  }
+  __syncthreads();
+  const int n_tiles = (sP.n_q + TQ - 1) / TQ;
+  attn_tile_cta(sP, b / n_tiles, (b % n_tiles) * TQ);
+}
+
 }  // namespace
 
 bool sparse_tile_eligible(const AttnParams& P) {
@@ -504,6 +524,27 @@ cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s) {
   const cudaError_t e = launch_pdl(k_attn_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, P);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Ps: device array of n AttnParams (copied by the caller), every call tile-eligible with
+// the same n_q and heads.
+cudaError_t launch_attn_tile_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
+                                     cudaStream_t s) {
+  static bool attr_set[128] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (!attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(k_attn_tile_batched,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  const int per = ((P0.n_q + TQ - 1) / TQ) * P0.H;
+  k_attn_tile_batched<<<(unsigned)((long long)per * n), NTHR, SMEM_BYTES, s>>>(Ps_dev, per);
+  count_launch();
+  return cudaGetLastError();
 }
 
 }  // namespace fl

@@ -149,6 +149,8 @@ struct AttnParams {
 
 bool sparse_tile_eligible(const AttnParams& P);
 cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s);
+cudaError_t launch_attn_tile_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
+                                     cudaStream_t s);
 bool sparse_fast_eligible(const AttnParams& P);
 cudaError_t launch_attn_sparse_fast(const AttnParams& P, cudaStream_t s);
 cudaError_t launch_attn_sparse_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,

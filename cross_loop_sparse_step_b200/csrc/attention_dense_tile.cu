@@ -107,7 +107,7 @@ __device__ __forceinline__ void load_q8(const AttnParams& P, int qi, int h, int 
   }
 }
 
-__global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
+__global__ void __maxnreg__(152) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
   const AttnParams& P = A.P;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
   const int total = t_max < 0 ? 0 : nc * n_pass;
   const float scale2 = P.scale * kLog2e;
   const uint32_t idesc = idesc_f16_f32(TQ, TC);
+  const uint32_t idesc_pv = idesc_f16_f32_bmn(TQ, HDT);   // V^ tiles are MN-major
 
   if (warp >= 4 && warp < 8) {
     // ================================================================ softmax warps
@@ -532,8 +533,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
 #pragma unroll
           for (int kk = 0; kk < TC / 16; ++kk) {
             const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_kmajor(v_t + off), idesc,
-                     (c > 0 || kk > 0) ? 1u : 0u);
+            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_mnmajor(v_t + kk * 2048, TC),
+                     idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit(&sh.pv_done);
         }
@@ -563,52 +564,13 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           (col >= 0 && pv_stat) ? log2f(__ldg(P.vnorm + (size_t)col * H + h)) : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
-      uint32_t chain = 0;
-      BaseRow brow[2];
-      const bool need_v = has_pv(pass);
-      if (col >= 0) {
-        load_base(P, 0, col, h, brow[0]);
-        if (need_v) load_base(P, 1, col, h, brow[1]);
+      uint32_t chain = 0;   // loops 2..loop that rewrote the column
+      if (col >= 0)
         for (int r = 2; r <= P.loop; ++r)
           if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
-      }
-#pragma unroll
-      for (int e0 = 0; e0 < HDT; e0 += 16) {   // K^ (pass cand: hi and lo parts)
-        float x[16];
-        if (col >= 0) reconstruct16(P, 0, col, h, brow[0], chain, e0, x);
-        else {
-#pragma unroll
-          for (int k = 0; k < 16; ++k) x[k] = 0.f;
-        }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const float* y = x + 8 * half;
-          *reinterpret_cast<uint4*>(a_tile + sw128_offset(jj, e0 + 8 * half, TC)) =
-              make_uint4(pack_h2(y[0], y[1]), pack_h2(y[2], y[3]), pack_h2(y[4], y[5]), pack_h2(y[6], y[7]));
-          if (pass == PASS_CAND) {
-            float lo[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) lo[k] = y[k] - __half2float(__float2half_rn(y[k]));
-            *reinterpret_cast<uint4*>(b_tile + sw128_offset(jj, e0 + 8 * half, TC)) =
-                make_uint4(pack_h2(lo[0], lo[1]), pack_h2(lo[2], lo[3]), pack_h2(lo[4], lo[5]),
-                           pack_h2(lo[6], lo[7]));
-          }
-        }
-      }
-      if (need_v) {
-#pragma unroll
-        for (int e0 = 0; e0 < HDT; e0 += 16) {   // V^ transposed: row e, column jj
-          float x[16];
-          if (col >= 0) reconstruct16(P, 1, col, h, brow[1], chain, e0, x);
-          else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) x[k] = 0.f;
-          }
-#pragma unroll
-          for (int k = 0; k < 16; ++k)
-            *reinterpret_cast<__half*>(b_tile + sw128_offset(e0 + k, jj, HDT)) = __float2half_rn(x[k]);
-        }
-      }
+      // K^ (pass cand: hi part in A, lo part in B) and, with P V^, V^ in B (MN-major)
+      decode_column(P, 0, col, h, chain, a_tile, pass == PASS_CAND ? b_tile : nullptr, jj);
+      if (has_pv(pass)) decode_column(P, 1, col, h, chain, b_tile, nullptr, jj);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.kv_full[grp]);

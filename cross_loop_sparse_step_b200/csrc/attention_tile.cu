@@ -11,8 +11,9 @@
 //   producer warps (two groups of four, one per pipeline stage) decode the chunk's K^
 //     and V^ rows - int8 base plus the residual chain of every loop that rewrote the
 //     column, fmaf(code, s, z) added in loop order, exactly the store's reconstruction -
-//     and write them as fp16 operand tiles in the 128-byte-swizzle layout: K^ as
-//     [column][element], V^ transposed as [element][column] (both K-major);
+//     and write them as fp16 operand tiles in the 128-byte-swizzle layout, both as
+//     [column][element] rows: K^ is the K-major B operand of Q K^T, V^ the MN-major B
+//     operand of P V^;
 //   the MMA warp issues S = Q K^T into one of two TMEM score buffers, then, once the
 //     softmax has written P, O += P V^ into the TMEM output accumulator
 //     (tcgen05.mma kind::f16, M 128, N 128, fp32 accumulation);
@@ -150,6 +151,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
 
   const float scale2 = P.scale * kLog2e;
   const uint32_t idesc = idesc_f16_f32(TQ, TC);
+  const uint32_t idesc_pv = idesc_f16_f32_bmn(TQ, HDT);   // V^ tiles are MN-major
 
   if (warp >= 4 && warp < 8) {
     // ================================================================ softmax warps
@@ -376,8 +378,8 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
 #pragma unroll
         for (int kk = 0; kk < TC / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-          mma_bf16(d, desc_sw128_kmajor(p_base + off), desc_sw128_kmajor(v_base + off), idesc,
-                   (c > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16(d, desc_sw128_kmajor(p_base + off), desc_sw128_mnmajor(v_base + kk * 2048, TC),
+                   idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&sh.pv_done);
         mma_commit(&sh.kv_empty[st]);
@@ -412,40 +414,13 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
       biasbuf[grp * TC + jj] = (col >= 0 && bias_g) ? __ldg(bias_g + col) * kLog2e : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
-      uint32_t chain = 0;
-      BaseRow brow[2];
-      if (col >= 0) {
-        load_base(P, 0, col, h, brow[0]);
-        load_base(P, 1, col, h, brow[1]);
+      uint32_t chain = 0;   // loops 2..loop that rewrote the column
+      if (col >= 0)
         for (int r = 2; r <= P.loop; ++r)
           if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
-      }
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        uint8_t* tile = which == 0 ? k_tile : v_tile;
-#pragma unroll
-        for (int e0 = 0; e0 < HDT; e0 += 16) {
-          float x[16];
-          if (col >= 0) reconstruct16(P, which, col, h, brow[which], chain, e0, x);
-          else {
-#pragma unroll
-            for (int k = 0; k < 16; ++k) x[k] = 0.f;
-          }
-          if (which == 0) {   // K^ row jj, elements e0..e0+15 (two 16-byte chunks)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const float* y = x + 8 * half;
-              *reinterpret_cast<uint4*>(tile + sw128_offset(jj, e0 + 8 * half, TC)) =
-                  make_uint4(pack_h2(y[0], y[1]), pack_h2(y[2], y[3]), pack_h2(y[4], y[5]),
-                             pack_h2(y[6], y[7]));
-            }
-          } else {            // V^ transposed: row e, column jj
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-              *reinterpret_cast<__half*>(tile + sw128_offset(e0 + k, jj, HDT)) = __float2half_rn(x[k]);
-          }
-        }
-      }
+      // K^ and V^ rows jj of the chunk (V^ is read as an MN-major operand of P V^)
+      decode_column(P, 0, col, h, chain, k_tile, nullptr, jj);
+      decode_column(P, 1, col, h, chain, v_tile, nullptr, jj);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
@@ -467,7 +442,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
-__global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
+__global__ void __maxnreg__(152) k_attn_tile(const __grid_constant__ AttnParams P) {
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
   attn_tile_cta(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
 }
@@ -475,7 +450,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ A
 // Many calls in one launch (batched decode: one store per sequence): CTA b works on call
 // b / per, per = tiles x heads of a call; the call's arguments are copied from global
 // memory into shared memory first.
-__global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams* __restrict__ Ps,
+__global__ void __maxnreg__(152) k_attn_tile_batched(const AttnParams* __restrict__ Ps,
                                                                  int per) {
   __shared__ AttnParams sP;
   const int call = blockIdx.x / per, b = blockIdx.x % per;

@@ -76,11 +76,77 @@ __device__ __forceinline__ void load_base(const AttnParams& P, int which, int co
   for (int k = 0; k < 4; ++k) b.sz[k] = k < ng ? __ldg(sp + k) : 0u;
 }
 
+// The residual rows of one column (K or V) for the loops 2..loop that rewrote the token,
+// in loop order: the code row, its bit width and its (s, z) words, fetched once per chunk
+// (CH rows held in registers; deeper chains walk the remaining loops run by run).
+constexpr int CH = 3;
+struct Chain {
+  int n;                       // rows held (<= CH)
+  uint32_t more;               // loops beyond the held rows (bit r: loop r)
+  const uint8_t* codes[CH];
+  int bits[CH];
+  uint32_t sz[CH][4];
+};
+
+// The rows of the loops in `mask` (bit r set: loop r lists the token) for K or V.
+__device__ __forceinline__ void load_chain(const AttnParams& P, int which, int col, int h,
+                                           uint32_t mask, Chain& c) {
+  const KvView& kv = P.kv;
+  const int ng = HDT / kv.g;
+  c.n = 0;
+  c.more = 0;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    c.codes[k] = nullptr; c.bits[k] = 0;
+    c.sz[k][0] = c.sz[k][1] = c.sz[k][2] = c.sz[k][3] = 0u;
+  }
+  while (mask) {
+    const int r = __ffs(mask) - 1;
+    mask &= mask - 1;
+    if (c.n >= CH) { c.more |= 1u << r; continue; }
+    const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
+    const size_t rh = (size_t)row * P.H + h;
+    const int b = kv.res_bits[r];
+    const uint8_t* cp = kv.codes[which][r] + rh * (b ? HDT * b / 8 : HDT * 4);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (b) {
+      const uint32_t* sp = reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[k] = k < ng ? __ldg(sp + k) : 0u;
+    }
+#pragma unroll
+    for (int k = 0; k < CH; ++k)   // selects keep the arrays in registers
+      if (k == c.n) {
+        c.codes[k] = cp; c.bits[k] = b;
+        c.sz[k][0] = w[0]; c.sz[k][1] = w[1]; c.sz[k][2] = w[2]; c.sz[k][3] = w[3];
+      }
+    ++c.n;
+  }
+}
+
+__device__ __forceinline__ void add_chain_run(int b, const uint8_t* cp, uint32_t szw, int e0,
+                                              float* acc) {
+  if (b == 0) {   // an unquantised loop stores the new value itself
+    const float4* rp = reinterpret_cast<const float4*>(cp) + e0 / 4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = __ldg(rp + k);
+      acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
+    }
+  } else if (b == 2) {
+    add_residual16<2>(cp, szw, e0, acc);
+  } else if (b == 4) {
+    add_residual16<4>(cp, szw, e0, acc);
+  } else {
+    add_residual16<8>(cp, szw, e0, acc);
+  }
+}
+
 // K^ or V^ elements [e0, e0 + 16) of token `col`: the base (already loaded), then the
-// residual rows of the loops in `chain` (bit r set: loop r rewrote the token), added in
-// loop order - the store's reconstruction.
+// held residual rows and any deeper loops, added in loop order - the store's
+// reconstruction.
 __device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, int col, int h,
-                                              const BaseRow& b, uint32_t chain, int e0,
+                                              const BaseRow& b, const Chain& ch, int e0,
                                               float* acc) {
   const KvView& kv = P.kv;
   const int g = kv.g, ng = HDT / g;
@@ -101,29 +167,70 @@ __device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, in
     for (int i = 0; i < 16; ++i)
       acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
   }
-  while (chain) {
-    const int r = __ffs(chain) - 1;
-    chain &= chain - 1;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    if (k < ch.n) {
+      const uint32_t szw = g == 32 ? ch.sz[k][e0 / 32] : ch.sz[k][e0 / 64];
+      add_chain_run(ch.bits[k], ch.codes[k], szw, e0, acc);
+    }
+  }
+  uint32_t more = ch.more;
+  while (more) {   // loops beyond the held rows: slot, scales and codes read run by run
+    const int r = __ffs(more) - 1;
+    more &= more - 1;
     const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
     const size_t rh = (size_t)row * P.H + h;
     const int bits = kv.res_bits[r];
-    if (bits == 0) {   // an unquantised loop stores the new value itself
-      const float4* rp = reinterpret_cast<const float4*>(kv.codes[which][r]) + rh * (HDT / 4) + e0 / 4;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 v = __ldg(rp + k);
-        acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
-      }
-      continue;
-    }
     const uint32_t rsz =
-        __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g);
-    if (bits == 2) add_residual16<2>(kv.codes[which][r] + rh * (HDT / 4), rsz, e0, acc);
-    else if (bits == 4) add_residual16<4>(kv.codes[which][r] + rh * (HDT / 2), rsz, e0, acc);
-    else add_residual16<8>(kv.codes[which][r] + rh * HDT, rsz, e0, acc);
+        bits ? __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g) : 0u;
+    add_chain_run(bits, kv.codes[which][r] + rh * (bits ? HDT * bits / 8 : HDT * 4), rsz, e0, acc);
   }
 }
 
+// Writes the 16 binary32 values x as fp16 into row `row` of a K-major [rows][128]
+// operand tile (two 16-byte chunks at elements e0 .. e0 + 15); with `lo` also the
+// remainders x - fp16(x) as fp16 into the same place of `lo` (split operands).
+__device__ __forceinline__ void store_run(uint8_t* tile, uint8_t* lo, int row, int e0,
+                                          const float* x) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const float* y = x + 8 * half;
+    const uint32_t off = sw128_offset(row, e0 + 8 * half, TC);
+    *reinterpret_cast<uint4*>(tile + off) =
+        make_uint4(pack_h2(y[0], y[1]), pack_h2(y[2], y[3]), pack_h2(y[4], y[5]), pack_h2(y[6], y[7]));
+    if (lo) {
+      float r[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) r[k] = y[k] - __half2float(__float2half_rn(y[k]));
+      *reinterpret_cast<uint4*>(lo + off) =
+          make_uint4(pack_h2(r[0], r[1]), pack_h2(r[2], r[3]), pack_h2(r[4], r[5]), pack_h2(r[6], r[7]));
+    }
+  }
+}
+
+// Decodes K^ or V^ of token `col` (col < 0: zeros) into row `row` of `tile` (and `lo`).
+__device__ __forceinline__ void decode_column(const AttnParams& P, int which, int col, int h,
+                                              uint32_t chain_mask, uint8_t* tile, uint8_t* lo,
+                                              int row) {
+  if (col < 0) {
+    float z[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) z[k] = 0.f;
+#pragma unroll
+    for (int e0 = 0; e0 < HDT; e0 += 16) store_run(tile, lo, row, e0, z);
+    return;
+  }
+  BaseRow br;
+  load_base(P, which, col, h, br);
+  Chain ch;
+  load_chain(P, which, col, h, chain_mask, ch);
+#pragma unroll
+  for (int e0 = 0; e0 < HDT; e0 += 16) {
+    float x[16];
+    reconstruct16(P, which, col, h, br, ch, e0, x);
+    store_run(tile, lo, row, e0, x);
+  }
+}
 
 // Status word value of a bounded wait that ran out: FL_ERR_TIMEOUT in the low byte, the
 // wait's site code above it (fl_check_device_status returns the low byte and keeps the

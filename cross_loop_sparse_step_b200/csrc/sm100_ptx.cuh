@@ -221,11 +221,30 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          | ((uint32_t)(M >> 4) << 24);   // m_dim
 }
 
+// Shared-memory matrix descriptor of an MN-major operand stored as [k][mn] rows of
+// 128-byte-swizzled 64-element atoms (the layout sw128_offset(k, mn, rows) gives): the
+// leading offset steps to the next 64 mn elements (rows x 128 bytes), the stride offset
+// to the next 8 k rows (1024 bytes). A K step of 16 advances the start by 2048 bytes.
+__device__ __forceinline__ uint64_t desc_sw128_mnmajor(uint32_t smem_addr, uint32_t rows) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)(((rows * 128u) >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: fp32 accumulator, fp16 A and B, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                       // c_format F32 (a_format, b_format 0: F16)
          | ((uint32_t)(N >> 3) << 17)    // n_dim
          | ((uint32_t)(M >> 4) << 24);   // m_dim
+}
+
+// The same with B MN-major (transpose-B bit).
+__host__ __device__ constexpr uint32_t idesc_f16_f32_bmn(int M, int N) {
+  return idesc_f16_f32(M, N) | (1u << 16);
 }
 
 }  // namespace sm100

@@ -422,6 +422,151 @@ def run_reference(args):
     return 0
 
 
+# ---------------------------------------------------------------- batched decode
+def run_decode(args, cfg):
+    """One layer of the decode step of a generated token, loops 2..R, for B sequences:
+    the block's q/k/v of the B new rows, each sequence's residual KV row appended,
+    sparse attention of every sequence over its own store in one launch, the output
+    projection and FFN. Timed per layer (CUDA events, graph replay excluded: the appends
+    are per-sequence launches); tokens/s extrapolates to L layers x (R - 1) loops and is
+    labelled as such (the dense loop 1 of a decode step is not part of this number)."""
+    import torch
+    from cross_loop_sparse_step_b200 import fl, synth
+    B, d, H, hd, F = (cfg[k] for k in ("batch", "d_model", "n_heads", "head_dim", "d_ffn"))
+    R, K, g, bits = cfg["n_loops"], cfg["col_k"], cfg["group"], cfg["res_bits"]
+    rs = synth.rng(0)
+    ctx = rs.integers(cfg["ctx_min"], cfg["ctx_max"] + 1, size=B)
+    n_max = int(ctx.max()) + 1
+    stores, bias, stats, rows0, args_keep = [], [], [], {}, []
+    res = {r: bits for r in range(2, R + 1)}
+    for b in range(B):
+        n_ctx = int(ctx[b])
+        n_tok = n_ctx + 1
+        k_act = int(math.ceil(cfg["active_frac"] * n_ctx))
+        act = torch.from_numpy(np.sort(rs.choice(n_ctx, size=k_act, replace=False)).astype(np.int32)).cuda()
+        st = fl.KVStore(n_tok, H, hd, g, cfg["base_bits"], res, R, {r: k_act + 1 for r in range(2, R + 1)})
+        fl.kv_residual_quant(st, 1, torch.randn(n_tok, H, hd, device="cuda"),
+                             torch.randn(n_tok, H, hd, device="cuda"))
+        for r in range(2, R + 1):
+            kr = torch.randn(k_act, H, hd, device="cuda") * 0.5 ** (r - 1)
+            fl.kv_residual_quant(st, r, kr, kr.clone(), act)
+        tok = torch.tensor([n_ctx], dtype=torch.int32, device="cuda")
+        fl.kv_append(st, 1, torch.randn(1, H, hd, device="cuda"), torch.randn(1, H, hd, device="cuda"), tok)
+        stores.append(st)
+        rows0[b] = k_act
+        bcols = synth.biased_columns(rs, n_ctx, cfg["bias_frac"])
+        bb = np.zeros(n_tok, np.float32)
+        bb[bcols] = cfg["bias_value"]
+        bb[0] = cfg["bias_value"]
+        bias.append(torch.from_numpy(bb).cuda())
+        S = np.full((H, 1, K + 1), 0xFFFF, np.uint16)
+        bc = bcols[bcols <= n_ctx][:K]
+        for h in range(H):
+            extra = np.setdiff1d(rs.integers(1, n_ctx + 1, size=2 * K), bc)
+            extra = rs.permutation(extra)[: K - len(bc)]
+            S[h, 0] = np.sort(np.concatenate([[0], bc, extra]))
+        stats.append((torch.from_numpy(S.view(np.int16)).cuda(),
+                      torch.rand(H, 1, device="cuda") * 0.5 + 0.5,
+                      torch.randn(H, 1, hd, device="cuda") * 0.1, tok))
+    torch.cuda.synchronize()
+    w = lambda *sh: (torch.randn(*sh, device="cuda") * 0.02).to(torch.bfloat16)
+    layer = {"w_qkv": w(3 * d, d), "w_o": w(d, d), "w_gate_up": w(2 * F, d), "w_down": w(d, F),
+             "g_attn": torch.ones(d, device="cuda"), "g_ffn": torch.ones(d, device="cuda")}
+    model = fl.LoopModel([layer], n_max, H, hd)
+    x = torch.randn(B, d, device="cuda")
+    pos = torch.from_numpy(ctx.astype(np.int32)).cuda()
+    q, k, v = (torch.empty(B, H, hd, device="cuda") for _ in range(3))
+    attn = torch.empty(B, H, hd, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(model.block_ws_bytes(B), dtype=torch.uint8, device="cuda")
+    q_row = torch.zeros(1, dtype=torch.int32, device="cuda")
+    calls = {}
+    for r in range(2, R + 1):
+        calls[r] = [fl.make_attn_args(q[b:b + 1], stats[b][3], stores[b], r, attn[b:b + 1],
+                                      col_bias=bias[b], sel=stats[b][0], mass=stats[b][1],
+                                      unsel=stats[b][2], q_row=q_row, stat_rows=1)
+                    for b in range(B)]
+    arr = {r: (fl.AttnArgs * B)(*calls[r]) for r in calls}
+    nb = fl._attn_b_ws(B)
+    aws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+    stream = fl.stream_handle()
+
+    def layer_step():
+        for r in range(2, R + 1):
+            fl.block_qkv(model, 0, x, pos, q, k, v, ws)
+            for b in range(B):
+                fl.kv_append(stores[b], r, k[b:b + 1], v[b:b + 1], stats[b][3], row0=rows0[b])
+            rc = fl._attn_b(arr[r], B, fl.ptr(aws), nb, stream)
+            if rc != 0:
+                raise fl.FLError(rc, "fl_sparse_loop_attn_batched")
+            fl.block_out_ffn(model, 0, x, attn, ws)
+
+    for _ in range(args.warmup):
+        layer_step()
+    torch.cuda.synchronize()
+    st = fl.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"decode warm-up reported {fl.status_str(st)}")
+    # attention alone, for its roofline
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record()
+    for _ in range(args.steps):
+        fl._attn_b(arr[R], B, fl.ptr(aws), nb, stream)
+    eb.record()
+    torch.cuda.synchronize()
+    attn_us = ea.elapsed_time(eb) / args.steps * 1e3
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        layer_step()
+    e1.record()
+    torch.cuda.synchronize()
+    st = fl.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"decode steps reported {fl.status_str(st)}")
+    per_layer_ms = e0.elapsed_time(e1) / args.steps      # loops 2..R of one layer
+    L = cfg["n_layers"]
+    step_ms = per_layer_ms * L
+    # algorithmic bytes of one attention launch: per (sequence, head) the carried
+    # columns' base codes and scales for K and V, the residual rows of the columns that
+    # have them, q, S, m, u read and o written
+    kv_b = 0
+    for b in range(B):
+        slot = stores[b].slot.cpu().numpy()
+        S = stats[b][0].cpu().numpy().view(np.uint16)
+        for h in range(H):
+            cols = S[h, 0][S[h, 0] != 0xFFFF].astype(np.int64)
+            kv_b += len(cols) * 2 * (hd + hd // g * 4)
+            for rr in range(2, R + 1):
+                kv_b += int((slot[rr][cols] >= 0).sum()) * 2 * (hd * bits // 8 + hd // g * 4)
+    fixed = B * H * (hd * 4 + (K + 1) * 2 + 4 + hd * 4 + hd * 2)
+    attn_bytes = kv_b + fixed
+    pk, pk_kind = peaks()
+    peak_h = pk.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    weights = 2 * (4 * d * d + 3 * d * F)
+    layer_bytes = (R - 1) * (attn_bytes + weights)
+    line = {
+        "metric": "decode tokens/s (loops 2..R of a generated token, extrapolated to all layers)",
+        "value": B / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "extrapolated": f"measured one layer (x{L} layers); the dense loop 1 of the step excluded",
+        "config": {"workload": cfg["name"], "batch": B, "context": [cfg["ctx_min"], cfg["ctx_max"]],
+                   "heads": f"{H}x{hd}", "col_k": K, "res_bits": bits, "loops": R},
+        "per_layer_us": per_layer_ms * 1e3,
+        "roofline": {"bound": "hbm", "kernel": "decode layer step (batched tile attention, "
+                     "KV append, projection GEMMs of the B rows)",
+                     "achieved": layer_bytes / (per_layer_ms / 1e3) / 1e9, "peak": peak_h,
+                     "unit": "GB/s", "frac": layer_bytes / (per_layer_ms / 1e3) / 1e9 / peak_h,
+                     "traffic": None, "bytes_per_layer": layer_bytes},
+        "attention_roofline": {"bound": "hbm", "kernel": "k_attn_tile_batched",
+                               "achieved": attn_bytes / (attn_us / 1e6) / 1e9, "peak": peak_h,
+                               "unit": "GB/s", "frac": attn_bytes / (attn_us / 1e6) / 1e9 / peak_h,
+                               "avg_launch_us": attn_us, "bytes_per_launch": attn_bytes},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- main
 def main():
     args = parse()
@@ -439,6 +584,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
+    if configs.CONFIGS[args.config].get("decode"):
+        return run_decode(args, configs.CONFIGS[args.config])
     cfg = apply_variant(configs.CONFIGS[args.config], args.variant)
     W = build_workload(cfg, fl, torch, synth, configs, seed=rank, n_layers=args.layers)
     R, N = W["R"], W["N"]

@@ -60,8 +60,19 @@ def c4(n_loops, res_bits):
     )
 
 
+# Batched decode (§5.3.3, Figure 5: decode with sparse attention and 2/4-bit residuals):
+# 64 sequences with 16K..32K cached tokens each; the generated token's loop r >= 2 step
+# per layer (its KV appended, sparse attention over 1024 carried columns plus the sink,
+# the block on the 64 new rows).
+C5 = dict(
+    name="ouro-2.6b-shape-decode-b64",
+    batch=64, ctx_min=16384, ctx_max=32768, d_model=2048, n_heads=16, head_dim=128,
+    d_ffn=5632, n_layers=48, n_loops=4, dtype="bf16", col_k=1024, base_bits=8,
+    res_bits=2, group=32, active_frac=0.15, bias_frac=0.02, bias_value=4.0, decode=True,
+)
+
 CONFIGS = {c["name"]: c for c in (C1, C1_SHRINK, C2, C3, c4(8, 2), c4(8, 4), c4(16, 2),
-                                   c4(16, 4))}
+                                   c4(16, 4), C5)}
 
 
 def active_counts(cfg):

@@ -107,7 +107,7 @@ __device__ __forceinline__ void load_q8(const AttnParams& P, int qi, int h, int 
   }
 }
 
-__global__ void __maxnreg__(152) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
+__global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
   const AttnParams& P = A.P;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(

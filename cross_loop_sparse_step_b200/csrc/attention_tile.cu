@@ -442,7 +442,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
-__global__ void __maxnreg__(152) k_attn_tile(const __grid_constant__ AttnParams P) {
+__global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
   attn_tile_cta(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
 }
@@ -450,7 +450,7 @@ __global__ void __maxnreg__(152) k_attn_tile(const __grid_constant__ AttnParams 
 // Many calls in one launch (batched decode: one store per sequence): CTA b works on call
 // b / per, per = tiles x heads of a call; the call's arguments are copied from global
 // memory into shared memory first.
-__global__ void __maxnreg__(152) k_attn_tile_batched(const AttnParams* __restrict__ Ps,
+__global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams* __restrict__ Ps,
                                                                  int per) {
   __shared__ AttnParams sP;
   const int call = blockIdx.x / per, b = blockIdx.x % per;

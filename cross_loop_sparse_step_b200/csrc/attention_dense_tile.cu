@@ -495,53 +495,71 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const uint32_t qh = smem_u32(smem + OFF_QHI);
       const uint32_t r1 = smem_u32(smem + OFF_R1);
       bool qlo_seen = false;
-      auto issue_qk = [&](int G) -> bool {
-        const int pass = pass_of(mode, G, nc);
-        const int st = G & 1;
-        if (!mbar_wait(&sh.kv_full[st], (G >> 1) & 1, abort, site_of(6 + 16 * mode, G, warp))) return false;
-        if (pass == PASS_CAND && !qlo_seen) {
-          if (!mbar_wait(&sh.qlo_ready, 0, abort, site_of(7 + 16 * mode, G, warp))) return false;
-          qlo_seen = true;
-        }
-        tc_fence_after();
-        const uint32_t a_t = smem_u32(smem + OFF_ST + 2 * st * TILE);
-        const uint32_t b_t = a_t + TILE;
-        const uint32_t d = tmem + (uint32_t)(st * TC);
+      // Issue whichever MMA is ready: QK^T of the next chunk once its operands are decoded
+      // and its score buffer is free (the softmax handed back chunk G - 2), the hand-back of
+      // the oldest chunk (P V^ where the pass has one, then the stage release) once the
+      // softmax is done with it. Neither waits on the other.
+      int qk = 0, pv = 0;
+      uint64_t t0 = globaltimer();
+      while (pv < total) {
+        bool prog = false;
+        if (qk < total && qk <= pv + 1 && mbar_test_wait(&sh.kv_full[qk & 1], (qk >> 1) & 1)) {
+          const int pass = pass_of(mode, qk, nc);
+          if (pass == PASS_CAND && !qlo_seen) qlo_seen = mbar_test_wait(&sh.qlo_ready, 0);
+          if (pass != PASS_CAND || qlo_seen) {
+            tc_fence_after();
+            const int st = qk & 1;
+            const uint32_t a_t = smem_u32(smem + OFF_ST + 2 * st * TILE);
+            const uint32_t b_t = a_t + TILE;
+            const uint32_t d = tmem + (uint32_t)(st * TC);
 #pragma unroll
-        for (int kk = 0; kk < HDT / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-          mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(a_t + off), idesc,
-                   kk > 0 ? 1u : 0u);
-          if (pass == PASS_CAND) {   // q_hi K_lo + q_lo K_hi
-            mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(b_t + off), idesc, 1u);
-            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_kmajor(a_t + off), idesc, 1u);
+            for (int kk = 0; kk < HDT / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+              mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(a_t + off), idesc,
+                       kk > 0 ? 1u : 0u);
+              if (pass == PASS_CAND) {   // q_hi K_lo + q_lo K_hi
+                mma_bf16(d, desc_sw128_kmajor(qh + off), desc_sw128_kmajor(b_t + off), idesc, 1u);
+                mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_kmajor(a_t + off), idesc, 1u);
+              }
+            }
+            mma_commit(&sh.s_full[st]);
+            ++qk;
+            prog = true;
           }
         }
-        mma_commit(&sh.s_full[st]);
-        return true;
-      };
-      bool ok = issue_qk(0);
-      for (int G = 0; ok && G < total; ++G) {
-        if (G + 1 < total && !issue_qk(G + 1)) break;
-        if (!mbar_wait(&sh.p_full[G & 1], (G >> 1) & 1, abort, site_of(8 + 16 * mode, G, warp))) break;
-        tc_fence_after();
-        const int pass = pass_of(mode, G, nc);
-        if (has_pv(pass)) {
-          const int st = G & 1, c = G % nc;
-          const uint32_t v_t = smem_u32(smem + OFF_ST + (2 * st + 1) * TILE);
-          const uint32_t d = tmem + 2u * TC;
+        if (pv < qk && mbar_test_wait(&sh.p_full[pv & 1], (pv >> 1) & 1)) {
+          tc_fence_after();
+          const int pass = pass_of(mode, pv, nc);
+          if (has_pv(pass)) {
+            const int st = pv & 1, c = pv % nc;
+            const uint32_t v_t = smem_u32(smem + OFF_ST + (2 * st + 1) * TILE);
+            const uint32_t d = tmem + 2u * TC;
 #pragma unroll
-          for (int kk = 0; kk < TC / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-            mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_mnmajor(v_t + kk * 2048, TC),
-                     idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < TC / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+              mma_bf16(d, desc_sw128_kmajor(r1 + off), desc_sw128_mnmajor(v_t + kk * 2048, TC),
+                       idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&sh.pv_done);
           }
-          mma_commit(&sh.pv_done);
+          // the stage (operand tiles and its column metadata) is free once the softmax has
+          // handed the chunk back - also in passes without P V^, whose metadata it reads
+          mma_commit(&sh.kv_empty[pv & 1]);
+          sh.prog[4] = pv;
+          ++pv;
+          prog = true;
         }
-        // the stage (operand tiles and its column metadata) is free once the softmax has
-        // handed the chunk back - also in passes without P V^, whose metadata it reads
-        mma_commit(&sh.kv_empty[G & 1]);
-        sh.prog[4] = G;
+        if (prog) {
+          t0 = globaltimer();
+        } else {
+          if (*abort) break;
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            const bool want_qk = qk < total && qk <= pv + 1;
+            atomicCAS(const_cast<int*>(abort), 0,
+                      site_of((want_qk ? 6 : 8) + 16 * mode, want_qk ? qk : pv, warp));
+            break;
+          }
+        }
       }
     }
     if (lane == 0) mma_commit(&sh.fin);
@@ -601,127 +619,113 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
 }
 
 // ---------------------------------------------------------------- kernel B: selection
-constexpr int SEL_THREADS = 256;
+constexpr int SEL_WARPS = 8;
 
 // Exact top-k of c_j = p_j ||V^_j|| (or p_j) among a row's candidates, equal values to
 // the smaller column: S' = {0} U kept (ascending - candidates are stored in column order),
-// m' = p_0 + sum of kept p_j. Rows at positions t <= k keep every column [0, t] (m' = 1).
-// A row whose candidates overflowed is listed for the exact per-query kernel.
-__global__ void __launch_bounds__(SEL_THREADS) k_dense_select(const __grid_constant__ DenseArgs A,
-                                                              int* ovf_n, int* ovf_list) {
+// m' = p_0 + sum of kept p_j. One warp per (row, head): the candidates' keys (binary32
+// bits of c, order-preserving for c >= 0) in shared memory, a radix select 8 bits at a
+// time with a per-warp histogram, then an ordered compaction by ballots. Rows at
+// positions t <= k keep every column [0, t] (m' = 1). A row whose candidates overflowed
+// is listed for the exact per-query kernel.
+__global__ void __launch_bounds__(SEL_WARPS * 32) k_dense_select(const __grid_constant__ DenseArgs A,
+                                                                 int* ovf_n, int* ovf_list) {
   const AttnParams& P = A.P;
   extern __shared__ uint8_t sm[];
-  const int qi = blockIdx.x % P.n_q, h = blockIdx.x / P.n_q;
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t* key = reinterpret_cast<uint32_t*>(sm) + (size_t)w * (A.cap + 256);
+  int* hist = reinterpret_cast<int*>(key + A.cap);
+  const long long rh = (long long)blockIdx.x * SEL_WARPS + w;
+  if (rh >= (long long)P.H * P.n_q) return;   // whole warp leaves; no block barrier below
+  const int qi = (int)(rh % P.n_q), h = (int)(rh / P.n_q);
   const int t = P.q_tok[qi];
   const int srow = P.q_row ? P.q_row[qi] : t;
   if (t < 0 || t >= P.kv.n_tok || srow < 0 || srow >= P.stat_rows) return;   // recorded in A
   uint16_t* so = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
-  const size_t rh = (size_t)h * P.n_q + qi;
   const int k = A.k;
   if (t <= k) {
-    for (int j = threadIdx.x; j < P.out_stride; j += SEL_THREADS)
-      so[j] = j <= t ? (uint16_t)j : (uint16_t)FL_SENTINEL;
-    if (threadIdx.x == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = 1.f;
+    for (int j = lane; j < P.out_stride; j += 32) so[j] = j <= t ? (uint16_t)j : (uint16_t)FL_SENTINEL;
+    if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = 1.f;
     return;
   }
   const int n = A.cnt[rh];
   if (n > A.cap || n < k) {   // overflow (or a count that cannot hold k): exact fallback
-    if (threadIdx.x == 0) {
-      const int slot = atomicAdd(ovf_n, 1);
-      ovf_list[slot] = (int)rh;
-    }
+    if (lane == 0) ovf_list[atomicAdd(ovf_n, 1)] = (int)rh;
     return;
   }
-  uint32_t* key = reinterpret_cast<uint32_t*>(sm);                 // [cap] c as bits
-  uint16_t* col = reinterpret_cast<uint16_t*>(key + A.cap);        // [cap]
-  float* pv = reinterpret_cast<float*>(col + ((A.cap + 1) & ~1));  // [cap]
-  __shared__ int hist[256];
-  __shared__ int s_dig, s_above, s_wsum[SEL_THREADS / 32], s_eqb[SEL_THREADS / 32];
-  __shared__ float s_mass[SEL_THREADS / 32];
   const bool pv_stat = P.stat_kind == FL_STAT_PV;
-  const uint16_t* cc = A.ccol + rh * A.cap;
-  const float* cp = A.cp + rh * A.cap;
-  for (int x = threadIdx.x; x < n; x += SEL_THREADS) {
-    const int cidx = cc[x];
+  const uint16_t* cc = A.ccol + (size_t)rh * A.cap;
+  const float* cp = A.cp + (size_t)rh * A.cap;
+  for (int x = lane; x < n; x += 32) {
     const float p = cp[x];
-    const float cv = pv_stat ? p * P.vnorm[(size_t)cidx * P.H + h] : p;
+    const float cv = pv_stat ? p * P.vnorm[(size_t)cc[x] * P.H + h] : p;
     key[x] = __float_as_uint(fmaxf(cv, 0.f));
-    col[x] = (uint16_t)cidx;
-    pv[x] = p;
   }
-  __syncthreads();
-  // radix select of the k-th largest key, 8 bits at a time
+  __syncwarp();
   uint32_t prefix = 0, pmask = 0;
   int need = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int b = threadIdx.x; b < 256; b += SEL_THREADS) hist[b] = 0;
-    __syncthreads();
-    for (int x = threadIdx.x; x < n; x += SEL_THREADS)
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int x = lane; x < n; x += 32)
       if ((key[x] & pmask) == prefix) atomicAdd(&hist[(key[x] >> shift) & 255u], 1);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0, d = 255;
-      for (; d > 0; --d) {
-        if (above + hist[d] >= need) break;
-        above += hist[d];
-      }
-      s_dig = d;
-      s_above = above;
+    __syncwarp();
+    // the digit holding the need-th largest: suffix sums over the 256 bins, 8 per lane
+    int cnt8[8], mine = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) { cnt8[i] = hist[255 - (lane * 8 + i)]; mine += cnt8[i]; }
+    int incl = mine;   // inclusive scan from the top digit down
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    __syncthreads();
-    prefix |= (uint32_t)s_dig << shift;
+    const int before = incl - mine;
+    int dig = -1, above = 0;
+    if (before < need && incl >= need) {
+      int acc = before;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (dig < 0 && acc + cnt8[i] >= need) { dig = 255 - (lane * 8 + i); above = acc; }
+        acc += cnt8[i];
+      }
+    }
+    const uint32_t who = __ballot_sync(0xffffffffu, dig >= 0);
+    const int src = who ? __ffs(who) - 1 : 0;
+    dig = __shfl_sync(0xffffffffu, dig, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    if (!who) { dig = 0; above = 0; }   // cannot happen with n >= k
+    prefix |= (uint32_t)dig << shift;
     pmask |= 255u << shift;
-    need -= s_above;
-    __syncthreads();
+    need -= above;
+    __syncwarp();
   }
-  // keep key > prefix, and the first `need` entries (smallest columns) with key == prefix;
-  // the candidates are in ascending column order, so a stable compaction keeps S' ascending
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // keep key > prefix, and the first `need` entries (smallest columns) with key == prefix
   const uint32_t lt = (1u << lane) - 1u;
   int written = 0, eq_seen = 0;
   float mass = 0.f;
-  for (int base = 0; base < n; base += SEL_THREADS) {
-    const int x = base + threadIdx.x;
+  for (int base = 0; base < n; base += 32) {
+    const int x = base + lane;
     const bool in = x < n;
     const uint32_t kv = in ? key[x] : 0u;
     const bool eq = in && kv == prefix;
     const uint32_t eb = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_eqb[w] = __popc(eb);
-    __syncthreads();
-    int eq_before = eq_seen + __popc(eb & lt), eq_tot = 0;
-    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) {
-      if (ww < w) eq_before += s_eqb[ww];
-      eq_tot += s_eqb[ww];
-    }
-    const bool keep = in && (kv > prefix || (eq && eq_before < need));
+    const bool keep = in && (kv > prefix || (eq && eq_seen + __popc(eb & lt) < need));
     const uint32_t kb = __ballot_sync(0xffffffffu, keep);
-    if (lane == 0) s_wsum[w] = __popc(kb);
-    __syncthreads();
-    int pos = written + __popc(kb & lt), tot = 0;
-    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) {
-      if (ww < w) pos += s_wsum[ww];
-      tot += s_wsum[ww];
-    }
+    const int pos = written + __popc(kb & lt);
     if (keep && pos < k) {
-      so[1 + pos] = col[x];
-      mass += pv[x];
+      so[1 + pos] = cc[x];
+      mass += cp[x];
     }
-    written += tot;
-    eq_seen += eq_tot;
-    __syncthreads();
+    written += __popc(kb);
+    eq_seen += __popc(eb);
   }
   written = min(written, k);
-  for (int j = 1 + written + threadIdx.x; j < P.out_stride; j += SEL_THREADS) so[j] = (uint16_t)FL_SENTINEL;
-  if (threadIdx.x == 0) so[0] = 0;
+  for (int j = 1 + written + lane; j < P.out_stride; j += 32) so[j] = (uint16_t)FL_SENTINEL;
+  if (lane == 0) so[0] = 0;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mass += __shfl_xor_sync(0xffffffffu, mass, o);
-  if (lane == 0) s_mass[w] = mass;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = A.p0[rh];
-    for (int ww = 0; ww < SEL_THREADS / 32; ++ww) m += s_mass[ww];
-    P.mass_out[(size_t)h * P.stat_rows + srow] = m;
-  }
+  if (lane == 0) P.mass_out[(size_t)h * P.stat_rows + srow] = A.p0[rh] + mass;
 }
 
 }  // namespace
@@ -788,14 +792,15 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   count_launch();
   if (e != cudaSuccess) return e;
   if (!P.sel_out) return cudaGetLastError();
-  const size_t sel_smem = (size_t)A.cap * 10 + 16;
+  const size_t sel_smem = (size_t)SEL_WARPS * (A.cap + 256) * 4;
   static int sel_attr[128] = {0};
   if ((int)sel_smem > sel_attr[dev]) {
     e = cudaFuncSetAttribute(k_dense_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem);
     if (e != cudaSuccess) return e;
     sel_attr[dev] = (int)sel_smem;
   }
-  k_dense_select<<<(unsigned)rows, SEL_THREADS, sel_smem, s>>>(A, ovf_n, ovf_list);
+  k_dense_select<<<(unsigned)((rows + SEL_WARPS - 1) / SEL_WARPS), SEL_WARPS * 32, sel_smem, s>>>(
+      A, ovf_n, ovf_list);
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -352,37 +352,54 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     if (lane == 0 && n_chunks > 0) {
       const uint32_t q_base = smem_u32(smem + OFF_Q);
       const uint32_t p_base = smem_u32(smem + OFF_P);
-      auto issue_qk = [&](int c) -> bool {
-        const int st = c & 1;
-        if (!mbar_wait(&sh.kv_full[st], (c >> 1) & 1, abort, 106)) return false;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + OFF_K0 + 2 * st * TILE);
-        const uint32_t d = tmem + (uint32_t)(st * TC);
+      // Issue whichever MMA is ready: QK^T of the next chunk once its operands are decoded
+      // and its score buffer is free (the softmax handed back chunk c - 2), P V^ of the
+      // oldest chunk once its P is written. Neither waits on the other, so the two producer
+      // groups decode concurrently.
+      int qk = 0, pv = 0;
+      uint64_t t0 = globaltimer();
+      while (pv < n_chunks) {
+        bool prog = false;
+        if (qk < n_chunks && qk <= pv + 1 && mbar_test_wait(&sh.kv_full[qk & 1], (qk >> 1) & 1)) {
+          tc_fence_after();
+          const int st = qk & 1;
+          const uint32_t k_base = smem_u32(smem + OFF_K0 + 2 * st * TILE);
+          const uint32_t d = tmem + (uint32_t)(st * TC);
 #pragma unroll
-        for (int kk = 0; kk < HDT / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-          mma_bf16(d, desc_sw128_kmajor(q_base + off), desc_sw128_kmajor(k_base + off), idesc,
-                   kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HDT / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+            mma_bf16(d, desc_sw128_kmajor(q_base + off), desc_sw128_kmajor(k_base + off), idesc,
+                     kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh.s_full[st]);
+          ++qk;
+          prog = true;
         }
-        mma_commit(&sh.s_full[st]);
-        return true;
-      };
-      bool ok = issue_qk(0);
-      for (int c = 0; ok && c < n_chunks; ++c) {
-        if (c + 1 < n_chunks && !issue_qk(c + 1)) break;
-        if (!mbar_wait(&sh.p_full[c & 1], (c >> 1) & 1, abort, 108)) break;
-        tc_fence_after();
-        const int st = c & 1;
-        const uint32_t v_base = smem_u32(smem + OFF_K0 + (2 * st + 1) * TILE);
-        const uint32_t d = tmem + 2u * TC;
+        if (pv < qk && mbar_test_wait(&sh.p_full[pv & 1], (pv >> 1) & 1)) {
+          tc_fence_after();
+          const int st = pv & 1;
+          const uint32_t v_base = smem_u32(smem + OFF_K0 + (2 * st + 1) * TILE);
+          const uint32_t d = tmem + 2u * TC;
 #pragma unroll
-        for (int kk = 0; kk < TC / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
-          mma_bf16(d, desc_sw128_kmajor(p_base + off), desc_sw128_mnmajor(v_base + kk * 2048, TC),
-                   idesc_pv, (c > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < TC / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (TQ * 128) + (kk & 3) * 32;
+            mma_bf16(d, desc_sw128_kmajor(p_base + off), desc_sw128_mnmajor(v_base + kk * 2048, TC),
+                     idesc_pv, (pv > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.pv_done);
+          mma_commit(&sh.kv_empty[st]);
+          ++pv;
+          prog = true;
         }
-        mma_commit(&sh.pv_done);
-        mma_commit(&sh.kv_empty[st]);
+        if (prog) {
+          t0 = globaltimer();
+        } else {
+          if (*abort) break;
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            atomicCAS(const_cast<int*>(abort), 0, qk < n_chunks && qk <= pv + 1 ? 106 : 108);
+            break;
+          }
+        }
       }
     }
     if (lane == 0) mma_commit(&sh.fin);   // arrives once every MMA issued above is done

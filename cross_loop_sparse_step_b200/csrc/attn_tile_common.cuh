@@ -5,6 +5,8 @@
 #include "fl_internal.cuh"
 #include "sm100_ptx.cuh"
 
+#include <utility>
+
 namespace fl {
 namespace tile {
 
@@ -55,73 +57,70 @@ __device__ __forceinline__ void add_residual16(const uint8_t* row_codes, uint32_
   }
 }
 
-// The base row of K or V (which = 0 / 1) of token `col`, head h: 128 int8 codes and the
-// (s, z) pairs of its groups, loaded together so one round of memory latency covers them.
-struct BaseRow {
-  uint4 raw[8];
-  uint32_t sz[4];
+// The residual rows of one column (K or V) for the loops 2..loop that rewrote the token,
+// in loop order: the code row, its bit width and its (s, z) words, fetched once per chunk.
+// Three rows are held in named registers (no arrays, so nothing goes to local memory);
+// deeper chains walk the remaining loops run by run.
+struct ChainRow {
+  const uint8_t* codes;
+  int bits;
+  uint32_t sz0, sz1, sz2, sz3;
+};
+struct Chain {
+  int n;            // rows held (<= 3)
+  uint32_t more;    // loops beyond the held rows (bit r: loop r)
+  ChainRow r0, r1, r2;
 };
 
-__device__ __forceinline__ void load_base(const AttnParams& P, int which, int col, int h,
-                                          BaseRow& b) {
-  const KvView& kv = P.kv;
-  if (kv.base_bits == 0) return;   // binary32 rows are read run by run
-  const size_t bh = (size_t)col * P.H + h;
-  const uint4* cp = reinterpret_cast<const uint4*>(kv.codes[which][1] + bh * HDT);
-#pragma unroll
-  for (int k = 0; k < 8; ++k) b.raw[k] = __ldg(cp + k);
-  const int ng = HDT / kv.g;
-  const uint32_t* sp = reinterpret_cast<const uint32_t*>(kv.sz[which][1]) + bh * ng;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) b.sz[k] = k < ng ? __ldg(sp + k) : 0u;
+template <int I>
+__device__ __forceinline__ uint32_t sz_word(const ChainRow& r) {
+  if constexpr (I == 0) return r.sz0;
+  else if constexpr (I == 1) return r.sz1;
+  else if constexpr (I == 2) return r.sz2;
+  else return r.sz3;
 }
 
-// The residual rows of one column (K or V) for the loops 2..loop that rewrote the token,
-// in loop order: the code row, its bit width and its (s, z) words, fetched once per chunk
-// (CH rows held in registers; deeper chains walk the remaining loops run by run).
-constexpr int CH = 3;
-struct Chain {
-  int n;                       // rows held (<= CH)
-  uint32_t more;               // loops beyond the held rows (bit r: loop r)
-  const uint8_t* codes[CH];
-  int bits[CH];
-  uint32_t sz[CH][4];
-};
+__device__ __forceinline__ ChainRow chain_row(const AttnParams& P, int which, int r, int col,
+                                              int h) {
+  const KvView& kv = P.kv;
+  const int ng = HDT / kv.g;
+  const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
+  const size_t rh = (size_t)row * P.H + h;
+  ChainRow c;
+  c.bits = kv.res_bits[r];
+  c.codes = kv.codes[which][r] + rh * (c.bits ? HDT * c.bits / 8 : HDT * 4);
+  c.sz0 = c.sz1 = c.sz2 = c.sz3 = 0u;
+  if (c.bits) {
+    const uint32_t* sp = reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng;
+    c.sz0 = __ldg(sp);
+    c.sz1 = __ldg(sp + 1);
+    if (ng == 4) { c.sz2 = __ldg(sp + 2); c.sz3 = __ldg(sp + 3); }
+  }
+  return c;
+}
 
 // The rows of the loops in `mask` (bit r set: loop r lists the token) for K or V.
 __device__ __forceinline__ void load_chain(const AttnParams& P, int which, int col, int h,
                                            uint32_t mask, Chain& c) {
-  const KvView& kv = P.kv;
-  const int ng = HDT / kv.g;
   c.n = 0;
   c.more = 0;
-#pragma unroll
-  for (int k = 0; k < CH; ++k) {
-    c.codes[k] = nullptr; c.bits[k] = 0;
-    c.sz[k][0] = c.sz[k][1] = c.sz[k][2] = c.sz[k][3] = 0u;
-  }
-  while (mask) {
-    const int r = __ffs(mask) - 1;
-    mask &= mask - 1;
-    if (c.n >= CH) { c.more |= 1u << r; continue; }
-    const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
-    const size_t rh = (size_t)row * P.H + h;
-    const int b = kv.res_bits[r];
-    const uint8_t* cp = kv.codes[which][r] + rh * (b ? HDT * b / 8 : HDT * 4);
-    uint32_t w[4] = {0u, 0u, 0u, 0u};
-    if (b) {
-      const uint32_t* sp = reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) w[k] = k < ng ? __ldg(sp + k) : 0u;
-    }
-#pragma unroll
-    for (int k = 0; k < CH; ++k)   // selects keep the arrays in registers
-      if (k == c.n) {
-        c.codes[k] = cp; c.bits[k] = b;
-        c.sz[k][0] = w[0]; c.sz[k][1] = w[1]; c.sz[k][2] = w[2]; c.sz[k][3] = w[3];
-      }
-    ++c.n;
-  }
+  c.r0 = c.r1 = c.r2 = ChainRow{nullptr, 0, 0u, 0u, 0u, 0u};
+  if (!mask) return;
+  int r = __ffs(mask) - 1;
+  mask &= mask - 1;
+  c.r0 = chain_row(P, which, r, col, h);
+  c.n = 1;
+  if (!mask) return;
+  r = __ffs(mask) - 1;
+  mask &= mask - 1;
+  c.r1 = chain_row(P, which, r, col, h);
+  c.n = 2;
+  if (!mask) return;
+  r = __ffs(mask) - 1;
+  mask &= mask - 1;
+  c.r2 = chain_row(P, which, r, col, h);
+  c.n = 3;
+  c.more = mask;
 }
 
 __device__ __forceinline__ void add_chain_run(int b, const uint8_t* cp, uint32_t szw, int e0,
@@ -139,51 +138,6 @@ __device__ __forceinline__ void add_chain_run(int b, const uint8_t* cp, uint32_t
     add_residual16<4>(cp, szw, e0, acc);
   } else {
     add_residual16<8>(cp, szw, e0, acc);
-  }
-}
-
-// K^ or V^ elements [e0, e0 + 16) of token `col`: the base (already loaded), then the
-// held residual rows and any deeper loops, added in loop order - the store's
-// reconstruction.
-__device__ __forceinline__ void reconstruct16(const AttnParams& P, int which, int col, int h,
-                                              const BaseRow& b, const Chain& ch, int e0,
-                                              float* acc) {
-  const KvView& kv = P.kv;
-  const int g = kv.g, ng = HDT / g;
-  if (kv.base_bits == 0) {   // unquantised store: the binary32 values themselves
-    const float4* rp = reinterpret_cast<const float4*>(kv.codes[which][1]) +
-                       ((size_t)col * P.H + h) * (HDT / 4) + e0 / 4;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float4 v = __ldg(rp + k);
-      acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
-    }
-  } else {
-    const uint32_t szw = g == 32 ? b.sz[e0 / 32] : b.sz[e0 / 64];
-    const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
-    const float z = half_bits_to_float((uint16_t)(szw >> 16));
-    const uint32_t w[4] = {b.raw[e0 / 16].x, b.raw[e0 / 16].y, b.raw[e0 / 16].z, b.raw[e0 / 16].w};
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-      acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
-  }
-#pragma unroll
-  for (int k = 0; k < CH; ++k) {
-    if (k < ch.n) {
-      const uint32_t szw = g == 32 ? ch.sz[k][e0 / 32] : ch.sz[k][e0 / 64];
-      add_chain_run(ch.bits[k], ch.codes[k], szw, e0, acc);
-    }
-  }
-  uint32_t more = ch.more;
-  while (more) {   // loops beyond the held rows: slot, scales and codes read run by run
-    const int r = __ffs(more) - 1;
-    more &= more - 1;
-    const int row = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
-    const size_t rh = (size_t)row * P.H + h;
-    const int bits = kv.res_bits[r];
-    const uint32_t rsz =
-        bits ? __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g) : 0u;
-    add_chain_run(bits, kv.codes[which][r] + rh * (bits ? HDT * bits / 8 : HDT * 4), rsz, e0, acc);
   }
 }
 
@@ -208,6 +162,63 @@ __device__ __forceinline__ void store_run(uint8_t* tile, uint8_t* lo, int row, i
   }
 }
 
+// One run of 16 elements [16 RUN, 16 RUN + 16) of a column: the base codes of the run
+// (8-bit, or binary32 when unquantised), the held residual rows, any deeper loops - the
+// store's reconstruction, added in loop order - written as fp16 (and its remainder).
+template <int RUN>
+__device__ __forceinline__ void decode_run16(const AttnParams& P, int which, int col, int h,
+                                             const uint8_t* base_codes, const uint32_t* base_sz,
+                                             const Chain& ch, uint8_t* tile, uint8_t* lo,
+                                             int row) {
+  constexpr int e0 = 16 * RUN;
+  const KvView& kv = P.kv;
+  const int g = kv.g, ng = HDT / g;
+  float acc[16];
+  if (kv.base_bits == 0) {
+    const float4* rp = reinterpret_cast<const float4*>(base_codes) + e0 / 4;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 v = __ldg(rp + k);
+      acc[4 * k] = v.x; acc[4 * k + 1] = v.y; acc[4 * k + 2] = v.z; acc[4 * k + 3] = v.w;
+    }
+  } else {
+    const uint4 w4 = __ldg(reinterpret_cast<const uint4*>(base_codes) + RUN);
+    const uint32_t szw = __ldg(base_sz + e0 / g);
+    const float s = half_bits_to_float((uint16_t)(szw & 0xFFFFu));
+    const float z = half_bits_to_float((uint16_t)(szw >> 16));
+    const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      acc[i] = __fmaf_rn((float)((w[i >> 2] >> ((i & 3) * 8)) & 0xFFu), s, z);
+  }
+  if (ch.n > 0)
+    add_chain_run(ch.r0.bits, ch.r0.codes, g == 32 ? sz_word<e0 / 32>(ch.r0) : sz_word<e0 / 64>(ch.r0), e0, acc);
+  if (ch.n > 1)
+    add_chain_run(ch.r1.bits, ch.r1.codes, g == 32 ? sz_word<e0 / 32>(ch.r1) : sz_word<e0 / 64>(ch.r1), e0, acc);
+  if (ch.n > 2)
+    add_chain_run(ch.r2.bits, ch.r2.codes, g == 32 ? sz_word<e0 / 32>(ch.r2) : sz_word<e0 / 64>(ch.r2), e0, acc);
+  uint32_t more = ch.more;
+  while (more) {   // loops beyond the held rows: slot, scales and codes read run by run
+    const int r = __ffs(more) - 1;
+    more &= more - 1;
+    const int rrow = __ldg(kv.slot + (size_t)r * kv.n_tok + col);
+    const size_t rh = (size_t)rrow * P.H + h;
+    const int bits = kv.res_bits[r];
+    const uint32_t rsz =
+        bits ? __ldg(reinterpret_cast<const uint32_t*>(kv.sz[which][r]) + rh * ng + e0 / g) : 0u;
+    add_chain_run(bits, kv.codes[which][r] + rh * (bits ? HDT * bits / 8 : HDT * 4), rsz, e0, acc);
+  }
+  store_run(tile, lo, row, e0, acc);
+}
+
+template <int... RUNS>
+__device__ __forceinline__ void decode_runs(const AttnParams& P, int which, int col, int h,
+                                            const uint8_t* bc, const uint32_t* bs, const Chain& ch,
+                                            uint8_t* tile, uint8_t* lo, int row,
+                                            std::integer_sequence<int, RUNS...>) {
+  (decode_run16<RUNS>(P, which, col, h, bc, bs, ch, tile, lo, row), ...);
+}
+
 // Decodes K^ or V^ of token `col` (col < 0: zeros) into row `row` of `tile` (and `lo`).
 __device__ __forceinline__ void decode_column(const AttnParams& P, int which, int col, int h,
                                               uint32_t chain_mask, uint8_t* tile, uint8_t* lo,
@@ -220,16 +231,15 @@ __device__ __forceinline__ void decode_column(const AttnParams& P, int which, in
     for (int e0 = 0; e0 < HDT; e0 += 16) store_run(tile, lo, row, e0, z);
     return;
   }
-  BaseRow br;
-  load_base(P, which, col, h, br);
+  const KvView& kv = P.kv;
+  const size_t bh = (size_t)col * P.H + h;
+  const uint8_t* bc = kv.codes[which][1] + bh * (kv.base_bits ? HDT : HDT * 4);
+  const uint32_t* bs = kv.base_bits ? reinterpret_cast<const uint32_t*>(kv.sz[which][1]) + bh * (HDT / kv.g)
+                                    : nullptr;
   Chain ch;
   load_chain(P, which, col, h, chain_mask, ch);
-#pragma unroll
-  for (int e0 = 0; e0 < HDT; e0 += 16) {
-    float x[16];
-    reconstruct16(P, which, col, h, br, ch, e0, x);
-    store_run(tile, lo, row, e0, x);
-  }
+  decode_runs(P, which, col, h, bc, bs, ch, tile, lo, row,
+              std::make_integer_sequence<int, HDT / 16>{});
 }
 
 // Status word value of a bounded wait that ran out: FL_ERR_TIMEOUT in the low byte, the

@@ -197,7 +197,7 @@ def build_workload(cfg, fl, torch, synth, configs, seed, n_layers=None):
     col_k = {r: cfg["col_k"][r] for r in range(2, R + 1)}
     sched = fl.make_schedule(R, cfg["first_sparse"], n_active, col_k)
     kmax = max(col_k.values())
-    run = fl.LoopRunner(model, sched, n_active, stores, kmax + 1 if kmax > 0 else 0)
+    run = fl.LoopRunner(model, sched, n_active, stores, fl.stat_stride(kmax) if kmax > 0 else 0)
     h0 = torch.from_numpy(synth.embeddings(g, N, d)).to(dev)
     # the dense loop 1 (the producer of loop 2's statistics): once cold, then timed warm
     # from the same embeddings (it rewrites the same base KV and statistics)

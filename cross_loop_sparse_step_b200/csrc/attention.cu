@@ -372,15 +372,24 @@ cudaError_t launch_attention_list(const AttnParams& P, const int* list, const in
 
 static bool attn_tile_enabled();
 
+
+// Staging of the store as fp16 rows (kv_stage.cu) pays off where several query tiles of a
+// head would decode the same columns: the dense producer, and sparse calls of more than
+// one tile. A single-tile call (decode) gathers its few columns straight from the store.
+static bool stage_sparse(const AttnParams& P) { return P.n_q > 128; }
+
+// Workspace of a call: the dense producer's candidate buffers, then the staged rows.
 size_t attention_ws_bytes(const fl_attn_args& a) {
-  if (a.sel || !a.kv) return 0;
+  if (!a.kv || !attn_tile_enabled()) return 0;
   const AttnParams P = make_attn_params(a, nullptr);
-  return attn_tile_enabled() && dense_tile_eligible(P) ? dense_tile_ws_bytes(P) : 0;
+  if (a.sel) return sparse_tile_eligible(P) && stage_sparse(P) ? kv_stage_bytes(P.kv, false) : 0;
+  if (!dense_tile_eligible(P)) return 0;
+  return align_up(dense_tile_ws_bytes(P)) + kv_stage_bytes(P.kv, P.sel_out != nullptr);
 }
 
 
 AttnParams make_attn_params(const fl_attn_args& a, int* st) {
-  AttnParams P;
+  AttnParams P{};
   P.q = a.q; P.q_bf16 = a.q_dt == FL_BF16;
   P.q_tok = a.q_tok; P.n_q = a.n_q; P.H = a.kv->n_heads; P.hd = a.kv->head_dim;
   P.scale = 1.0f / sqrtf((float)P.hd);
@@ -424,20 +433,25 @@ static bool attn_tile_enabled() {
 
 cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   if (a.n_q <= 0) return cudaSuccess;
-  AttnParams P;
-  P.q = a.q; P.q_bf16 = a.q_dt == FL_BF16;
-  P.q_tok = a.q_tok; P.n_q = a.n_q; P.H = a.kv->n_heads; P.hd = a.kv->head_dim;
-  P.scale = 1.0f / sqrtf((float)P.hd);
-  P.kv = make_view(*a.kv); P.loop = a.loop; P.bias = a.col_bias;
-  P.sel = a.sel; P.mass = a.mass; P.unsel = a.unsel;
-  P.stat_rows = a.stat_rows; P.sel_stride = a.sel_stride; P.q_row = a.q_row;
-  P.k_next = a.k_next; P.sel_out = a.sel_out; P.mass_out = a.mass_out; P.unsel_out = a.unsel_out;
-  P.out_stride = a.out_stride; P.stat_kind = a.stat_kind; P.vnorm = a.kv->vnorm;
-  P.out = a.out; P.out_bf16 = a.out_dt == FL_BF16; P.st = st;
+  AttnParams P = make_attn_params(a, st);
   const bool sparse = a.sel != nullptr;
-  if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) return launch_attn_tile(P, s);
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) {
+    const size_t sb = kv_stage_bytes(P.kv, false);
+    if (stage_sparse(P) && ws && a.ws_bytes >= sb) {
+      const cudaError_t e = launch_kv_stage(P.kv, P.loop, ws, false, &P.stage, s);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_attn_tile(P, s);
+  }
   if (!sparse && attn_tile_enabled() && dense_tile_eligible(P)) {
-    if (P.sel_out && a.ws_bytes < dense_tile_ws_bytes(P)) return cudaErrorInvalidValue;
+    const size_t db = dense_tile_ws_bytes(P);
+    if (P.sel_out && a.ws_bytes < db) return cudaErrorInvalidValue;
+    const bool lo = P.sel_out != nullptr;
+    if (ws && a.ws_bytes >= align_up(db) + kv_stage_bytes(P.kv, lo)) {
+      const cudaError_t e = launch_kv_stage(P.kv, P.loop, ws + align_up(db), lo, &P.stage, s);
+      if (e != cudaSuccess) return e;
+    }
     return launch_attn_dense_tile(P, a.ws, s);
   }
   if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);

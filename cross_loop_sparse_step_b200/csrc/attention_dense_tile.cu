@@ -107,6 +107,9 @@ __device__ __forceinline__ void load_q8(const AttnParams& P, int qi, int h, int 
   }
 }
 
+// STAGED: operand rows gathered from the staged fp16 rows (P.stage), else decoded from
+// the store by the producers.
+template <bool STAGED>
 __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_constant__ DenseArgs A) {
   const AttnParams& P = A.P;
   extern __shared__ uint8_t smem_raw[];
@@ -551,8 +554,9 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         }
         if (prog) {
           t0 = globaltimer();
-        } else {
+        } else {   // nothing ready: yield the issue slots to the softmax warp of this SMSP
           if (*abort) break;
+          __nanosleep(32);
           if (globaltimer() - t0 > kWaitLimitNs) {
             const bool want_qk = qk < total && qk <= pv + 1;
             atomicCAS(const_cast<int*>(abort), 0,
@@ -582,13 +586,21 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           (col >= 0 && pv_stat) ? log2f(__ldg(P.vnorm + (size_t)col * H + h)) : 0.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
-      uint32_t chain = 0;   // loops 2..loop that rewrote the column
-      if (col >= 0)
-        for (int r = 2; r <= P.loop; ++r)
-          if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
       // K^ (pass cand: hi part in A, lo part in B) and, with P V^, V^ in B (MN-major)
-      decode_column(P, 0, col, h, chain, a_tile, pass == PASS_CAND ? b_tile : nullptr, jj);
-      if (has_pv(pass)) decode_column(P, 1, col, h, chain, b_tile, nullptr, jj);
+      if constexpr (STAGED) {   // gathered from the staged fp16 rows
+        const size_t hoff = (size_t)h * n_tok * HDT;
+        copy_rows_warp(P.stage.khi + hoff, a_tile, col, (warp & 3) * 32, lane);
+        if (pass == PASS_CAND) copy_rows_warp(P.stage.klo + hoff, b_tile, col, (warp & 3) * 32, lane);
+        if (has_pv(pass)) copy_rows_warp(P.stage.vhi + hoff, b_tile, col, (warp & 3) * 32, lane);
+        cp_async_wait_all();
+      } else {             // decoded from the store
+        uint32_t chain = 0;   // loops 2..loop that rewrote the column
+        if (col >= 0)
+          for (int r = 2; r <= P.loop; ++r)
+            if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
+        decode_column(P, 0, col, h, chain, a_tile, pass == PASS_CAND ? b_tile : nullptr, jj);
+        if (has_pv(pass)) decode_column(P, 1, col, h, chain, b_tile, nullptr, jj);
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
@@ -760,10 +772,11 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_attn_dense_tile,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    for (auto k : {k_attn_dense_tile<true>, k_attn_dense_tile<false>}) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev] = true;
   }
   DenseArgs A{};
@@ -788,7 +801,8 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   }
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
   A.mode = P.sel_out ? 1 : 0;
-  cudaError_t e = launch_pdl(k_attn_dense_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
+  auto kern = P.stage.khi ? k_attn_dense_tile<true> : k_attn_dense_tile<false>;
+  cudaError_t e = launch_pdl(kern, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
   count_launch();
   if (e != cudaSuccess) return e;
   if (!P.sel_out) return cudaGetLastError();
@@ -805,7 +819,7 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   A.mode = 2;
-  e = launch_pdl(k_attn_dense_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
+  e = launch_pdl(kern, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
   count_launch();
   if (e != cudaSuccess) return e;
   // rows whose candidates overflowed: the warp-per-query kernel (loop 1, 8-bit base) or

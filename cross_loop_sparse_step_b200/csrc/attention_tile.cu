@@ -50,7 +50,8 @@ constexpr uint32_t OFF_P = OFF_K0 + 4 * TILE;
 constexpr uint32_t OFF_BITS = OFF_P + TILE;
 constexpr uint32_t OFF_PRE = OFF_BITS + MAX_WORDS * 4;
 constexpr uint32_t OFF_BIAS = OFF_PRE + MAX_WORDS * 2;   // [2][TC] float (log2 units)
-constexpr uint32_t SMEM_BYTES = OFF_BIAS + 2 * TC * 4 + 1024;
+constexpr uint32_t OFF_MASK = OFF_BIAS + 2 * TC * 4;     // [2][TQ] uint4: membership of a chunk
+constexpr uint32_t SMEM_BYTES = OFF_MASK + 2 * TQ * 16 + 1024;
 
 struct TileShared {
   uint64_t kv_full[2], kv_empty[2], meta_full[2], s_full[2], p_full[2], pv_done, fin;
@@ -66,7 +67,87 @@ __device__ __forceinline__ int union_rank(const uint32_t* bits, const uint16_t* 
   return (int)pre[w] + __popc(bits[w] & ((1u << (col & 31)) - 1u));
 }
 
+// A query's carried set walked in column order (= union-rank order), 16 entries buffered
+// and the next 16 requested ahead. Rows whose stride is a multiple of 8 are 16-byte
+// aligned and read 8 entries per load; other strides entry by entry.
+struct SetWalk {
+  const uint16_t* row;
+  int stride, vi, p;
+  bool vec, ended;
+  uint4 c0, c1, n0, n1;   // current 16 entries (two per word), the next 16
+};
+
+// entries 8 i .. 8 i + 7 of the row, sentinels beyond it
+__device__ __forceinline__ uint4 set_vec(const SetWalk& w, int i) {
+  constexpr uint32_t S2 = 0xFFFFFFFFu;   // two sentinels
+  if (8 * i >= w.stride) return make_uint4(S2, S2, S2, S2);
+  if (w.vec) return __ldg(reinterpret_cast<const uint4*>(w.row) + i);
+  uint32_t e[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int j = 8 * i + k;
+    e[k] = j < w.stride ? (uint32_t)__ldg(w.row + j) : (uint32_t)FL_SENTINEL;
+  }
+  return make_uint4(e[0] | e[1] << 16, e[2] | e[3] << 16, e[4] | e[5] << 16, e[6] | e[7] << 16);
+}
+
+__device__ __forceinline__ void set_init(SetWalk& w, const uint16_t* row, int stride, bool valid) {
+  w.row = row;
+  w.stride = valid ? stride : 0;
+  w.vec = (stride & 7) == 0 && (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  w.ended = !valid;
+  w.c0 = set_vec(w, 0); w.c1 = set_vec(w, 1); w.n0 = set_vec(w, 2); w.n1 = set_vec(w, 3);
+  w.vi = 4;
+  w.p = 0;
+}
+
+__device__ __forceinline__ int set_entry(const SetWalk& w) {
+  const uint4 v = w.p < 8 ? w.c0 : w.c1;
+  const int q = (w.p >> 1) & 3;
+  const uint32_t x = q == 0 ? v.x : (q == 1 ? v.y : (q == 2 ? v.z : v.w));
+  return (int)((x >> ((w.p & 1) * 16)) & 0xFFFFu);
+}
+
+__device__ __forceinline__ void set_advance(SetWalk& w) {
+  if (++w.p == 16) {
+    w.c0 = w.n0; w.c1 = w.n1;
+    w.n0 = set_vec(w, w.vi); w.n1 = set_vec(w, w.vi + 1);
+    w.vi += 2;
+    w.p = 0;
+  }
+}
+
+// The membership mask of the chunk of union ranks [lo, lo + TC) for a query at position
+// t: its entries in the chunk, walked on from where the previous call stopped. Entries
+// that are not columns of the query (beyond t or the store) are recorded and skipped.
+__device__ __forceinline__ uint4 walk_chunk(SetWalk& w, int t, int n_tok, int lo,
+                                            const uint32_t* bits, const uint16_t* pre, int* st) {
+  uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+  while (!w.ended) {
+    const int c = set_entry(w);
+    if (c == (int)FL_SENTINEL) { w.ended = true; break; }
+    if (c >= n_tok || c > t) {
+      record_error(st, FL_ERR_RANGE);
+      set_advance(w);
+      continue;
+    }
+    const int r = union_rank(bits, pre, c) - lo;
+    if (r >= TC) break;   // a later chunk's entry
+    if (r >= 0) {
+      const uint32_t bit = 1u << (r & 31);
+      const int wd = r >> 5;
+      m0 |= wd == 0 ? bit : 0u; m1 |= wd == 1 ? bit : 0u;
+      m2 |= wd == 2 ? bit : 0u; m3 |= wd == 3 ? bit : 0u;
+    }
+    set_advance(w);
+  }
+  return make_uint4(m0, m1, m2, m3);
+}
+
 // One CTA: head h, the tile of queries starting at q0 of the call described by P.
+// STAGED: K^ / V^ rows are gathered from the staged fp16 rows (P.stage), else decoded
+// from the store by the producers.
+template <bool STAGED>
 __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -101,6 +182,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   tc_fence_after();
   const uint32_t tmem = sh.tmem;
 
+  const bool vec_rows = (stride & 7) == 0 && (reinterpret_cast<uintptr_t>(P.sel) & 15) == 0;
   // ---- the union of the tile's column sets (entries that are not valid columns of the
   // query - beyond its position or the store - are recorded and skipped here and below)
   for (int i = warp; i < TQ; i += NWARPS) {
@@ -110,12 +192,42 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     const int srow = P.q_row ? P.q_row[qi] : t;
     if (t < 0 || t >= n_tok || srow < 0 || srow >= P.stat_rows) continue;
     const uint16_t* row = P.sel + ((size_t)h * P.stat_rows + srow) * stride;
-    for (int e0 = 0; e0 < stride; e0 += 32) {
-      const int e = e0 + lane;
-      const int c = e < stride ? (int)row[e] : (int)FL_SENTINEL;
-      const bool ok = c != (int)FL_SENTINEL && c < n_tok && c <= t;
-      if (ok) atomicOr(&bits[c >> 5], 1u << (c & 31));
-      if (__all_sync(0xffffffffu, c == (int)FL_SENTINEL)) break;   // padding reached
+    if (vec_rows) {   // 16-byte rows: 4 loads of 8 entries in flight per lane
+      const uint4* rv = reinterpret_cast<const uint4*>(row);
+      const int nv = stride >> 3;
+      for (int v0 = 0; v0 < nv; v0 += 128) {
+        uint4 w4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int vi = v0 + 32 * k + lane;
+          w4[k] = vi < nv ? __ldg(rv + vi) : make_uint4(~0u, ~0u, ~0u, ~0u);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t ws[4] = {w4[k].x, w4[k].y, w4[k].z, w4[k].w};
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int c = (int)((ws[m >> 1] >> ((m & 1) * 16)) & 0xFFFFu);
+            if (c != (int)FL_SENTINEL && c < n_tok && c <= t) atomicOr(&bits[c >> 5], 1u << (c & 31));
+          }
+        }
+        if (__all_sync(0xffffffffu, (w4[3].w >> 16) == FL_SENTINEL)) break;   // padding reached
+      }
+      continue;
+    }
+    for (int e0 = 0; e0 < stride; e0 += 256) {   // 8 loads in flight per lane
+      int c8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e = e0 + 32 * k + lane;
+        c8[k] = e < stride ? (int)__ldg(row + e) : (int)FL_SENTINEL;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = c8[k];
+        if (c != (int)FL_SENTINEL && c < n_tok && c <= t) atomicOr(&bits[c >> 5], 1u << (c & 31));
+      }
+      if (__all_sync(0xffffffffu, c8[7] == (int)FL_SENTINEL)) break;   // padding reached
     }
   }
   __syncthreads();
@@ -171,99 +283,73 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     // the query row as fp16 into Q (zeros for rows without a query)
     {
       uint8_t* qt = smem + OFF_Q;
-      for (int e0 = 0; e0 < HDT; e0 += 8) {
-        float x[8];
+      // 32 elements per step, their loads issued together (read-only path)
+#pragma unroll 1
+      for (int e0 = 0; e0 < HDT; e0 += 32) {
+        float x[32];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) x[k] = 0.f;
+        for (int k = 0; k < 32; ++k) x[k] = 0.f;
         if (valid) {
           const size_t off = ((size_t)qi * H + h) * HDT + e0;
           if (P.q_bf16) {
-            const uint4 v = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off);
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+            const uint4* qp = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(P.q) + off);
+            uint4 w[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) { x[2 * k] = __low2float(b2[k]); x[2 * k + 1] = __high2float(b2[k]); }
+            for (int k = 0; k < 4; ++k) w[k] = __ldg(qp + k);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&w[k]);
+#pragma unroll
+              for (int m = 0; m < 4; ++m) { x[8 * k + 2 * m] = __low2float(b2[m]); x[8 * k + 2 * m + 1] = __high2float(b2[m]); }
+            }
           } else {
-            const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
-            const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off + 4);
-            x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+            const float4* qp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(P.q) + off);
+            float4 w[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) w[k] = __ldg(qp + k);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) { x[4 * k] = w[k].x; x[4 * k + 1] = w[k].y; x[4 * k + 2] = w[k].z; x[4 * k + 3] = w[k].w; }
           }
         }
-        *reinterpret_cast<uint4*>(qt + sw128_offset(i, e0, TQ)) =
-            make_uint4(pack_h2(x[0], x[1]), pack_h2(x[2], x[3]), pack_h2(x[4], x[5]), pack_h2(x[6], x[7]));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<uint4*>(qt + sw128_offset(i, e0 + 8 * k, TQ)) =
+              make_uint4(pack_h2(x[8 * k], x[8 * k + 1]), pack_h2(x[8 * k + 2], x[8 * k + 3]),
+                         pack_h2(x[8 * k + 4], x[8 * k + 5]), pack_h2(x[8 * k + 6], x[8 * k + 7]));
       }
       fence_proxy_async_smem();
     }
     // named barrier: Q written by the 4 softmax warps before the MMA warp issues QK
     asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");
 
-    const uint16_t* srow_p = valid ? P.sel + ((size_t)h * P.stat_rows + srow) * stride : nullptr;
-    // The set is walked 8 entries at a time in step with the chunks: gr[] holds the union
-    // ranks of the current group (-1: entry skipped), the next group's loads are issued one
-    // group ahead so their latency overlaps a chunk.
-    int ent = 0;
-    bool ended = !valid;       // a sentinel or the end of the row was reached
-    uint32_t nx[8];
-    int gr[8], gmax = -1;
-    auto load_next = [&]() {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        nx[k] = (!ended && ent + k < stride) ? (uint32_t)srow_p[ent + k] : (uint32_t)FL_SENTINEL;
-      ent += 8;
-    };
-    auto take_next = [&]() {   // ranks of the loaded group; load the one after
-      gmax = -1;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int c = (int)nx[k];
-        gr[k] = -1;
-        if (ended || c == (int)FL_SENTINEL) { ended = true; continue; }
-        if (c >= n_tok || c > t) { record_error(P.st, FL_ERR_RANGE); continue; }
-        gr[k] = union_rank(bits, pre, c);
-        gmax = gr[k];
-      }
-      if (ent >= stride) ended = true;
-      load_next();
-    };
-#pragma unroll
-    for (int k = 0; k < 8; ++k) gr[k] = -1;
-    load_next();
-    if (valid) take_next();
     float m_used = -INFINITY, lsum = 0.f;
     const float m_in = valid ? P.mass[(size_t)h * P.stat_rows + srow] : 0.f;
     uint8_t* pt = smem + OFF_P;
+    const uint4* maskbuf = reinterpret_cast<const uint4*>(smem + OFF_MASK);
     for (int c = 0; c < n_chunks; ++c) {   // leaves only through warp-uniform waits
-      uint32_t mask[4] = {0u, 0u, 0u, 0u};
-      const int lo = c * TC, hi = lo + TC;
-      while (true) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int pos = gr[k] - lo;
-          const uint32_t bit = (pos >= 0 && pos < TC) ? 1u << (pos & 31) : 0u;
-          const int w = pos >> 5;   // selects, so the mask stays in registers
-          mask[0] |= w == 0 ? bit : 0u;
-          mask[1] |= w == 1 ? bit : 0u;
-          mask[2] |= w == 2 ? bit : 0u;
-          mask[3] |= w == 3 ? bit : 0u;
-        }
-        if (gmax < hi && !ended) take_next();
-        else break;
-      }
-      __syncwarp();   // reconverge before the warp-collective TMEM accesses
       const int sb = c & 1;
       // waits agree across the warp: the TMEM loads below are warp-collective
       if (!warp_wait(&sh.s_full[sb], (c >> 1) & 1, abort, 101)) break;
       if (!warp_wait(&sh.meta_full[sb], (c >> 1) & 1, abort, 102)) break;
       tc_fence_after();
+      const uint4 mk = maskbuf[sb * TQ + i];   // this row's members among the chunk's columns
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = biasbuf + sb * TC;
+      // columns in groups of 16 (16 TMEM words per load keeps the row in registers)
+      auto mask16 = [&](int g) -> uint32_t {
+        const uint32_t w = g < 2 ? mk.x : (g < 4 ? mk.y : (g < 6 ? mk.z : mk.w));
+        return (w >> ((g & 1) * 16)) & 0xFFFFu;
+      };
       float cmax = -INFINITY;
+#pragma unroll 1
+      for (int g = 0; g < 8; ++g) {
+        const uint32_t mw = mask16(g);
+        if (!__any_sync(0xffffffffu, mw)) continue;   // no member in the warp's rows
+        float v[16];
+        tmem_ld16(s_addr + g * 16, v);
 #pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
-        float v[32];
-        tmem_ld32(s_addr + g4 * 32, v);
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (mask[g4] & (1u << j)) cmax = fmaxf(cmax, fmaf(v[j], scale2, bias[g4 * 32 + j]));
+        for (int j = 0; j < 16; ++j)
+          cmax = fmaxf(cmax, (mw >> j) & 1u ? fmaf(v[j], scale2, bias[g * 16 + j]) : -INFINITY);
       }
       float alpha = 1.f;
       bool rescale = false;
@@ -287,24 +373,26 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
           tmem_st32(o_addr + g4 * 32, v);
         }
       }
+#pragma unroll 1
+      for (int g = 0; g < 8; ++g) {
+        const uint32_t mw = mask16(g);
+        uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (__any_sync(0xffffffffu, mw)) {
+          float v[16];
+          tmem_ld16(s_addr + g * 16, v);
 #pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {
-        float v[32];
-        tmem_ld32(s_addr + g4 * 32, v);
-        uint32_t pk[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float a = 0.f, b = 0.f;
-          if (mask[g4] & (1u << j)) a = exp2f(fmaf(v[j], scale2, bias[g4 * 32 + j]) - m_used);
-          if (mask[g4] & (1u << (j + 1))) b = exp2f(fmaf(v[j + 1], scale2, bias[g4 * 32 + j + 1]) - m_used);
-          const __half2 hv = __floats2half2_rn(a, b);
-          const float2 back = __half22float2(hv);
-          lsum += back.x + back.y;
-          pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int j = 0; j < 16; j += 2) {
+            const float ea = exp2f(fmaf(v[j], scale2, bias[g * 16 + j]) - m_used);
+            const float eb = exp2f(fmaf(v[j + 1], scale2, bias[g * 16 + j + 1]) - m_used);
+            const __half2 hv = __floats2half2_rn((mw >> j) & 1u ? ea : 0.f, (mw >> (j + 1)) & 1u ? eb : 0.f);
+            const float2 back = __half22float2(hv);
+            lsum += back.x + back.y;
+            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
         }
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          *reinterpret_cast<uint4*>(pt + sw128_offset(i, g4 * 32 + q * 8, TQ)) =
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(pt + sw128_offset(i, g * 16 + q * 8, TQ)) =
               make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
       }
       fence_proxy_async_smem();
@@ -393,8 +481,9 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
         }
         if (prog) {
           t0 = globaltimer();
-        } else {
+        } else {   // nothing ready: yield the issue slots to the softmax warp of this SMSP
           if (*abort) break;
+          __nanosleep(32);
           if (globaltimer() - t0 > kWaitLimitNs) {
             atomicCAS(const_cast<int*>(abort), 0, qk < n_chunks && qk <= pv + 1 ? 106 : 108);
             break;
@@ -410,6 +499,17 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     const float* bias_g = P.bias;
     uint8_t* k_tile = smem + OFF_K0 + 2 * grp * TILE;
     uint8_t* v_tile = k_tile + TILE;
+    uint4* maskbuf = reinterpret_cast<uint4*>(smem + OFF_MASK) + grp * TQ;
+    // this lane also walks the set of query jj of the tile, for the membership masks
+    const int qi = q0 + jj;
+    int t = -1, srow = 0;
+    if (qi < P.n_q) {
+      t = P.q_tok[qi];
+      srow = P.q_row ? P.q_row[qi] : t;
+      if (t < 0 || t >= n_tok || srow < 0 || srow >= P.stat_rows) t = -1;   // recorded by the softmax
+    }
+    SetWalk walk;
+    set_init(walk, t >= 0 ? P.sel + ((size_t)h * P.stat_rows + srow) * stride : P.sel, stride, t >= 0);
     for (int c = grp; c < n_chunks; c += 2) {
       if (__any_sync(0xffffffffu, *abort != 0)) break;   // warp-uniform exit
       if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort, 109)) break;
@@ -428,16 +528,27 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
         col = m ? lo * 32 + __ffs(m) - 1 : -1;
         if (col < 0 || col >= n_tok) { record_error(P.st, FL_ERR_RANGE); col = -1; }
       }
+      // K^ and V^ rows jj of the chunk (V^ is read as an MN-major operand of P V^):
+      // gathered from the staged fp16 rows (the copies fly while the masks are walked) ...
+      if constexpr (STAGED) {
+        const size_t hoff = (size_t)h * n_tok * HDT;
+        copy_rows_warp(P.stage.khi + hoff, k_tile, col, (warp & 3) * 32, lane);
+        copy_rows_warp(P.stage.vhi + hoff, v_tile, col, (warp & 3) * 32, lane);
+      }
       biasbuf[grp * TC + jj] = (col >= 0 && bias_g) ? __ldg(bias_g + col) * kLog2e : 0.f;
+      maskbuf[jj] = walk_chunk(walk, t, n_tok, c * TC, bits, pre, P.st);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
-      uint32_t chain = 0;   // loops 2..loop that rewrote the column
-      if (col >= 0)
-        for (int r = 2; r <= P.loop; ++r)
-          if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
-      // K^ and V^ rows jj of the chunk (V^ is read as an MN-major operand of P V^)
-      decode_column(P, 0, col, h, chain, k_tile, nullptr, jj);
-      decode_column(P, 1, col, h, chain, v_tile, nullptr, jj);
+      if constexpr (STAGED) {
+        cp_async_wait_all();
+      } else {             // ... or decoded from the store
+        uint32_t chain = 0;   // loops 2..loop that rewrote the column
+        if (col >= 0)
+          for (int r = 2; r <= P.loop; ++r)
+            if (__ldg(P.kv.slot + (size_t)r * n_tok + col) >= 0) chain |= 1u << r;
+        decode_column(P, 0, col, h, chain, k_tile, nullptr, jj);
+        decode_column(P, 1, col, h, chain, v_tile, nullptr, jj);
+      }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
@@ -459,9 +570,10 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
+template <bool STAGED>
 __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
-  attn_tile_cta(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
+  attn_tile_cta<STAGED>(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
 }
 
 // Many calls in one launch (batched decode: one store per sequence): CTA b works on call
@@ -478,7 +590,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams*
   }
   __syncthreads();
   const int n_tiles = (sP.n_q + TQ - 1) / TQ;
-  attn_tile_cta(sP, b / n_tiles, (b % n_tiles) * TQ);
+  attn_tile_cta<false>(sP, b / n_tiles, (b % n_tiles) * TQ);
 }
 
 }  // namespace
@@ -507,13 +619,16 @@ cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    const cudaError_t e = cudaFuncSetAttribute(k_attn_tile, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    for (auto k : {k_attn_tile<true>, k_attn_tile<false>}) {
+      const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+    }
     attr_set[dev] = true;
   }
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
-  const cudaError_t e = launch_pdl(k_attn_tile, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, P);
+  const cudaError_t e = launch_pdl(P.stage.khi ? k_attn_tile<true> : k_attn_tile<false>,
+                                   dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, P);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

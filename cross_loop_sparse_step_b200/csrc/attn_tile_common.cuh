@@ -242,6 +242,25 @@ __device__ __forceinline__ void decode_column(const AttnParams& P, int which, in
               std::make_integer_sequence<int, HDT / 16>{});
 }
 
+// Rows wrow0 .. wrow0 + 31 of a K-major operand tile from staged fp16 rows, by one warp:
+// lane l names the column of row wrow0 + l (col < 0: zeros); each row (256 bytes) is
+// copied by 16 lanes, 16 bytes each, two rows per step, as asynchronous copies into the
+// swizzled places. src points at the head's [n_tok][HDT] rows. The caller waits for its
+// copies and fences them for the tensor cores before handing the tile over.
+__device__ __forceinline__ void copy_rows_warp(const __half* src, uint8_t* tile, int col,
+                                               int wrow0, int lane) {
+  const int half = lane >> 4, piece = lane & 15;
+  const uint32_t t = smem_u32(tile);
+#pragma unroll 4
+  for (int s = 0; s < 16; ++s) {
+    const int rr = 2 * s + half;
+    const int c = __shfl_sync(0xffffffffu, col, rr);
+    const uint32_t off = sw128_offset(wrow0 + rr, 8 * piece, TC);
+    if (c >= 0) cp_async16(t + off, src + (size_t)c * HDT + 8 * piece);
+    else *reinterpret_cast<uint4*>(tile + off) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
 // Status word value of a bounded wait that ran out: FL_ERR_TIMEOUT in the low byte, the
 // wait's site code above it (fl_check_device_status returns the low byte and keeps the
 // site for fl_last_error_detail).

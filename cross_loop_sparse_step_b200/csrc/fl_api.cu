@@ -540,18 +540,21 @@ fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n
 }
 
 // ---------------------------------------------------------------- loop step
-// Workspace of the dense attention calls of a schedule that hand statistics to a sparse
-// successor: every token queries, with the largest such budget (an upper bound).
+// Workspace of the attention calls of a schedule (an upper bound over its loops): the
+// store staged as fp16 rows (K^ hi and V^; K^ lo too where a dense call hands statistics
+// to a sparse successor) and, for such a call, the dense producer's candidate buffers
+// with every token querying at the largest such budget.
 static size_t loop_attn_ws(const fl_model* m, const fl_schedule* s) {
-  if (!s) return 0;
+  if (!s || m->head_dim != 128) return 0;
+  const size_t rows = (size_t)m->n_heads * m->n_tok * m->head_dim * sizeof(uint16_t);
   int kmax = 0;
   for (int r = 1; r < s->n_loops && r < FL_MAX_LOOPS; ++r)
     if ((r == 1 || s->col_k[r] == 0) && s->col_k[r + 1] > kmax) kmax = s->col_k[r + 1];
-  if (kmax == 0) return 0;
+  if (kmax == 0) return 2 * rows;
   AttnParams P{};
   P.H = m->n_heads; P.hd = m->head_dim; P.n_q = m->n_tok; P.k_next = kmax;
   P.sel_out = reinterpret_cast<uint16_t*>(1);
-  return dense_tile_ws_bytes(P);
+  return align_up(dense_tile_ws_bytes(P), 256) + 3 * rows;
 }
 
 static size_t loop_ws_layout(const fl_model* m, const fl_schedule* sc, Carver* c, int32_t** iota,

@@ -128,6 +128,17 @@ __device__ __forceinline__ void reconstruct(const KvView& kv, int which, int upt
 }
 
 // Arguments of the attention kernels (a by-value copy of fl_attn_args plus the store view).
+// fp16 operand rows of a whole store at one loop, [H][n_tok][hd] each (kv_stage.cu);
+// klo (K^ - fp16(K^) as fp16) only where a split-operand pass needs it.
+struct KvStage {
+  __half* khi;
+  __half* klo;
+  __half* vhi;
+};
+size_t kv_stage_bytes(const KvView& kv, bool with_lo);
+cudaError_t launch_kv_stage(const KvView& kv, int loop, void* buf, bool with_lo, KvStage* out,
+                            cudaStream_t s);
+
 struct AttnParams {
   const void* q; int q_bf16;
   const int32_t* q_tok;
@@ -145,6 +156,7 @@ struct AttnParams {
   const float* vnorm;
   void* out; int out_bf16;
   int* st;
+  KvStage stage;   // khi == NULL: the kernels decode the store themselves
 };
 
 bool sparse_tile_eligible(const AttnParams& P);

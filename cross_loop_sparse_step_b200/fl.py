@@ -366,6 +366,13 @@ def make_schedule(n_loops, first_sparse, n_active, col_k, stat_kind=STAT_PV):
     return s
 
 
+def stat_stride(k):
+    """Statistics row stride for a budget of k columns plus the sink: k + 1 rounded up to
+    a multiple of 8, so every row of the uint16 column sets starts on a 16-byte boundary
+    (the attention kernels then read the sets 8 entries per load)."""
+    return (k + 1 + 7) // 8 * 8
+
+
 class LoopRunner:
     """Device state of an R-loop run (fl_loop_state) plus the model and schedule."""
 

@@ -48,7 +48,7 @@ def carried_sets(cfg, act, g):
     query, random others before it (the shape of loop 1's statistics)."""
     N, H, k = cfg["n_tok"], cfg["n_heads"], cfg["col_k"][2]
     bias_cols = synth.biased_columns(g, N, cfg["bias_frac"])
-    S = np.full((H, len(act), k + 1), 0xFFFF, np.uint16)
+    S = np.full((H, len(act), fl.stat_stride(k)), 0xFFFF, np.uint16)
     for i, t in enumerate(act):
         t = int(t)
         if t <= k:
@@ -63,7 +63,7 @@ def carried_sets(cfg, act, g):
             else:
                 pool = np.setdiff1d(np.arange(1, t + 1), bc)
                 extra = g.choice(pool, need, replace=False)
-            S[h, i] = np.sort(np.concatenate([[0], bc, extra]))
+            S[h, i, : k + 1] = np.sort(np.concatenate([[0], bc, extra]))
     return S
 
 
@@ -103,7 +103,7 @@ def main():
         q = torch.randn(N, H, hd, device="cuda")
         tok = torch.arange(N, dtype=torch.int32, device="cuda")
         out = torch.empty(N, H, hd, dtype=torch.bfloat16, device="cuda")
-        S = torch.empty(H, N, k + 1, dtype=torch.int16, device="cuda")
+        S = torch.empty(H, N, fl.stat_stride(k), dtype=torch.int16, device="cuda")
         m = torch.empty(H, N, device="cuda")
         u = torch.empty(H, N, hd, device="cuda")
         calls.append(lambda: fl.sparse_loop_attn(q, tok, st, 1, out, col_bias=bias, k_next=k,

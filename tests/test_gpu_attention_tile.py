@@ -30,11 +30,17 @@ CASES = [
      {r: max(410, int(4096 * 0.8 ** (r - 2))) for r in range(2, 17)}, 512, True, 32, True),
     ("32k-shape", 32768, 16, 32, 2, {2: 2}, {2: 4916}, 2048, True, 24, True),
 ]
+# the same with the statistics stride padded to a multiple of 8 (16-byte rows: the sets
+# are read 8 entries per load, the layout the loop step allocates)
+PADDED = {"bf16-256", "4k-shape", "32k-shape", "ragged-37"}
+CASES = [c + (False,) for c in CASES] + [(c[0] + "-stride8",) + c[1:] + (True,) for c in CASES
+                                         if c[0] in PADDED]
 
 
-@pytest.mark.parametrize("name,n,H,g,R,bits,counts,k,use_bias,sample,bf16", CASES,
+@pytest.mark.parametrize("name,n,H,g,R,bits,counts,k,use_bias,sample,bf16,pad", CASES,
                          ids=[c[0] for c in CASES])
-def test_tile_attention_matches_oracle(name, n, H, g, R, bits, counts, k, use_bias, sample, bf16):
+def test_tile_attention_matches_oracle(name, n, H, g, R, bits, counts, k, use_bias, sample, bf16,
+                                       pad):
     from cross_loop_sparse_step_b200 import fl
     hd = 128
     rs = synth.rng(7000 + n + R + k)
@@ -54,6 +60,10 @@ def test_tile_attention_matches_oracle(name, n, H, g, R, bits, counts, k, use_bi
     # random sets for the checked queries (and for a few early tokens whose set is their
     # whole prefix), evenly spaced sets for the others
     S, m, u = _stats(rs, n, H, hd, k, act, bias_cols, act[pick])
+    if pad:
+        Sp = np.full(S.shape[:2] + (fl.stat_stride(k),), 0xFFFF, S.dtype)
+        Sp[..., : S.shape[2]] = S
+        S = Sp
     q = synth.query_values(rs, len(act), H, hd)
     tdt = torch.bfloat16 if bf16 else torch.float32
     if bf16:

@@ -382,7 +382,10 @@ static bool stage_sparse(const AttnParams& P) { return P.n_q > 128; }
 size_t attention_ws_bytes(const fl_attn_args& a) {
   if (!a.kv || !attn_tile_enabled()) return 0;
   const AttnParams P = make_attn_params(a, nullptr);
-  if (a.sel) return sparse_tile_eligible(P) && stage_sparse(P) ? kv_stage_bytes(P.kv, false) : 0;
+  if (a.sel) {
+    if (!sparse_tile_eligible(P) || !stage_sparse(P)) return 0;
+    return align_up(kv_stage_bytes(P.kv, false)) + sel_bitmap_bytes(P);
+  }
   if (!dense_tile_eligible(P)) return 0;
   return align_up(dense_tile_ws_bytes(P)) + kv_stage_bytes(P.kv, P.sel_out != nullptr);
 }
@@ -437,10 +440,16 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   const bool sparse = a.sel != nullptr;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
   if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) {
-    const size_t sb = kv_stage_bytes(P.kv, false);
+    const size_t sb = align_up(kv_stage_bytes(P.kv, false));
     if (stage_sparse(P) && ws && a.ws_bytes >= sb) {
-      const cudaError_t e = launch_kv_stage(P.kv, P.loop, ws, false, &P.stage, s);
+      cudaError_t e = launch_kv_stage(P.kv, P.loop, ws, false, &P.stage, s);
       if (e != cudaSuccess) return e;
+      if (a.ws_bytes >= sb + sel_bitmap_bytes(P)) {
+        e = launch_sel_bitmap(P, ws + sb, s);
+        if (e != cudaSuccess) return e;
+      } else {
+        P.stage.khi = nullptr;   // staged rows without set bitmaps: decode in the tiles
+      }
     }
     return launch_attn_tile(P, s);
   }

@@ -67,6 +67,51 @@ __device__ __forceinline__ int union_rank(const uint32_t* bits, const uint16_t* 
   return (int)pre[w] + __popc(bits[w] & ((1u << (col & 31)) - 1u));
 }
 
+// Column of union rank R (R < n_union): the last bitmap word whose prefix <= R, then the
+// bit within it; -1 for R >= U.
+__device__ __forceinline__ int rank_column(const uint32_t* bits, const uint16_t* pre, int n_words,
+                                           int U, int R) {
+  if (R >= U) return -1;
+  int lo = 0, hi = n_words - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int)pre[mid] <= R) lo = mid;
+    else hi = mid - 1;
+  }
+  uint32_t m = bits[lo];
+  for (int k = R - (int)pre[lo]; k > 0 && m; --k) m &= m - 1u;
+  return m ? lo * 32 + __ffs(m) - 1 : -1;
+}
+
+// The membership mask of union ranks [r0, r0 + TC) for a query whose set is the bitmap
+// qbm: the union's words over the chunk's column span [c0, c1], each AND-ed with the
+// query's word; every hit lands at its rank within the chunk (the union bits below it).
+// The word loop has the same trip count on every lane.
+__device__ __forceinline__ uint4 bitmap_chunk_mask(const uint32_t* bits, const uint32_t* qbm,
+                                                   int c0, int c1) {
+  uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
+  const int wa = c0 >> 5, wb = c1 >> 5;
+  int base = 0;
+#pragma unroll 4
+  for (int w = wa; w <= wb; ++w) {
+    uint32_t ub = bits[w];
+    if (w == wa) ub &= ~((1u << (c0 & 31)) - 1u);
+    if (w == wb && (c1 & 31) != 31) ub &= (2u << (c1 & 31)) - 1u;
+    uint32_t hit = qbm ? (ub & __ldg(qbm + w)) : 0u;
+    while (hit) {
+      const int b = __ffs(hit) - 1;
+      hit &= hit - 1u;
+      const int pos = base + __popc(ub & ((1u << b) - 1u));
+      const uint32_t bit = 1u << (pos & 31);
+      const int wd = pos >> 5;
+      m0 |= wd == 0 ? bit : 0u; m1 |= wd == 1 ? bit : 0u;
+      m2 |= wd == 2 ? bit : 0u; m3 |= wd == 3 ? bit : 0u;
+    }
+    base += __popc(ub);
+  }
+  return make_uint4(m0, m1, m2, m3);
+}
+
 // A query's carried set walked in column order (= union-rank order), 16 entries buffered
 // and the next 16 requested ahead. Rows whose stride is a multiple of 8 are 16-byte
 // aligned and read 8 entries per load; other strides entry by entry.
@@ -145,10 +190,15 @@ __device__ __forceinline__ uint4 walk_chunk(SetWalk& w, int t, int n_tok, int lo
 }
 
 // One CTA: head h, the tile of queries starting at q0 of the call described by P.
-// STAGED: K^ / V^ rows are gathered from the staged fp16 rows (P.stage), else decoded
-// from the store by the producers.
-template <bool STAGED>
+// MODE: DECODE - chunks of the tile's union, K^ / V^ decoded from the store by the
+// producers; UNION - chunks of the union, rows gathered from the staged fp16 rows;
+// CONTIG - chunks of the plain column range [0, t_max] of the tile (for tiles whose union
+// is nearly every column anyway: no union, no ranks), staged rows, and each query's
+// membership read from the bitmap of its set (P.sel_bm).
+enum TileMode : int { DECODE = 0, UNION = 1, CONTIG = 2 };
+template <int MODE>
 __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0) {
+  constexpr bool STAGED = MODE != DECODE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -172,9 +222,11 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.fin, 1);
     sh.abort_flag = 0;
+    sh.n_union = -1;
     fence_barrier_init();
   }
-  for (int w = threadIdx.x; w < n_words; w += NTHR) bits[w] = 0u;
+  if (MODE != CONTIG)
+    for (int w = threadIdx.x; w < n_words; w += NTHR) bits[w] = 0u;
   if (warp == 12) tmem_alloc(&sh.tmem, 512);
   griddep_wait();
   tc_fence_before();
@@ -182,6 +234,15 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   tc_fence_after();
   const uint32_t tmem = sh.tmem;
 
+  if constexpr (MODE == CONTIG) {   // the tile's column range: [0, largest position]
+    if (threadIdx.x < TQ && q0 + (int)threadIdx.x < P.n_q) {
+      const int t = P.q_tok[q0 + threadIdx.x];
+      if (t >= 0 && t < n_tok) atomicMax(&sh.n_union, t);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) sh.n_union += 1;
+    __syncthreads();
+  } else {
   const bool vec_rows = (stride & 7) == 0 && (reinterpret_cast<uintptr_t>(P.sel) & 15) == 0;
   // ---- the union of the tile's column sets (entries that are not valid columns of the
   // query - beyond its position or the store - are recorded and skipped here and below)
@@ -258,6 +319,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     }
   }
   __syncthreads();
+  }
   const int U = sh.n_union;
   const int n_chunks = (U + TC - 1) / TC;
 
@@ -326,13 +388,24 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     const float m_in = valid ? P.mass[(size_t)h * P.stat_rows + srow] : 0.f;
     uint8_t* pt = smem + OFF_P;
     const uint4* maskbuf = reinterpret_cast<const uint4*>(smem + OFF_MASK);
+    // CONTIG: this row's membership words, chunk by chunk, one chunk read ahead
+    const uint4* bmrow = MODE == CONTIG && valid
+        ? reinterpret_cast<const uint4*>(P.sel_bm + ((size_t)h * P.n_q + qi) * P.bm_words) : nullptr;
+    uint4 mk_next = make_uint4(0u, 0u, 0u, 0u);
+    if (MODE == CONTIG && bmrow && n_chunks > 0) mk_next = __ldg(bmrow);
     for (int c = 0; c < n_chunks; ++c) {   // leaves only through warp-uniform waits
       const int sb = c & 1;
       // waits agree across the warp: the TMEM loads below are warp-collective
       if (!warp_wait(&sh.s_full[sb], (c >> 1) & 1, abort, 101)) break;
       if (!warp_wait(&sh.meta_full[sb], (c >> 1) & 1, abort, 102)) break;
       tc_fence_after();
-      const uint4 mk = maskbuf[sb * TQ + i];   // this row's members among the chunk's columns
+      uint4 mk;   // this row's members among the chunk's columns
+      if constexpr (MODE == CONTIG) {
+        mk = mk_next;
+        if (bmrow && c + 1 < n_chunks) mk_next = __ldg(bmrow + c + 1);
+      } else {
+        mk = maskbuf[sb * TQ + i];
+      }
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = biasbuf + sb * TC;
       // columns in groups of 16 (16 TMEM words per load keeps the row in registers)
@@ -340,60 +413,97 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
         const uint32_t w = g < 2 ? mk.x : (g < 4 ? mk.y : (g < 6 ? mk.z : mk.w));
         return (w >> ((g & 1) * 16)) & 0xFFFFu;
       };
-      float cmax = -INFINITY;
-#pragma unroll 1
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t mw = mask16(g);
-        if (!__any_sync(0xffffffffu, mw)) continue;   // no member in the warp's rows
-        float v[16];
-        tmem_ld16(s_addr + g * 16, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          cmax = fmaxf(cmax, (mw >> j) & 1u ? fmaf(v[j], scale2, bias[g * 16 + j]) : -INFINITY);
-      }
-      float alpha = 1.f;
-      bool rescale = false;
-      if (cmax > m_used + kRescale) {
-        if (m_used != -INFINITY && lsum > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
-        m_used = cmax;
-      }
       // P of the previous chunk must have been consumed (and O completed) before P is
       // rewritten or O rescaled
       if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, 103)) break;
       tc_fence_after();
-      if (rescale) lsum *= alpha;
-      if (__any_sync(0xffffffffu, rescale)) {   // warp-collective; alpha = 1 elsewhere
-        const uint32_t o_addr = tmem + lane_base + 2u * TC;
-#pragma unroll 1
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(o_addr + g4 * 32, v);
+      // P = 2^(s - m_used) as fp16 into the P tile, the row sum over the fp16 values;
+      // with `detect`, whether a member column lies more than 2^8 above m_used. The 16-word
+      // loads of the next group fly while a group is processed.
+      const float lsum0 = lsum;
+      auto p_pass = [&](bool detect) -> bool {
+        const float2 sc2 = make_float2(scale2, scale2);
+        const float2 negm = make_float2(-m_used, -m_used);
+        float2 acc = make_float2(0.f, 0.f);          // the row sum, two partial sums
+        __half2 hmax = __float2half2_rn(0.f);         // largest P written (overflow check)
+        auto group = [&](int g, const uint32_t (&r)[16]) {
+          const uint32_t mw = mask16(g);
+          uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          if (__any_sync(0xffffffffu, mw)) {
+            const float2* b2 = reinterpret_cast<const float2*>(bias + g * 16);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] *= alpha;
-          tmem_st32(o_addr + g4 * 32, v);
-        }
-      }
+            for (int j = 0; j < 16; j += 2) {
+              // x = s * scale2 + bias, P = 2^(x - m_used) for a pair of columns; members
+              // kept by a 16-bit lane mask (all ones or zero per column)
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                          sc2, b2[j / 2]);
+              const float2 d = __fadd2_rn(x, negm);
+              const __half2 hv = __floats2half2_rn(exp2f(d.x), exp2f(d.y));
+              const uint32_t ma = (uint32_t)((int)(mw << (31 - j)) >> 31);
+              const uint32_t mb = (uint32_t)((int)(mw << (30 - j)) >> 31);
+              const uint32_t pm = __byte_perm(ma, mb, 0x5410);
+              const uint32_t pv = *reinterpret_cast<const uint32_t*>(&hv) & pm;
+              const __half2 ph = *reinterpret_cast<const __half2*>(&pv);
+              if (detect) hmax = __hmax2(hmax, ph);
+              acc = __fadd2_rn(acc, __half22float2(ph));
+              pk[j / 2] = pv;
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            *reinterpret_cast<uint4*>(pt + sw128_offset(i, g * 16 + q * 8, TQ)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        };
+        uint32_t ra[16], rb[16];
+        tmem_ld16_issue(s_addr, ra);
 #pragma unroll 1
-      for (int g = 0; g < 8; ++g) {
-        const uint32_t mw = mask16(g);
-        uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-        if (__any_sync(0xffffffffu, mw)) {
+        for (int g = 0; g < 8; g += 2) {
+          tmem_ld16_wait(ra);
+          tmem_ld16_issue(s_addr + (g + 1) * 16, rb);
+          group(g, ra);
+          tmem_ld16_wait(rb);
+          if (g + 2 < 8) tmem_ld16_issue(s_addr + (g + 2) * 16, ra);
+          group(g + 1, rb);
+        }
+        lsum += acc.x + acc.y;
+        // a member more than 2^8 above m_used: P above 256 (or infinite, m_used = -inf)
+        const float2 hm = __half22float2(hmax);
+        return detect && fmaxf(hm.x, hm.y) > 256.f;
+      };
+      // One pass against the running maximum. A row with a member more than 2^8 above it
+      // (a P above 256 after fp16 rounding) takes the maximum of the chunk first (O and the
+      // sum rescaled) and writes P again; the common case needs no maximum pass.
+      if (__any_sync(0xffffffffu, p_pass(true))) {
+        float cmax = -INFINITY;
+#pragma unroll 1
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t mw = mask16(g);
+          if (!__any_sync(0xffffffffu, mw)) continue;   // no member in the warp's rows
           float v[16];
           tmem_ld16(s_addr + g * 16, v);
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const float ea = exp2f(fmaf(v[j], scale2, bias[g * 16 + j]) - m_used);
-            const float eb = exp2f(fmaf(v[j + 1], scale2, bias[g * 16 + j + 1]) - m_used);
-            const __half2 hv = __floats2half2_rn((mw >> j) & 1u ? ea : 0.f, (mw >> (j + 1)) & 1u ? eb : 0.f);
-            const float2 back = __half22float2(hv);
-            lsum += back.x + back.y;
-            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          for (int j = 0; j < 16; ++j)
+            cmax = fmaxf(cmax, (mw >> j) & 1u ? fmaf(v[j], scale2, bias[g * 16 + j]) : -INFINITY);
+        }
+        float alpha = 1.f;
+        bool rescale = false;
+        if (cmax > m_used + kRescale) {
+          if (m_used != -INFINITY && lsum0 > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
+          m_used = cmax;
+        }
+        lsum = rescale ? lsum0 * alpha : lsum0;
+        if (__any_sync(0xffffffffu, rescale)) {   // warp-collective; alpha = 1 elsewhere
+          const uint32_t o_addr = tmem + lane_base + 2u * TC;
+#pragma unroll 1
+          for (int g4 = 0; g4 < 4; ++g4) {
+            float v[32];
+            tmem_ld32(o_addr + g4 * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= alpha;
+            tmem_st32(o_addr + g4 * 32, v);
           }
         }
-#pragma unroll
-        for (int q = 0; q < 2; ++q)
-          *reinterpret_cast<uint4*>(pt + sw128_offset(i, g * 16 + q * 8, TQ)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        p_pass(false);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -492,6 +602,51 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
       }
     }
     if (lane == 0) mma_commit(&sh.fin);   // arrives once every MMA issued above is done
+  } else if constexpr (STAGED) {
+    // ========================================== producers (rows from the staged store)
+    // two groups of four warps, one per stage (chunk parity): the chunk's columns, their
+    // K^ / V^ rows as asynchronous copies (16 lanes per row), the column biases, and in
+    // UNION mode the membership masks of the tile's queries (lane jj walks the set of
+    // query jj while the copies fly)
+    const int grp = warp < 4 ? 0 : 1;
+    const int jj = (warp & 3) * 32 + lane;
+    uint8_t* k_tile = smem + OFF_K0 + 2 * grp * TILE;
+    uint8_t* v_tile = k_tile + TILE;
+    uint4* maskbuf = reinterpret_cast<uint4*>(smem + OFF_MASK) + grp * TQ;
+    const size_t hoff = (size_t)h * n_tok * HDT;
+    // UNION: query jj's bitmap row (invalid queries have none: recorded by the softmax)
+    const uint32_t* qbm = nullptr;
+    if constexpr (MODE == UNION) {
+      const int qi = q0 + jj;
+      if (qi < P.n_q) {
+        const int t = P.q_tok[qi];
+        const int srow = P.q_row ? P.q_row[qi] : t;
+        if (t >= 0 && t < n_tok && srow >= 0 && srow < P.stat_rows)
+          qbm = P.sel_bm + ((size_t)h * P.n_q + qi) * P.bm_words;
+      }
+    }
+    for (int c = grp; c < n_chunks; c += 2) {
+      if (__any_sync(0xffffffffu, *abort != 0)) break;   // warp-uniform exit
+      if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort, 109)) break;
+      const int col = MODE == CONTIG ? (c * TC + jj < U ? c * TC + jj : -1)
+                                     : rank_column(bits, pre, n_words, U, c * TC + jj);
+      copy_rows_warp(P.stage.khi + hoff, k_tile, col, (warp & 3) * 32, lane);
+      copy_rows_warp(P.stage.vhi + hoff, v_tile, col, (warp & 3) * 32, lane);
+      biasbuf[grp * TC + jj] = (col >= 0 && P.bias) ? __ldg(P.bias + col) * kLog2e : 0.f;
+      if constexpr (MODE == UNION) {
+        // the chunk's first and last columns (the same on every lane)
+        const int c0 = rank_column(bits, pre, n_words, U, c * TC);
+        const int c1 = rank_column(bits, pre, n_words, U, min(U, c * TC + TC) - 1);
+        maskbuf[jj] = bitmap_chunk_mask(bits, qbm, c0, c1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
+      cp_async_wait_all();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.kv_full[grp]);
+    }
+    cp_async_wait_all();   // nothing in flight when the CTA retires
   } else {
     // ================================================================ producer warps
     const int grp = warp < 4 ? 0 : 1;          // stage = chunk parity
@@ -513,35 +668,13 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     for (int c = grp; c < n_chunks; c += 2) {
       if (__any_sync(0xffffffffu, *abort != 0)) break;   // warp-uniform exit
       if (c >= 2 && !warp_wait(&sh.kv_empty[grp], ((c >> 1) - 1) & 1, abort, 109)) break;
-      // column of rank c * TC + jj: the last word whose prefix <= rank, then the bit
       const int R = c * TC + jj;
-      int col = -1;
-      if (R < U) {
-        int lo = 0, hi = n_words - 1;
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if ((int)pre[mid] <= R) lo = mid;
-          else hi = mid - 1;
-        }
-        uint32_t m = bits[lo];
-        for (int k = R - (int)pre[lo]; k > 0 && m; --k) m &= m - 1u;
-        col = m ? lo * 32 + __ffs(m) - 1 : -1;
-        if (col < 0 || col >= n_tok) { record_error(P.st, FL_ERR_RANGE); col = -1; }
-      }
-      // K^ and V^ rows jj of the chunk (V^ is read as an MN-major operand of P V^):
-      // gathered from the staged fp16 rows (the copies fly while the masks are walked) ...
-      if constexpr (STAGED) {
-        const size_t hoff = (size_t)h * n_tok * HDT;
-        copy_rows_warp(P.stage.khi + hoff, k_tile, col, (warp & 3) * 32, lane);
-        copy_rows_warp(P.stage.vhi + hoff, v_tile, col, (warp & 3) * 32, lane);
-      }
+      const int col = rank_column(bits, pre, n_words, U, R);
       biasbuf[grp * TC + jj] = (col >= 0 && bias_g) ? __ldg(bias_g + col) * kLog2e : 0.f;
       maskbuf[jj] = walk_chunk(walk, t, n_tok, c * TC, bits, pre, P.st);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
-      if constexpr (STAGED) {
-        cp_async_wait_all();
-      } else {             // ... or decoded from the store
+      {   // decoded from the store
         uint32_t chain = 0;   // loops 2..loop that rewrote the column
         if (col >= 0)
           for (int r = 2; r <= P.loop; ++r)
@@ -570,10 +703,10 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
   if (threadIdx.x == 0 && sh.abort_flag) record_error(P.st, timeout_code(sh.abort_flag));
 }
 
-template <bool STAGED>
+template <int MODE>
 __global__ void __launch_bounds__(NTHR, 1) k_attn_tile(const __grid_constant__ AttnParams P) {
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
-  attn_tile_cta<STAGED>(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
+  attn_tile_cta<MODE>(P, blockIdx.x / n_tiles, (blockIdx.x % n_tiles) * TQ);
 }
 
 // Many calls in one launch (batched decode: one store per sequence): CTA b works on call
@@ -590,10 +723,74 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams*
   }
   __syncthreads();
   const int n_tiles = (sP.n_q + TQ - 1) / TQ;
-  attn_tile_cta<false>(sP, b / n_tiles, (b % n_tiles) * TQ);
+  attn_tile_cta<DECODE>(sP, b / n_tiles, (b % n_tiles) * TQ);
+}
+
+// The bitmaps of the call's carried sets: one warp per (head, query) builds its row in
+// shared memory (the set's entries OR-ed in, read 8 per lane at a time), then writes it
+// out whole. Entries beyond the query's position or the store are recorded and left out.
+constexpr int BM_WARPS = 4;
+__global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P, uint32_t* __restrict__ bm) {
+  extern __shared__ uint32_t sbm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long rh = (long long)blockIdx.x * BM_WARPS + warp;
+  if (rh >= (long long)P.H * P.n_q) return;   // whole warp; no block barrier below
+  griddep_wait();
+  uint32_t* mine = sbm + (size_t)warp * P.bm_words;
+  for (int w = lane; w < P.bm_words; w += 32) mine[w] = 0u;
+  __syncwarp();
+  const int i = (int)(rh % P.n_q), h = (int)(rh / P.n_q);
+  const int n_tok = P.kv.n_tok, stride = P.sel_stride;
+  const int t = P.q_tok[i];
+  const int srow = P.q_row ? P.q_row[i] : t;
+  if (t >= 0 && t < n_tok && srow >= 0 && srow < P.stat_rows) {   // else recorded by the attention
+    const uint16_t* row = P.sel + ((size_t)h * P.stat_rows + srow) * stride;
+    for (int e0 = 0; e0 < stride; e0 += 256) {
+      int c8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int e = e0 + 32 * k + lane;
+        c8[k] = e < stride ? (int)__ldg(row + e) : (int)FL_SENTINEL;
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int c = c8[k];
+        if (c == (int)FL_SENTINEL) continue;
+        if (c < n_tok && c <= t) atomicOr(&mine[c >> 5], 1u << (c & 31));
+        else record_error(P.st, FL_ERR_RANGE);
+      }
+      if (__all_sync(0xffffffffu, c8[7] == (int)FL_SENTINEL)) break;   // padding reached
+    }
+  }
+  __syncwarp();
+  uint4* dst = reinterpret_cast<uint4*>(bm + (size_t)rh * P.bm_words);
+  const uint4* src = reinterpret_cast<const uint4*>(mine);
+  for (int w = lane; w < P.bm_words / 4; w += 32) dst[w] = src[w];
 }
 
 }  // namespace
+
+bool sparse_contig(const AttnParams& P) {
+  return (size_t)P.sel_stride * 16 >= (size_t)P.kv.n_tok;
+}
+
+static int bm_words_of(const AttnParams& P) { return (P.kv.n_tok + TC - 1) / TC * 4; }
+
+size_t sel_bitmap_bytes(const AttnParams& P) {
+  return (size_t)P.H * P.n_q * bm_words_of(P) * sizeof(uint32_t);
+}
+
+cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s) {
+  P.bm_words = bm_words_of(P);
+  P.sel_bm = static_cast<const uint32_t*>(buf);
+  const long long rows = (long long)P.H * P.n_q;
+  if (rows <= 0) return cudaSuccess;
+  const size_t smem = (size_t)BM_WARPS * P.bm_words * sizeof(uint32_t);   // <= 32 KB
+  const cudaError_t e = launch_pdl(k_sel_bitmap, dim3((unsigned)((rows + BM_WARPS - 1) / BM_WARPS)),
+                                   dim3(BM_WARPS * 32), smem, s, P, static_cast<uint32_t*>(buf));
+  count_launch();
+  return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 bool sparse_tile_eligible(const AttnParams& P) {
   if (P.hd != HDT || P.kv.hd != HDT || !P.sel) return false;
@@ -619,7 +816,7 @@ cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   if (!attr_set[dev]) {
-    for (auto k : {k_attn_tile<true>, k_attn_tile<false>}) {
+    for (auto k : {k_attn_tile<DECODE>, k_attn_tile<UNION>, k_attn_tile<CONTIG>}) {
       const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                  (int)SMEM_BYTES);
       if (e != cudaSuccess) return e;
@@ -627,8 +824,9 @@ cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s) {
     attr_set[dev] = true;
   }
   const int n_tiles = (P.n_q + TQ - 1) / TQ;
-  const cudaError_t e = launch_pdl(P.stage.khi ? k_attn_tile<true> : k_attn_tile<false>,
-                                   dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, P);
+  auto kern = !P.stage.khi || !P.sel_bm ? k_attn_tile<DECODE>
+                                        : (sparse_contig(P) ? k_attn_tile<CONTIG> : k_attn_tile<UNION>);
+  const cudaError_t e = launch_pdl(kern, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, P);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -547,14 +547,23 @@ fl_status fl_block_out_ffn(const fl_model* m, int32_t layer, float* x, int32_t n
 static size_t loop_attn_ws(const fl_model* m, const fl_schedule* s) {
   if (!s || m->head_dim != 128) return 0;
   const size_t rows = (size_t)m->n_heads * m->n_tok * m->head_dim * sizeof(uint16_t);
+  // the sparse loops' set bitmaps (tiles over plain column ranges): H x active x words
+  size_t bm = 0;
+  for (int r = 2; r <= s->n_loops && r <= FL_MAX_LOOPS; ++r)
+    if (s->col_k[r] > 0) {
+      const size_t b = (size_t)m->n_heads * s->n_active[r] * ((m->n_tok + 127) / 128 * 4) * 4;
+      bm = b > bm ? b : bm;
+    }
   int kmax = 0;
   for (int r = 1; r < s->n_loops && r < FL_MAX_LOOPS; ++r)
     if ((r == 1 || s->col_k[r] == 0) && s->col_k[r + 1] > kmax) kmax = s->col_k[r + 1];
-  if (kmax == 0) return 2 * rows;
+  const size_t sparse = align_up(2 * rows, 256) + bm;
+  if (kmax == 0) return sparse;
   AttnParams P{};
   P.H = m->n_heads; P.hd = m->head_dim; P.n_q = m->n_tok; P.k_next = kmax;
   P.sel_out = reinterpret_cast<uint16_t*>(1);
-  return align_up(dense_tile_ws_bytes(P), 256) + 3 * rows;
+  const size_t dense = align_up(dense_tile_ws_bytes(P), 256) + 3 * rows;
+  return dense > sparse ? dense : sparse;
 }
 
 static size_t loop_ws_layout(const fl_model* m, const fl_schedule* sc, Carver* c, int32_t** iota,

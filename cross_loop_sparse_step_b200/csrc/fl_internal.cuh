@@ -157,7 +157,17 @@ struct AttnParams {
   void* out; int out_bf16;
   int* st;
   KvStage stage;   // khi == NULL: the kernels decode the store themselves
+  // bitmaps of the carried sets, [H][n_q][bm_words] (bit j of word w: column 32 w + j),
+  // for query tiles that walk plain column ranges; NULL: tiles walk their sets' union
+  const uint32_t* sel_bm;
+  int bm_words;
 };
+// Sparse calls whose tiles walk plain column ranges (their unions are nearly every column
+// before the tile: the budget is a sizeable fraction of the prompt), the bitmaps' size,
+// and their construction from the call's column sets.
+bool sparse_contig(const AttnParams& P);
+size_t sel_bitmap_bytes(const AttnParams& P);
+cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s);
 
 bool sparse_tile_eligible(const AttnParams& P);
 cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s);

@@ -438,7 +438,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
               const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
                                           sc2, b2[j / 2]);
               const float2 d = __fadd2_rn(x, negm);
-              const __half2 hv = __floats2half2_rn(exp2f(d.x), exp2f(d.y));
+              const __half2 hv = __floats2half2_rn(ex2_ftz(d.x), ex2_ftz(d.y));
               const uint32_t ma = (uint32_t)((int)(mw << (31 - j)) >> 31);
               const uint32_t mb = (uint32_t)((int)(mw << (30 - j)) >> 31);
               const uint32_t pm = __byte_perm(ma, mb, 0x5410);

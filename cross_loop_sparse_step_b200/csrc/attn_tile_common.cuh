@@ -27,6 +27,15 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
+// 2^x by the PTX ex2.approx.ftz instruction (relative error about 2^-22; subnormal
+// inputs and results flushed to zero). Used for softmax weights that are rounded to fp16
+// right after, whose smallest subnormal is 2^-24: flushing below 2^-126 changes none.
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);

@@ -628,6 +628,7 @@ def main():
             lib.fl_set_timing_events(kind, None, None, 0)
 
     simt_captured = 0
+    attn_paths_step = None   # attention calls of one step by kernel path
     graph = None        # the timed step
     graph_h = None      # the same step with kernel events (per-kernel times, replayed apart:
     kernels_per_step = None   # event nodes between kernels would hold back their overlap)
@@ -637,11 +638,13 @@ def main():
         c0 = lib.fl_launch_count()
         lib.fl_gemm_bf16_cuda_core_count.restype = ctypes.c_int64
         s0 = lib.fl_gemm_bf16_cuda_core_count()
+        p0 = fl.attn_path_counts()
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             step_loops(W)
         kernels_per_step = lib.fl_launch_count() - c0
         simt_captured = lib.fl_gemm_bf16_cuda_core_count() - s0
+        attn_paths_step = {k: v - p0[k] for k, v in fl.attn_path_counts().items() if v - p0[k]}
         restore(W)
         torch.cuda.synchronize()
         arm_hooks()
@@ -837,6 +840,7 @@ def main():
             "launch_mode": "cuda-graph replay" if graph is not None else "eager",
             "clocks": clk,
             "gemm_bf16_cuda_core_launches": int(simt_launches),
+            "attention_paths_per_step": attn_paths_step,
             "knobs": knobs,
             "kv_bytes_per_token_per_layer": kvb,
             "kv_dense_bytes_per_token_per_layer": dense,

@@ -13,6 +13,8 @@
 //      next loop's m' and u' from the kept / dropped columns.
 #include <float.h>
 #include <vector>
+#include <atomic>
+
 #include "fl_internal.cuh"
 
 namespace fl {
@@ -372,6 +374,14 @@ cudaError_t launch_attention_list(const AttnParams& P, const int* list, const in
 
 static bool attn_tile_enabled();
 
+static std::atomic<long long> g_attn_paths[N_ATTN_PATHS];
+void count_attn_path(int path) {
+  if (path >= 0 && path < N_ATTN_PATHS) g_attn_paths[path].fetch_add(1, std::memory_order_relaxed);
+}
+long long attn_path_count(int path) {
+  return path >= 0 && path < N_ATTN_PATHS ? g_attn_paths[path].load() : 0;
+}
+
 
 // Staging of the store as fp16 rows (kv_stage.cu) pays off where several query tiles of a
 // head would decode the same columns: the dense producer, and sparse calls of more than
@@ -417,6 +427,7 @@ cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, 
   if (e != cudaSuccess) return e;
   bool tile = attn_tile_enabled();
   for (int i = 0; tile && i < n; ++i) tile = sparse_tile_eligible(host[i]);
+  count_attn_path(tile ? PATH_TILE_DECODE : PATH_SPARSE_WARP);
   if (tile) return launch_attn_tile_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
   int loop_max = 1;   // shared-memory slices sized for the deepest call
   for (int i = 0; i < n; ++i) loop_max = host[i].loop > loop_max ? host[i].loop : loop_max;
@@ -451,6 +462,7 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
         P.stage.khi = nullptr;   // staged rows without set bitmaps: decode in the tiles
       }
     }
+    count_attn_path(!P.stage.khi ? PATH_TILE_DECODE : (sparse_contig(P) ? PATH_TILE_CONTIG : PATH_TILE_UNION));
     return launch_attn_tile(P, s);
   }
   if (!sparse && attn_tile_enabled() && dense_tile_eligible(P)) {
@@ -461,10 +473,12 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
       const cudaError_t e = launch_kv_stage(P.kv, P.loop, ws + align_up(db), lo, &P.stage, s);
       if (e != cudaSuccess) return e;
     }
+    count_attn_path(PATH_DENSE_TILE);
     return launch_attn_dense_tile(P, a.ws, s);
   }
-  if (sparse && sparse_fast_eligible(P)) return launch_attn_sparse_fast(P, s);
-  if (!sparse && dense_fast_eligible(P)) return launch_attn_dense_fast(P, s);
+  if (sparse && sparse_fast_eligible(P)) { count_attn_path(PATH_SPARSE_WARP); return launch_attn_sparse_fast(P, s); }
+  if (!sparse && dense_fast_eligible(P)) { count_attn_path(PATH_DENSE_WARP); return launch_attn_dense_fast(P, s); }
+  count_attn_path(PATH_GENERAL);
   const int max_cols = sparse ? a.sel_stride : a.kv->n_tok;
   if (sparse) {
     if (P.hd == 128) return launch_t<128, 16>(P, max_cols, s);

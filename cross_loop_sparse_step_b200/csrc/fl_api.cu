@@ -309,6 +309,11 @@ int64_t fl_launch_count(void) { return (int64_t)g_launches.load(); }
 
 int64_t fl_gemm_bf16_cuda_core_count(void) { return (int64_t)g_bf16_simt.load(); }
 
+int32_t fl_attn_path_counts(int64_t* out, int32_t n) {
+  for (int i = 0; out && i < n && i < N_ATTN_PATHS; ++i) out[i] = attn_path_count(i);
+  return N_ATTN_PATHS;
+}
+
 fl_status fl_set_timing_events(int32_t kind, void* const* begin, void* const* end, int32_t n) {
   FL_CHECK(kind >= 0 && kind < TIMED_KINDS && n >= 0, FL_ERR_INVALID_ARG);
   FL_CHECK(n == 0 || (begin && end), FL_ERR_INVALID_ARG);

@@ -169,6 +169,11 @@ bool sparse_contig(const AttnParams& P);
 size_t sel_bitmap_bytes(const AttnParams& P);
 cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s);
 
+// attention calls by path (fl_attn_path_counts)
+enum AttnPath : int { PATH_TILE_CONTIG = 0, PATH_TILE_UNION, PATH_TILE_DECODE, PATH_DENSE_TILE,
+                      PATH_SPARSE_WARP, PATH_DENSE_WARP, PATH_GENERAL, N_ATTN_PATHS };
+void count_attn_path(int path);
+long long attn_path_count(int path);
 bool sparse_tile_eligible(const AttnParams& P);
 cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s);
 cudaError_t launch_attn_tile_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,

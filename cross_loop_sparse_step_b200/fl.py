@@ -97,6 +97,7 @@ def _sig(name, res, args):
 
 
 _status_str = _sig("fl_status_str", ctypes.c_char_p, [c_i32])
+_attn_paths = _sig("fl_attn_path_counts", c_i32, [ctypes.POINTER(ctypes.c_int64), c_i32])
 _version = _sig("fl_version", ctypes.c_char_p, [])
 _check = _sig("fl_check_device_status", c_i32, [vp])
 _detail = _sig("fl_last_error_detail", c_i32, [])
@@ -366,11 +367,23 @@ def make_schedule(n_loops, first_sparse, n_active, col_k, stat_kind=STAT_PV):
     return s
 
 
+ATTN_PATHS = ("tile-column-ranges", "tile-union", "tile-decode", "dense-tile", "sparse-warp",
+              "dense-warp", "general")
+
+
+def attn_path_counts():
+    """Attention calls of this process by the kernel path that ran (fl_attn_path_counts)."""
+    buf = (ctypes.c_int64 * len(ATTN_PATHS))()
+    n = _attn_paths(buf, len(ATTN_PATHS))
+    assert n == len(ATTN_PATHS), n
+    return {name: int(buf[i]) for i, name in enumerate(ATTN_PATHS)}
+
+
 def stat_stride(k):
-    """Statistics row stride for a budget of k columns plus the sink: k + 1 rounded up to
-    a multiple of 8, so every row of the uint16 column sets starts on a 16-byte boundary
-    (the attention kernels then read the sets 8 entries per load)."""
-    return (k + 1 + 7) // 8 * 8
+    """Statistics row stride for a budget of k columns plus the sink: k + 1. (A sparse
+    call whose budget for the next loop is unchanged keeps its statistics in place; the
+    attention recognises that case by k_next + 1 >= stride.)"""
+    return k + 1
 
 
 class LoopRunner:

@@ -67,6 +67,17 @@ int64_t fl_launch_count(void);
  * and are not counted. */
 int64_t fl_gemm_bf16_cuda_core_count(void);
 
+/* Attention calls (fl_sparse_loop_attn, fl_sparse_loop_attn_batched and the attention of
+ * fl_loop_step) by the kernel path that ran, in this process: out[i] for i < n of
+ *   0 sparse query tiles over column ranges (store staged as fp16 rows, set bitmaps)
+ *   1 sparse query tiles over the union of the tile's sets (staged rows, set bitmaps)
+ *   2 sparse query tiles decoding the store themselves (single-tile and batched calls)
+ *   3 dense query tiles (the producer of the next loop's statistics)
+ *   4 sparse warp-per-query kernel   5 dense warp-per-query kernel   6 general kernel
+ * Returns the number of paths (7); n may be smaller. Counted when the host dispatches,
+ * so a captured graph's replays are not counted again. */
+int32_t fl_attn_path_counts(int64_t* out, int32_t n);
+
 /* Measurement hook. With n > 0 the library records the caller's events begin[i] and
  * end[i] (each a cudaEvent_t passed as void*) on the launch stream around its next n
  * launches of one kind (0: the projection GEMMs, 1: the attention kernel);

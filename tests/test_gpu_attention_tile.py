@@ -61,7 +61,7 @@ def test_tile_attention_matches_oracle(name, n, H, g, R, bits, counts, k, use_bi
     # whole prefix), evenly spaced sets for the others
     S, m, u = _stats(rs, n, H, hd, k, act, bias_cols, act[pick])
     if pad:
-        Sp = np.full(S.shape[:2] + (fl.stat_stride(k),), 0xFFFF, S.dtype)
+        Sp = np.full(S.shape[:2] + ((k + 1 + 7) // 8 * 8,), 0xFFFF, S.dtype)
         Sp[..., : S.shape[2]] = S
         S = Sp
     q = synth.query_values(rs, len(act), H, hd)

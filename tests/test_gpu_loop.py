@@ -187,16 +187,25 @@ def test_4k_workload_24_layers_invariants():
     colk = {r: cfg["col_k"][r] for r in range(2, R + 1)}
     sched = fl.make_schedule(R, 2, n_active, colk)
     k = colk[2]
-    run = fl.LoopRunner(model, sched, n_active, stores, k + 1)
+    run = fl.LoopRunner(model, sched, n_active, stores, fl.stat_stride(k))
     run.h.copy_(dev(synth.embeddings(g, N, d)))
+    p0 = fl.attn_path_counts()
     run.step(1)
+    p1 = fl.attn_path_counts()
+    # loop 1: every layer's dense attention on the tensor-core producer
+    assert p1["dense-tile"] - p0["dense-tile"] == L, (p0, p1)
     cur, prev, _ = synth.pareto_delta_pair(g, N, d, 2)
     run.x_prev.copy_(run.h - dev((cur - prev).astype(np.float32)))
     for r in range(2, R + 1):
         h_before = host(run.h).copy()
         kv_before = [host(s.codes[(1, 0)]).copy() for s in stores[:2]]
+        p0 = fl.attn_path_counts()
         run.step(r)
+        p1 = fl.attn_path_counts()
         assert fl.check_device_status() == 0
+        # a sparse loop: every layer on the query-tile kernel over staged rows
+        tiles = sum(p1[x] - p0[x] for x in ("tile-column-ranges", "tile-union"))
+        assert tiles == L and sum(p1.values()) - sum(p0.values()) == L, (r, p0, p1)
         act = host(run.act[r])
         assert len(act) == n_active[r] == 820
         assert np.all(np.diff(act) > 0) and act.min() >= 0 and act.max() < N

@@ -53,8 +53,10 @@ enum : int { PASS_FLASH = 0, PASS_HIST = 1, PASS_CAND = 2, PASS_UNSEL = 3 };
 constexpr uint32_t OFF_QHI = 0;
 constexpr uint32_t OFF_R1 = OFF_QHI + TILE;      // P | histogram [NBIN][TQ] u16 | Q lo
 constexpr uint32_t OFF_ST = OFF_R1 + TILE;       // stage s: tile A at OFF_ST + 2 s TILE, B after
-constexpr uint32_t OFF_META = OFF_ST + 4 * TILE; // [2][TC] bias (log2 units), [2][TC] log2 ||V^||
-constexpr uint32_t SMEM_BYTES = OFF_META + 4 * TC * 4 + 1024;
+// [2][TC] bias (log2 units), [2][TC] log2 ||V^||, [2][TC] their sum, [2][4] the four
+// producer warps' largest log2 ||V^|| of the chunk
+constexpr uint32_t OFF_META = OFF_ST + 4 * TILE;
+constexpr uint32_t SMEM_BYTES = OFF_META + (6 * TC + 8) * 4 + 1024;
 static_assert(NBIN * TQ * 2 <= TILE, "histogram fits its region");
 
 struct DenseArgs {
@@ -196,52 +198,81 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     }
     asm volatile("bar.sync 1, %0;" ::"n"(5 * 32) : "memory");
 
-    // unselected pass: the row's maximum and sum, and its S' walked in step with the chunks
+    // unselected pass: the row's final maximum and sum; S' read as a bitmap of columns
     float m_used = -INFINITY, lsum = 0.f;
-    const uint16_t* sel_row = nullptr;
-    int ent = 0;
-    bool ended = true;
-    uint32_t nx[8];
-    int gr[8], gmax = -1;
-    auto load_next = [&]() {
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        nx[k] = (!ended && ent + k < P.out_stride) ? (uint32_t)sel_row[ent + k] : (uint32_t)FL_SENTINEL;
-      ent += 8;
-    };
-    auto take_next = [&]() {
-      gmax = -1;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int c = (int)nx[k];
-        gr[k] = -1;
-        if (ended || c == (int)FL_SENTINEL) { ended = true; continue; }
-        if (c > t) continue;
-        gr[k] = c;
-        gmax = c;
-      }
-      if (ent >= P.out_stride) ended = true;
-      load_next();
-    };
-#pragma unroll
-    for (int k = 0; k < 8; ++k) gr[k] = -1;
+    const uint4* bmrow = nullptr;
+    uint4 sw_next = make_uint4(0u, 0u, 0u, 0u);   // S' words of the next chunk, read ahead
     if (mode == 2 && valid) {
       const float2 ml = A.m1l[rh];
       m_used = ml.x;
       lsum = ml.y;
-      sel_row = P.sel_out + ((size_t)h * P.stat_rows + srow) * P.out_stride;
-      ended = false;
-      load_next();
-      take_next();
+      bmrow = reinterpret_cast<const uint4*>(P.sel_bm + ((size_t)h * P.n_q + qi) * P.bm_words);
+      if (nc > 0) sw_next = __ldg(bmrow);
     }
     const bool sel_row_stats = stats && valid && t > A.k;   // rows that rank columns
     // m_used: the reference of P and the sum (raised only by more than 2^8); m_true: the
-    // exact running maximum, which anchors the histogram
+    // running maximum (up to the fp16 rounding of P), which anchors the histogram
     float m_true = -INFINITY, lvmax = -INFINITY, ktop = 0.f, thr = -INFINITY, p0 = 0.f;
     int cand = 0;
     uint16_t* hist = reinterpret_cast<uint16_t*>(smem + OFF_R1);
+    uint32_t* hist32 = reinterpret_cast<uint32_t*>(smem + OFF_R1);   // two rows' counts per word
     uint8_t* pt = smem + OFF_R1;
     const bool pv_stat = P.stat_kind == FL_STAT_PV;
+    const float2 sc2 = make_float2(scale2, scale2);
+
+    // P = 2^(x - m_used) (x = s * scale2 + bias) as fp16 into the P tile for the columns of
+    // the 16-column groups' masks mask16(g); the row sum over the fp16 values when `sum`;
+    // the largest P written (in fp16) is returned. TMEM loads of the next group fly while
+    // a group is processed.
+    auto p_pass = [&](uint32_t s_addr, const float* bias, auto mask16, bool sum) -> float {
+      const float2 negm = make_float2(-m_used, -m_used);
+      float2 acc = make_float2(0.f, 0.f);
+      __half2 hmax = __float2half2_rn(0.f);
+      auto group = [&](int g, const uint32_t (&r)[16]) {
+        const uint32_t mw = mask16(g);
+        uint32_t pk[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+        if (__any_sync(0xffffffffu, mw)) {
+          const float2* b2 = reinterpret_cast<const float2*>(bias + g * 16);
+#pragma unroll
+          for (int j = 0; j < 16; j += 2) {
+            const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                        sc2, b2[j / 2]);
+            const float2 d = __fadd2_rn(x, negm);
+            const __half2 hv = __floats2half2_rn(ex2_ftz(d.x), ex2_ftz(d.y));
+            const uint32_t ma = (uint32_t)((int)(mw << (31 - j)) >> 31);
+            const uint32_t mb = (uint32_t)((int)(mw << (30 - j)) >> 31);
+            const uint32_t pv = *reinterpret_cast<const uint32_t*>(&hv) & __byte_perm(ma, mb, 0x5410);
+            const __half2 ph = *reinterpret_cast<const __half2*>(&pv);
+            hmax = __hmax2(hmax, ph);
+            if (sum) acc = __fadd2_rn(acc, __half22float2(ph));
+            pk[j / 2] = pv;
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          *reinterpret_cast<uint4*>(pt + sw128_offset(i, g * 16 + q * 8, TQ)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+      };
+      uint32_t ra[16], rb[16];
+      tmem_ld16_issue(s_addr, ra);
+#pragma unroll 1
+      for (int g = 0; g < 8; g += 2) {
+        tmem_ld16_wait(ra);
+        tmem_ld16_issue(s_addr + (g + 1) * 16, rb);
+        group(g, ra);
+        tmem_ld16_wait(rb);
+        if (g + 2 < 8) tmem_ld16_issue(s_addr + (g + 2) * 16, ra);
+        group(g + 1, rb);
+      }
+      if (sum) lsum += acc.x + acc.y;
+      const float2 hm = __half22float2(hmax);
+      return fmaxf(hm.x, hm.y);
+    };
+    // causal columns of a 16-column group: [0, nin) of the chunk
+    auto causal16 = [](int g, int nin) -> uint32_t {
+      const int n = nin - g * 16;
+      return n >= 16 ? 0xFFFFu : (n > 0 ? (1u << n) - 1u : 0u);
+    };
 
     for (int G = 0; G < total; ++G) {
       const int pass = pass_of(mode, G, nc);
@@ -253,62 +284,61 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const uint32_t s_addr = tmem + lane_base + (uint32_t)(sb * TC);
       const float* bias = meta + sb * TC;
       const float* lvn = meta + 2 * TC + sb * TC;
+      const float* blv = meta + 4 * TC + sb * TC;           // bias + log2 ||V^||
       const int nin = t < 0 ? 0 : min(max(t - c * TC + 1, 0), TC);   // causal columns
       if (pass == PASS_FLASH) {
-        float cmax = -INFINITY;
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(s_addr + g4 * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int jj = g4 * 32 + j;
-            if (jj < nin) {
-              cmax = fmaxf(cmax, fmaf(v[j], scale2, bias[jj]));
-              lvmax = fmaxf(lvmax, lvn[jj]);
-            }
+        // the largest log2 ||V^|| the row saw: the chunk's (producers) or, on the diagonal
+        // chunk, over the row's own columns
+        if (stats) {
+          if (nin == TC) {
+            const float* lm = meta + 6 * TC + sb * 4;
+            lvmax = fmaxf(lvmax, fmaxf(fmaxf(lm[0], lm[1]), fmaxf(lm[2], lm[3])));
+          } else {
+            for (int jj = 0; jj < nin; ++jj) lvmax = fmaxf(lvmax, lvn[jj]);
           }
-        }
-        m_true = fmaxf(m_true, cmax);
-        float alpha = 1.f;
-        bool rescale = false;
-        if (cmax > m_used + kRescale) {
-          if (m_used != -INFINITY && lsum > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
-          m_used = cmax;
         }
         if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, site_of(3 + 16 * mode, G, warp))) break;
         tc_fence_after();
-        if (rescale) lsum *= alpha;
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t o_addr = tmem + lane_base + 2u * TC;
+        // one pass against the running maximum; a row whose P exceeds 2^8 (a column more
+        // than 8 above m_used, or the first chunk) takes the chunk's maximum first (O and
+        // the sum rescaled) and writes P again
+        const float lsum0 = lsum;
+        auto mk = [&](int g) { return causal16(g, nin); };
+        const float pmax = p_pass(s_addr, bias, mk, true);
+        const bool over = pmax > 256.f;
+        if (!over && pmax > 0.f) m_true = fmaxf(m_true, m_used + log2f(pmax) + 1.f / 1024);
+        if (__any_sync(0xffffffffu, over)) {
+          float cmax = -INFINITY;
 #pragma unroll 1
-          for (int g4 = 0; g4 < 4; ++g4) {
-            float v[32];
-            tmem_ld32(o_addr + g4 * 32, v);
+          for (int g = 0; g < 8; ++g) {
+            const uint32_t mw = causal16(g, nin);
+            if (!__any_sync(0xffffffffu, mw)) continue;
+            float v[16];
+            tmem_ld16(s_addr + g * 16, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= alpha;
-            tmem_st32(o_addr + g4 * 32, v);
+            for (int j = 0; j < 16; ++j)
+              cmax = fmaxf(cmax, (mw >> j) & 1u ? fmaf(v[j], scale2, bias[g * 16 + j]) : -INFINITY);
           }
-        }
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(s_addr + g4 * 32, v);
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int jj = g4 * 32 + j;
-            const float a = jj < nin ? exp2f(fmaf(v[j], scale2, bias[jj]) - m_used) : 0.f;
-            const float b = jj + 1 < nin ? exp2f(fmaf(v[j + 1], scale2, bias[jj + 1]) - m_used) : 0.f;
-            const __half2 hv = __floats2half2_rn(a, b);
-            const float2 back = __half22float2(hv);
-            lsum += back.x + back.y;
-            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
+          m_true = fmaxf(m_true, cmax);
+          float alpha = 1.f;
+          bool rescale = false;
+          if (cmax > m_used + kRescale) {
+            if (m_used != -INFINITY && lsum0 > 0.f) { alpha = exp2f(m_used - cmax); rescale = true; }
+            m_used = cmax;
           }
+          lsum = rescale ? lsum0 * alpha : lsum0;
+          if (__any_sync(0xffffffffu, rescale)) {
+            const uint32_t o_addr = tmem + lane_base + 2u * TC;
+#pragma unroll 1
+            for (int g4 = 0; g4 < 4; ++g4) {
+              float v[32];
+              tmem_ld32(o_addr + g4 * 32, v);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(pt + sw128_offset(i, g4 * 32 + q * 8, TQ)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+              for (int j = 0; j < 32; ++j) v[j] *= alpha;
+              tmem_st32(o_addr + g4 * 32, v);
+            }
+          }
+          p_pass(s_addr, bias, mk, true);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -343,24 +373,41 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           if (stats) {
             if (valid) A.m1l[rh] = make_float2(m_used, lsum);
             ktop = m_true + (pv_stat ? lvmax : 0.f);
-            // the histogram takes the P region over (every thread saw the last P V^ finish)
+            // the histogram takes the P region over (every thread saw the last P V^ finish);
+            // a row's counts are 16-bit halves of words shared with the neighbouring row,
+            // both in this warp
             for (int b = 0; b < NBIN; ++b) hist[b * TQ + i] = 0;
+            __syncwarp();
           }
         }
       } else if (pass == PASS_HIST) {
+        {
+          // kappa = s * scale2 + bias + log2 ||V^|| binned by (ktop - kappa) * 8 below the
+          // row's upper bound; bins incremented by shared-memory atomics (no read-modify-
+          // write chain through a row's counts). Every lane runs the loop (the TMEM loads
+          // are warp-collective); rows that rank nothing have empty masks.
+          const float kt8 = ktop * kBinsPerLog2;
+          const float2 nb2 = make_float2(-kBinsPerLog2, -kBinsPerLog2);
+          const uint32_t inc = (i & 1) ? 0x10000u : 1u;
+          uint32_t* hrow = hist32 + (i >> 1);
+#pragma unroll 1
+          for (int g = 0; g < 8; ++g) {
+            uint32_t mw = sel_row_stats ? causal16(g, nin) : 0u;
+            if (c == 0 && g == 0) mw &= ~1u;   // the sink is kept apart
+            if (!__any_sync(0xffffffffu, mw)) continue;
+            float v[16];
+            tmem_ld16(s_addr + g * 16, v);
+            const float2* b2 = reinterpret_cast<const float2*>(blv + g * 16);
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(s_addr + g4 * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int jj = g4 * 32 + j;
-            if (sel_row_stats && jj < nin && (c > 0 || jj > 0)) {
-              const float kap = fmaf(v[j], scale2, bias[jj]) + (pv_stat ? lvn[jj] : 0.f);
-              float bf = (ktop - kap) * kBinsPerLog2;
-              bf = fminf(fmaxf(bf, 0.f), (float)(NBIN - 1));   // NaN-free: kap finite or -inf
-              const int b = (int)bf;
-              hist[b * TQ + i] += 1;
+            for (int j = 0; j < 16; j += 2) {
+              const float2 kap = __ffma2_rn(make_float2(v[j], v[j + 1]), sc2,
+                                            pv_stat ? b2[j / 2] : make_float2(bias[g * 16 + j], bias[g * 16 + j + 1]));
+              const float2 bf = __ffma2_rn(kap, nb2, make_float2(kt8, kt8));
+              // NaN-free: kappa finite or -inf
+              const int ba = (int)fminf(fmaxf(bf.x, 0.f), (float)(NBIN - 1));
+              const int bb = (int)fminf(fmaxf(bf.y, 0.f), (float)(NBIN - 1));
+              if ((mw >> j) & 1u) atomicAdd(hrow + ba * (TQ / 2), inc);
+              if ((mw >> (j + 1)) & 1u) atomicAdd(hrow + bb * (TQ / 2), inc);
             }
           }
         }
@@ -368,6 +415,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
         if (lane == 0) sh.prog[warp - 4] = G;
         if (c == nc - 1) {
+          __syncwarp();
           // ---- the bin of the k-th largest; the candidate threshold one margin below it
           if (sel_row_stats) {
             int acc = 0, b = 0;
@@ -428,46 +476,16 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           A.cnt[rh] = cand;
           A.p0[rh] = p0;
         }
-      } else {   // PASS_UNSEL: u' over the columns outside S'
-        uint32_t mask[4] = {0u, 0u, 0u, 0u};   // columns of S' in this chunk
-        const int lo = c * TC, hi = lo + TC;
-        while (true) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int pos = gr[k] - lo;
-            const uint32_t bit = (pos >= 0 && pos < TC) ? 1u << (pos & 31) : 0u;
-            const int w = pos >> 5;
-            mask[0] |= w == 0 ? bit : 0u;
-            mask[1] |= w == 1 ? bit : 0u;
-            mask[2] |= w == 2 ? bit : 0u;
-            mask[3] |= w == 3 ? bit : 0u;
-          }
-          if (gmax < hi && !ended) take_next();
-          else break;
-        }
-        __syncwarp();   // reconverge before the warp-collective TMEM accesses
+      } else {   // PASS_UNSEL: u' over the causal columns outside S'
+        const uint4 sw = sw_next;   // S' among the chunk's columns
+        if (bmrow && c + 1 < nc) sw_next = __ldg(bmrow + c + 1);
         if (c > 0 && !warp_wait(&sh.pv_done, (c - 1) & 1, abort, site_of(11 + 16 * mode, G, warp))) break;
         tc_fence_after();
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(s_addr + g4 * 32, v);
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const int jj = g4 * 32 + j;
-            const bool ina = jj < nin && !(mask[g4] & (1u << j));
-            const bool inb = jj + 1 < nin && !(mask[g4] & (1u << (j + 1)));
-            const float a = ina ? exp2f(fmaf(v[j], scale2, bias[jj]) - m_used) : 0.f;
-            const float b = inb ? exp2f(fmaf(v[j + 1], scale2, bias[jj + 1]) - m_used) : 0.f;
-            const __half2 hv = __floats2half2_rn(a, b);
-            pk[j / 2] = *reinterpret_cast<const uint32_t*>(&hv);
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(pt + sw128_offset(i, g4 * 32 + q * 8, TQ)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
+        auto mk = [&](int g) -> uint32_t {
+          const uint32_t w = g < 2 ? sw.x : (g < 4 ? sw.y : (g < 6 ? sw.z : sw.w));
+          return causal16(g, nin) & ~((w >> ((g & 1) * 16)) & 0xFFFFu);
+        };
+        p_pass(s_addr, bias, mk, false);
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
@@ -581,9 +599,15 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const int c = G % nc;
       const int colv = c * TC + jj;
       const int col = colv <= t_max ? colv : -1;
-      meta[grp * TC + jj] = (col >= 0 && P.bias) ? __ldg(P.bias + col) * kLog2e : 0.f;
-      meta[2 * TC + grp * TC + jj] =
-          (col >= 0 && pv_stat) ? log2f(__ldg(P.vnorm + (size_t)col * H + h)) : 0.f;
+      const float bv = (col >= 0 && P.bias) ? __ldg(P.bias + col) * kLog2e : 0.f;
+      const float lv = (col >= 0 && pv_stat) ? log2f(__ldg(P.vnorm + (size_t)col * H + h)) : 0.f;
+      meta[grp * TC + jj] = bv;
+      meta[2 * TC + grp * TC + jj] = lv;
+      meta[4 * TC + grp * TC + jj] = bv + lv;
+      float lm = col >= 0 ? lv : -INFINITY;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+      if (lane == 0) meta[6 * TC + grp * 4 + (warp & 3)] = lm;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
       // K^ (pass cand: hi part in A, lo part in B) and, with P V^, V^ in B (MN-major)
@@ -748,7 +772,7 @@ size_t dense_tile_ws_bytes(const AttnParams& P) {
   const size_t rows = (size_t)P.H * P.n_q;
   return align_up(rows * sizeof(float2)) + 2 * align_up(rows * 4) + align_up(rows * cap * 2) +
          align_up(rows * cap * 4) + align_up(4) + align_up(rows * 4) +
-         align_up((size_t)((P.n_q + TQ - 1) / TQ) * P.H * 12 * 4);
+         align_up((size_t)((P.n_q + TQ - 1) / TQ) * P.H * 12 * 4) + align_up(sel_bitmap_bytes(P));
 }
 
 bool dense_tile_eligible(const AttnParams& P) {
@@ -786,6 +810,7 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   const size_t rows = (size_t)P.H * P.n_q;
   int* ovf_n = nullptr;
   int* ovf_list = nullptr;
+  uint8_t* bm_buf = nullptr;
   if (P.sel_out) {
     uint8_t* p = static_cast<uint8_t*>(ws);
     A.m1l = reinterpret_cast<float2*>(p); p += align_up(rows * sizeof(float2));
@@ -795,7 +820,8 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
     A.cp = reinterpret_cast<float*>(p); p += align_up(rows * A.cap * 4);
     ovf_n = reinterpret_cast<int*>(p); p += align_up(4);
     ovf_list = reinterpret_cast<int*>(p); p += align_up(rows * 4);
-    A.dbg = reinterpret_cast<int*>(p);
+    A.dbg = reinterpret_cast<int*>(p); p += align_up((size_t)((P.n_q + TQ - 1) / TQ) * P.H * 12 * 4);
+    bm_buf = p;
     cudaError_t e = cudaMemsetAsync(ovf_n, 0, sizeof(int), s);
     if (e != cudaSuccess) return e;
   }
@@ -818,6 +844,17 @@ cudaError_t launch_attn_dense_tile(const AttnParams& P, void* ws, cudaStream_t s
   count_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  // S' as bitmaps for the unselected pass (rows finished by the exact kernels below get
+  // theirs from stale sets: their u' is overwritten there)
+  {
+    AttnParams Q = P;
+    Q.sel = P.sel_out;
+    Q.sel_stride = P.out_stride;
+    e = launch_sel_bitmap(Q, bm_buf, s, false);
+    if (e != cudaSuccess) return e;
+    A.P.sel_bm = Q.sel_bm;
+    A.P.bm_words = Q.bm_words;
+  }
   A.mode = 2;
   e = launch_pdl(kern, dim3(n_tiles * P.H), dim3(NTHR), SMEM_BYTES, s, A);
   count_launch();

@@ -730,7 +730,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams*
 // shared memory (the set's entries OR-ed in, read 8 per lane at a time), then writes it
 // out whole. Entries beyond the query's position or the store are recorded and left out.
 constexpr int BM_WARPS = 4;
-__global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P, uint32_t* __restrict__ bm) {
+__global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P, uint32_t* __restrict__ bm,
+                                                               int record) {
   extern __shared__ uint32_t sbm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long rh = (long long)blockIdx.x * BM_WARPS + warp;
@@ -757,7 +758,7 @@ __global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P
         const int c = c8[k];
         if (c == (int)FL_SENTINEL) continue;
         if (c < n_tok && c <= t) atomicOr(&mine[c >> 5], 1u << (c & 31));
-        else record_error(P.st, FL_ERR_RANGE);
+        else if (record) record_error(P.st, FL_ERR_RANGE);
       }
       if (__all_sync(0xffffffffu, c8[7] == (int)FL_SENTINEL)) break;   // padding reached
     }
@@ -780,14 +781,15 @@ size_t sel_bitmap_bytes(const AttnParams& P) {
   return (size_t)P.H * P.n_q * bm_words_of(P) * sizeof(uint32_t);
 }
 
-cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s) {
+cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s, bool record) {
   P.bm_words = bm_words_of(P);
   P.sel_bm = static_cast<const uint32_t*>(buf);
   const long long rows = (long long)P.H * P.n_q;
   if (rows <= 0) return cudaSuccess;
   const size_t smem = (size_t)BM_WARPS * P.bm_words * sizeof(uint32_t);   // <= 32 KB
   const cudaError_t e = launch_pdl(k_sel_bitmap, dim3((unsigned)((rows + BM_WARPS - 1) / BM_WARPS)),
-                                   dim3(BM_WARPS * 32), smem, s, P, static_cast<uint32_t*>(buf));
+                                   dim3(BM_WARPS * 32), smem, s, P, static_cast<uint32_t*>(buf),
+                                   record ? 1 : 0);
   count_launch();
   return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -566,6 +566,7 @@ static size_t loop_attn_ws(const fl_model* m, const fl_schedule* s) {
   if (kmax == 0) return sparse;
   AttnParams P{};
   P.H = m->n_heads; P.hd = m->head_dim; P.n_q = m->n_tok; P.k_next = kmax;
+  P.kv.n_tok = m->n_tok;
   P.sel_out = reinterpret_cast<uint16_t*>(1);
   const size_t dense = align_up(dense_tile_ws_bytes(P), 256) + 3 * rows;
   return dense > sparse ? dense : sparse;

@@ -167,7 +167,7 @@ struct AttnParams {
 // and their construction from the call's column sets.
 bool sparse_contig(const AttnParams& P);
 size_t sel_bitmap_bytes(const AttnParams& P);
-cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s);
+cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s, bool record = true);
 
 // attention calls by path (fl_attn_path_counts)
 enum AttnPath : int { PATH_TILE_CONTIG = 0, PATH_TILE_UNION, PATH_TILE_DECODE, PATH_DENSE_TILE,

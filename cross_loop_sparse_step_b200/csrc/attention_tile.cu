@@ -88,7 +88,7 @@ __device__ __forceinline__ int rank_column(const uint32_t* bits, const uint16_t*
 // query's word; every hit lands at its rank within the chunk (the union bits below it).
 // The word loop has the same trip count on every lane.
 __device__ __forceinline__ uint4 bitmap_chunk_mask(const uint32_t* bits, const uint32_t* qbm,
-                                                   int c0, int c1) {
+                                                   int c0, int c1, int t) {
   uint32_t m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u;
   const int wa = c0 >> 5, wb = c1 >> 5;
   int base = 0;
@@ -97,7 +97,13 @@ __device__ __forceinline__ uint4 bitmap_chunk_mask(const uint32_t* bits, const u
     uint32_t ub = bits[w];
     if (w == wa) ub &= ~((1u << (c0 & 31)) - 1u);
     if (w == wb && (c1 & 31) != 31) ub &= (2u << (c1 & 31)) - 1u;
-    uint32_t hit = qbm ? (ub & __ldg(qbm + w)) : 0u;
+    // the query's words cover its own columns [0, t] only
+    uint32_t qb = 0u;
+    if (qbm && w <= (t >> 5)) {
+      qb = __ldg(qbm + w);
+      if (w == (t >> 5) && (t & 31) != 31) qb &= (2u << (t & 31)) - 1u;
+    }
+    uint32_t hit = ub & qb;
     while (hit) {
       const int b = __ffs(hit) - 1;
       hit &= hit - 1u;
@@ -401,8 +407,17 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
       tc_fence_after();
       uint4 mk;   // this row's members among the chunk's columns
       if constexpr (MODE == CONTIG) {
+        // the bitmap covers the row's own columns: the words of later chunks are not its
+        const int nin = valid ? min(max(t - c * TC + 1, 0), TC) : 0;
         mk = mk_next;
         if (bmrow && c + 1 < n_chunks) mk_next = __ldg(bmrow + c + 1);
+        if (nin < TC) {
+          const uint32_t m4[4] = {nin >= 32 ? ~0u : (nin > 0 ? (1u << nin) - 1u : 0u),
+                                  nin >= 64 ? ~0u : (nin > 32 ? (1u << (nin - 32)) - 1u : 0u),
+                                  nin >= 96 ? ~0u : (nin > 64 ? (1u << (nin - 64)) - 1u : 0u),
+                                  nin > 96 ? (1u << (nin - 96)) - 1u : 0u};
+          mk.x &= m4[0]; mk.y &= m4[1]; mk.z &= m4[2]; mk.w &= m4[3];
+        }
       } else {
         mk = maskbuf[sb * TQ + i];
       }
@@ -616,13 +631,16 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
     const size_t hoff = (size_t)h * n_tok * HDT;
     // UNION: query jj's bitmap row (invalid queries have none: recorded by the softmax)
     const uint32_t* qbm = nullptr;
+    int tq = -1;
     if constexpr (MODE == UNION) {
       const int qi = q0 + jj;
       if (qi < P.n_q) {
         const int t = P.q_tok[qi];
         const int srow = P.q_row ? P.q_row[qi] : t;
-        if (t >= 0 && t < n_tok && srow >= 0 && srow < P.stat_rows)
+        if (t >= 0 && t < n_tok && srow >= 0 && srow < P.stat_rows) {
           qbm = P.sel_bm + ((size_t)h * P.n_q + qi) * P.bm_words;
+          tq = t;
+        }
       }
     }
     for (int c = grp; c < n_chunks; c += 2) {
@@ -637,7 +655,7 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
         // the chunk's first and last columns (the same on every lane)
         const int c0 = rank_column(bits, pre, n_words, U, c * TC);
         const int c1 = rank_column(bits, pre, n_words, U, min(U, c * TC + TC) - 1);
-        maskbuf[jj] = bitmap_chunk_mask(bits, qbm, c0, c1);
+        maskbuf[jj] = bitmap_chunk_mask(bits, qbm, c0, c1, tq);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sh.meta_full[grp]);
@@ -727,8 +745,10 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_tile_batched(const AttnParams*
 }
 
 // The bitmaps of the call's carried sets: one warp per (head, query) builds its row in
-// shared memory (the set's entries OR-ed in, read 8 per lane at a time), then writes it
-// out whole. Entries beyond the query's position or the store are recorded and left out.
+// shared memory (the set's entries OR-ed in, 16 per lane in flight), then writes it out.
+// Only the words of the query's own columns are written (whole 128-column chunks up to
+// its position); readers mask the columns beyond a query's position themselves. Entries
+// beyond the query's position or the store are recorded (with `record`) and left out.
 constexpr int BM_WARPS = 4;
 __global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P, uint32_t* __restrict__ bm,
                                                                int record) {
@@ -737,36 +757,36 @@ __global__ void __launch_bounds__(BM_WARPS * 32) k_sel_bitmap(const AttnParams P
   const long long rh = (long long)blockIdx.x * BM_WARPS + warp;
   if (rh >= (long long)P.H * P.n_q) return;   // whole warp; no block barrier below
   griddep_wait();
-  uint32_t* mine = sbm + (size_t)warp * P.bm_words;
-  for (int w = lane; w < P.bm_words; w += 32) mine[w] = 0u;
-  __syncwarp();
   const int i = (int)(rh % P.n_q), h = (int)(rh / P.n_q);
   const int n_tok = P.kv.n_tok, stride = P.sel_stride;
   const int t = P.q_tok[i];
   const int srow = P.q_row ? P.q_row[i] : t;
-  if (t >= 0 && t < n_tok && srow >= 0 && srow < P.stat_rows) {   // else recorded by the attention
-    const uint16_t* row = P.sel + ((size_t)h * P.stat_rows + srow) * stride;
-    for (int e0 = 0; e0 < stride; e0 += 256) {
-      int c8[8];
+  if (t < 0 || t >= n_tok || srow < 0 || srow >= P.stat_rows) return;   // recorded by the attention
+  const int nw = min((t / TC + 1) * 4, P.bm_words);   // words of the query's chunks
+  uint32_t* mine = sbm + (size_t)warp * P.bm_words;
+  for (int w = lane; w < nw; w += 32) mine[w] = 0u;
+  __syncwarp();
+  const uint16_t* row = P.sel + ((size_t)h * P.stat_rows + srow) * stride;
+  for (int e0 = 0; e0 < stride; e0 += 512) {
+    int c16[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int e = e0 + 32 * k + lane;
-        c8[k] = e < stride ? (int)__ldg(row + e) : (int)FL_SENTINEL;
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int c = c8[k];
-        if (c == (int)FL_SENTINEL) continue;
-        if (c < n_tok && c <= t) atomicOr(&mine[c >> 5], 1u << (c & 31));
-        else if (record) record_error(P.st, FL_ERR_RANGE);
-      }
-      if (__all_sync(0xffffffffu, c8[7] == (int)FL_SENTINEL)) break;   // padding reached
+    for (int k = 0; k < 16; ++k) {
+      const int e = e0 + 32 * k + lane;
+      c16[k] = e < stride ? (int)__ldg(row + e) : (int)FL_SENTINEL;
     }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int c = c16[k];
+      if (c == (int)FL_SENTINEL) continue;
+      if (c <= t) atomicOr(&mine[c >> 5], 1u << (c & 31));
+      else if (record) record_error(P.st, FL_ERR_RANGE);
+    }
+    if (__all_sync(0xffffffffu, c16[15] == (int)FL_SENTINEL)) break;   // padding reached
   }
   __syncwarp();
   uint4* dst = reinterpret_cast<uint4*>(bm + (size_t)rh * P.bm_words);
   const uint4* src = reinterpret_cast<const uint4*>(mine);
-  for (int w = lane; w < P.bm_words / 4; w += 32) dst[w] = src[w];
+  for (int w = lane; w < nw / 4; w += 32) dst[w] = src[w];
 }
 
 }  // namespace

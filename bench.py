@@ -65,8 +65,8 @@ def apply_variant(cfg, variant):
         c["tok_frac"] = {r: 1.0 for r in loops}
     if variant == "dense-early":
         c["first_sparse"] = 3
-        c["col_k"] = dict(c["col_k"], **{2: 0})
-        c["tok_frac"] = dict(c["tok_frac"], **{2: 1.0})
+        c["col_k"] = {**c["col_k"], 2: 0}
+        c["tok_frac"] = {**c["tok_frac"], 2: 1.0}
     if variant == "shrink":
         k0 = c["col_k"][2]
         c["col_k"] = {r: max(1, k0 >> (r - 2)) for r in loops}

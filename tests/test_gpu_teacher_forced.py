@@ -269,3 +269,12 @@ def test_4k_workload_all_layers_all_loops():
     rep = run_teacher_forced(dict(configs.C2), configs.C2["n_loops"])
     print("teacher-forced 4K:", rep)
     assert all(v > 0 for v in rep["checked"].values())
+
+
+def test_32k_workload_all_layers_loops_1_2():
+    """The 32K Ouro-2.6B-shape workload the benchmark times: all 48 layers, the dense loop 1
+    (statistics for loop 2, k = 2048 of up to 32K columns) and the sparse loop 2 over the
+    column-range tiles, on a sample of tokens."""
+    rep = run_teacher_forced(dict(configs.C3), 2, n_tap=64, n_dense_check=10)
+    print("teacher-forced 32K:", rep)
+    assert all(v > 0 for v in rep["checked"].values())

@@ -374,6 +374,10 @@ cudaError_t launch_attention_list(const AttnParams& P, const int* list, const in
 
 static bool attn_tile_enabled();
 
+// Sparse calls of at most this many queries stream each query's columns (a query tile
+// would be nearly empty and its union would not be shared).
+constexpr int kStreamMaxQ = 32;
+
 static std::atomic<long long> g_attn_paths[N_ATTN_PATHS];
 void count_attn_path(int path) {
   if (path >= 0 && path < N_ATTN_PATHS) g_attn_paths[path].fetch_add(1, std::memory_order_relaxed);
@@ -425,8 +429,13 @@ cudaError_t launch_attention_batched(const fl_attn_args* args, int n, void* ws, 
   // pageable source: the copy is staged before this call returns
   cudaError_t e = cudaMemcpyAsync(ws, host.data(), n * sizeof(AttnParams), cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return e;
-  bool tile = attn_tile_enabled();
+  bool stream = attn_tile_enabled(), tile = stream;
+  for (int i = 0; stream && i < n; ++i) stream = sparse_decode_eligible(host[i]) && host[i].n_q <= kStreamMaxQ;
   for (int i = 0; tile && i < n; ++i) tile = sparse_tile_eligible(host[i]);
+  if (stream) {
+    count_attn_path(PATH_SPARSE_STREAM);
+    return launch_attn_decode_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
+  }
   count_attn_path(tile ? PATH_TILE_DECODE : PATH_SPARSE_WARP);
   if (tile) return launch_attn_tile_batched(host[0], static_cast<const AttnParams*>(ws), n, s);
   int loop_max = 1;   // shared-memory slices sized for the deepest call
@@ -450,6 +459,10 @@ cudaError_t launch_attention(const fl_attn_args& a, int* st, cudaStream_t s) {
   AttnParams P = make_attn_params(a, st);
   const bool sparse = a.sel != nullptr;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  if (sparse && attn_tile_enabled() && P.n_q <= kStreamMaxQ && sparse_decode_eligible(P)) {
+    count_attn_path(PATH_SPARSE_STREAM);
+    return launch_attn_decode(P, s);
+  }
   if (sparse && attn_tile_enabled() && sparse_tile_eligible(P)) {
     const size_t sb = align_up(kv_stage_bytes(P.kv, false));
     if (stage_sparse(P) && ws && a.ws_bytes >= sb) {

@@ -171,10 +171,17 @@ cudaError_t launch_sel_bitmap(AttnParams& P, void* buf, cudaStream_t s, bool rec
 
 // attention calls by path (fl_attn_path_counts)
 enum AttnPath : int { PATH_TILE_CONTIG = 0, PATH_TILE_UNION, PATH_TILE_DECODE, PATH_DENSE_TILE,
-                      PATH_SPARSE_WARP, PATH_DENSE_WARP, PATH_GENERAL, N_ATTN_PATHS };
+                      PATH_SPARSE_WARP, PATH_DENSE_WARP, PATH_GENERAL, PATH_SPARSE_STREAM,
+                      N_ATTN_PATHS };
 void count_attn_path(int path);
 long long attn_path_count(int path);
 bool sparse_tile_eligible(const AttnParams& P);
+// Sparse calls with few queries (decode): one CTA per (query, head) streaming its carried
+// columns from the quantised store (attention_decode.cu).
+bool sparse_decode_eligible(const AttnParams& P);
+cudaError_t launch_attn_decode(const AttnParams& P, cudaStream_t s);
+cudaError_t launch_attn_decode_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
+                                       cudaStream_t s);
 cudaError_t launch_attn_tile(const AttnParams& P, cudaStream_t s);
 cudaError_t launch_attn_tile_batched(const AttnParams& P0, const AttnParams* Ps_dev, int n,
                                      cudaStream_t s);

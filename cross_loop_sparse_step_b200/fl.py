@@ -368,7 +368,7 @@ def make_schedule(n_loops, first_sparse, n_active, col_k, stat_kind=STAT_PV):
 
 
 ATTN_PATHS = ("tile-column-ranges", "tile-union", "tile-decode", "dense-tile", "sparse-warp",
-              "dense-warp", "general")
+              "dense-warp", "general", "sparse-stream")
 
 
 def attn_path_counts():

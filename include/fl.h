@@ -74,7 +74,9 @@ int64_t fl_gemm_bf16_cuda_core_count(void);
  *   2 sparse query tiles decoding the store themselves (single-tile and batched calls)
  *   3 dense query tiles (the producer of the next loop's statistics)
  *   4 sparse warp-per-query kernel   5 dense warp-per-query kernel   6 general kernel
- * Returns the number of paths (7); n may be smaller. Counted when the host dispatches,
+ *   7 sparse calls of few queries (decode): one CTA per (query, head) streaming its
+ *     carried columns from the quantised store
+ * Returns the number of paths (8); n may be smaller. Counted when the host dispatches,
  * so a captured graph's replays are not counted again. */
 int32_t fl_attn_path_counts(int64_t* out, int32_t n);
 

@@ -273,6 +273,21 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
       const int n = nin - g * 16;
       return n >= 16 ? 0xFFFFu : (n > 0 ? (1u << n) - 1u : 0u);
     };
+    // fn(g, r) for the chunk's eight 16-column groups of S, the loads of the next group
+    // flying while a group is processed (every lane runs it: the loads are warp-collective)
+    auto for_groups = [&](uint32_t s_addr, auto fn) {
+      uint32_t ra[16], rb[16];
+      tmem_ld16_issue(s_addr, ra);
+#pragma unroll 1
+      for (int g = 0; g < 8; g += 2) {
+        tmem_ld16_wait(ra);
+        tmem_ld16_issue(s_addr + (g + 1) * 16, rb);
+        fn(g, ra);
+        tmem_ld16_wait(rb);
+        if (g + 2 < 8) tmem_ld16_issue(s_addr + (g + 2) * 16, ra);
+        fn(g + 1, rb);
+      }
+    };
 
     for (int G = 0; G < total; ++G) {
       const int pass = pass_of(mode, G, nc);
@@ -384,24 +399,21 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
         {
           // kappa = s * scale2 + bias + log2 ||V^|| binned by (ktop - kappa) * 8 below the
           // row's upper bound; bins incremented by shared-memory atomics (no read-modify-
-          // write chain through a row's counts). Every lane runs the loop (the TMEM loads
-          // are warp-collective); rows that rank nothing have empty masks.
+          // write chain through a row's counts); rows that rank nothing have empty masks
           const float kt8 = ktop * kBinsPerLog2;
           const float2 nb2 = make_float2(-kBinsPerLog2, -kBinsPerLog2);
           const uint32_t inc = (i & 1) ? 0x10000u : 1u;
           uint32_t* hrow = hist32 + (i >> 1);
-#pragma unroll 1
-          for (int g = 0; g < 8; ++g) {
+          const float* kb = pv_stat ? blv : bias;
+          for_groups(s_addr, [&](int g, const uint32_t (&r)[16]) {
             uint32_t mw = sel_row_stats ? causal16(g, nin) : 0u;
             if (c == 0 && g == 0) mw &= ~1u;   // the sink is kept apart
-            if (!__any_sync(0xffffffffu, mw)) continue;
-            float v[16];
-            tmem_ld16(s_addr + g * 16, v);
-            const float2* b2 = reinterpret_cast<const float2*>(blv + g * 16);
+            if (!__any_sync(0xffffffffu, mw)) return;
+            const float2* b2 = reinterpret_cast<const float2*>(kb + g * 16);
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-              const float2 kap = __ffma2_rn(make_float2(v[j], v[j + 1]), sc2,
-                                            pv_stat ? b2[j / 2] : make_float2(bias[g * 16 + j], bias[g * 16 + j + 1]));
+              const float2 kap = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                            sc2, b2[j / 2]);
               const float2 bf = __ffma2_rn(kap, nb2, make_float2(kt8, kt8));
               // NaN-free: kappa finite or -inf
               const int ba = (int)fminf(fmaxf(bf.x, 0.f), (float)(NBIN - 1));
@@ -409,7 +421,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
               if ((mw >> j) & 1u) atomicAdd(hrow + ba * (TQ / 2), inc);
               if ((mw >> (j + 1)) & 1u) atomicAdd(hrow + bb * (TQ / 2), inc);
             }
-          }
+          });
         }
         tc_fence_before();
         mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
@@ -445,30 +457,46 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           mbar_arrive(&sh.qlo_ready);
         }
       } else if (pass == PASS_CAND) {
+        // the columns at or above the threshold (kappa from the split-operand scores) are
+        // candidates, written in column order with p = 2^(x - max) / sum; the sink apart
         const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
         uint16_t* ccol = A.ccol + rh * A.cap;
         float* cpr = A.cp + rh * A.cap;
+        for_groups(s_addr, [&](int g, const uint32_t (&r)[16]) {
+          const uint32_t mw = sel_row_stats ? causal16(g, nin) : 0u;
+          if (!__any_sync(0xffffffffu, mw)) return;
+          const float2* b2 = reinterpret_cast<const float2*>(bias + g * 16);
+          const float2* l2 = reinterpret_cast<const float2*>(lvn + g * 16);
+          float x[16];
+          uint32_t hits = 0u;
 #pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          float v[32];
-          tmem_ld32(s_addr + g4 * 32, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int jj = g4 * 32 + j;
-            if (sel_row_stats && jj < nin) {
-              const float s2 = fmaf(v[j], scale2, bias[jj]);
-              if (c == 0 && jj == 0) {
-                p0 = exp2f(s2 - m_used) * inv_l;
-              } else if (s2 + (pv_stat ? lvn[jj] : 0.f) >= thr) {
-                if (cand < A.cap) {
-                  ccol[cand] = (uint16_t)(c * TC + jj);
-                  cpr[cand] = exp2f(s2 - m_used) * inv_l;
-                }
-                ++cand;
-              }
-            }
+          for (int j = 0; j < 16; j += 2) {
+            const float2 xx = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
+                                         sc2, b2[j / 2]);
+            const float2 kap = pv_stat ? __fadd2_rn(xx, l2[j / 2]) : xx;
+            x[j] = xx.x;
+            x[j + 1] = xx.y;
+            hits |= (kap.x >= thr ? 1u : 0u) << j;
+            hits |= (kap.y >= thr ? 1u : 0u) << (j + 1);
           }
-        }
+          hits &= mw;
+          if (c == 0 && g == 0 && (mw & 1u)) {
+            p0 = exp2f(x[0] - m_used) * inv_l;
+            hits &= ~1u;
+          }
+          while (hits) {
+            const int j = __ffs(hits) - 1;
+            hits &= hits - 1u;
+            float xj = x[0];
+#pragma unroll
+            for (int q = 1; q < 16; ++q) xj = j == q ? x[q] : xj;   // select, no local memory
+            if (cand < A.cap) {
+              ccol[cand] = (uint16_t)(c * TC + g * 16 + j);
+              cpr[cand] = exp2f(xj - m_used) * inv_l;
+            }
+            ++cand;
+          }
+        });
         tc_fence_before();
         mbar_arrive(&sh.p_full[sb]);   // one barrier per score buffer (see the header)
         if (lane == 0) sh.prog[warp - 4] = G;

@@ -38,6 +38,18 @@ METRIC = "loop-step tokens/s at R loops + % of HBM/tensor roofline; KV bytes/tok
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes of one attention call (ncu dram__bytes_read.sum + dram__bytes_write.sum of
+# the call's kernels, one capture each) at a workload's sparse-loop shape; None where not
+# captured for the current kernels. Summaries and commands: profiles/.
+ATTN_TRAFFIC = {
+    "ouro-2.6b-shape-prefill-32k": {
+        "bytes": (158.77 + 211.36 + 315.78 + 127.90 + 520.55 + 17.00) * 1e6,
+        "per_kernel_mb": {"k_kv_stage": 370.13, "k_sel_bitmap": 443.68, "k_attn_tile<2>": 537.55},
+        "source": "kernel case sparse-attn 32k (4916 queries x 16 heads, 2048 + 1 carried "
+                  "columns, 2-bit residuals: the loop-2 call of this workload)"},
+}
+
+
 # Component toggles and loop schedules (paper §5.3 Figure 4: the contribution of each
 # lazy update; §4.1: dense early loops; §4.2: progressive pruning with smaller budgets).
 VARIANTS = {
@@ -754,10 +766,12 @@ def main():
                  "timing": timing_note}
     all_sparse = all(abytes[r][3] for r in abytes)
     if all_sparse:
-        attn_line = {"bound": "hbm", "kernel": "k_attn_tile (sparse, carried mass, tcgen05)",
+        tr = ATTN_TRAFFIC.get(cfg["name"]) if cfg.get("variant", "flashloop") == "flashloop" else None
+        attn_line = {"bound": "hbm", "kernel": "sparse attention call: k_kv_stage + k_sel_bitmap + "
+                     "k_attn_tile (tcgen05, carried mass)",
                      "achieved": attn_gbs, "peak": peak_h, "unit": "GB/s",
-                     "frac": attn_gbs / peak_h, "traffic": None,
-                     "peak_source": f"{pk_kind} HBM copy"}
+                     "frac": attn_gbs / peak_h, "traffic": tr["bytes"] if tr else None,
+                     "traffic_detail": tr, "peak_source": f"{pk_kind} HBM copy"}
     else:   # dense attention in some timed loop: tensor-bound on its algorithmic FLOP
         attn_line = {"bound": "tensor", "kernel": "k_attn_tile / k_attn_dense_tile (tcgen05)",
                      "achieved": attn_alg_flops / attn_s / 1e12, "peak": peak_t,

@@ -238,11 +238,11 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
             const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
                                         sc2, b2[j / 2]);
             const float2 d = __fadd2_rn(x, negm);
-            const __half2 hv = __floats2half2_rn(ex2_ftz(d.x), ex2_ftz(d.y));
-            const uint32_t ma = (uint32_t)((int)(mw << (31 - j)) >> 31);
-            const uint32_t mb = (uint32_t)((int)(mw << (30 - j)) >> 31);
-            const uint32_t pv = *reinterpret_cast<const uint32_t*>(&hv) & __byte_perm(ma, mb, 0x5410);
-            const __half2 ph = *reinterpret_cast<const __half2*>(&pv);
+            // non-members at -inf: 2^-inf = 0
+            const float da = (mw >> j) & 1u ? d.x : -INFINITY;
+            const float db = (mw >> (j + 1)) & 1u ? d.y : -INFINITY;
+            const __half2 ph = __floats2half2_rn(ex2_ftz(da), ex2_ftz(db));
+            const uint32_t pv = *reinterpret_cast<const uint32_t*>(&ph);
             hmax = __hmax2(hmax, ph);
             if (sum) acc = __fadd2_rn(acc, __half22float2(ph));
             pk[j / 2] = pv;

@@ -448,17 +448,15 @@ __device__ __forceinline__ void attn_tile_cta(const AttnParams& P, int h, int q0
             const float2* b2 = reinterpret_cast<const float2*>(bias + g * 16);
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
-              // x = s * scale2 + bias, P = 2^(x - m_used) for a pair of columns; members
-              // kept by a 16-bit lane mask (all ones or zero per column)
+              // x = s * scale2 + bias, P = 2^(x - m_used) for a pair of columns
               const float2 x = __ffma2_rn(make_float2(__uint_as_float(r[j]), __uint_as_float(r[j + 1])),
                                           sc2, b2[j / 2]);
               const float2 d = __fadd2_rn(x, negm);
-              const __half2 hv = __floats2half2_rn(ex2_ftz(d.x), ex2_ftz(d.y));
-              const uint32_t ma = (uint32_t)((int)(mw << (31 - j)) >> 31);
-              const uint32_t mb = (uint32_t)((int)(mw << (30 - j)) >> 31);
-              const uint32_t pm = __byte_perm(ma, mb, 0x5410);
-              const uint32_t pv = *reinterpret_cast<const uint32_t*>(&hv) & pm;
-              const __half2 ph = *reinterpret_cast<const __half2*>(&pv);
+              // non-members at -inf: 2^-inf = 0
+              const float da = (mw >> j) & 1u ? d.x : -INFINITY;
+              const float db = (mw >> (j + 1)) & 1u ? d.y : -INFINITY;
+              const __half2 ph = __floats2half2_rn(ex2_ftz(da), ex2_ftz(db));
+              const uint32_t pv = *reinterpret_cast<const uint32_t*>(&ph);
               if (detect) hmax = __hmax2(hmax, ph);
               acc = __fadd2_rn(acc, __half22float2(ph));
               pk[j / 2] = pv;

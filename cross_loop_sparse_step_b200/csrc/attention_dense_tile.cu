@@ -215,7 +215,6 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
     float m_true = -INFINITY, lvmax = -INFINITY, ktop = 0.f, thr = -INFINITY, p0 = 0.f;
     int cand = 0;
     uint16_t* hist = reinterpret_cast<uint16_t*>(smem + OFF_R1);
-    uint32_t* hist32 = reinterpret_cast<uint32_t*>(smem + OFF_R1);   // two rows' counts per word
     uint8_t* pt = smem + OFF_R1;
     const bool pv_stat = P.stat_kind == FL_STAT_PV;
     const float2 sc2 = make_float2(scale2, scale2);
@@ -388,22 +387,18 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
           if (stats) {
             if (valid) A.m1l[rh] = make_float2(m_used, lsum);
             ktop = m_true + (pv_stat ? lvmax : 0.f);
-            // the histogram takes the P region over (every thread saw the last P V^ finish);
-            // a row's counts are 16-bit halves of words shared with the neighbouring row,
-            // both in this warp
+            // the histogram takes the P region over (every thread saw the last P V^ finish)
             for (int b = 0; b < NBIN; ++b) hist[b * TQ + i] = 0;
-            __syncwarp();
           }
         }
       } else if (pass == PASS_HIST) {
         {
           // kappa = s * scale2 + bias + log2 ||V^|| binned by (ktop - kappa) * 8 below the
-          // row's upper bound; bins incremented by shared-memory atomics (no read-modify-
-          // write chain through a row's counts); rows that rank nothing have empty masks
+          // row's upper bound; each thread counts its own row's bins (16-bit counts in
+          // shared memory, no atomics); rows that rank nothing have empty masks
           const float kt8 = ktop * kBinsPerLog2;
           const float2 nb2 = make_float2(-kBinsPerLog2, -kBinsPerLog2);
-          const uint32_t inc = (i & 1) ? 0x10000u : 1u;
-          uint32_t* hrow = hist32 + (i >> 1);
+          uint16_t* hrow = hist + i;
           const float* kb = pv_stat ? blv : bias;
           for_groups(s_addr, [&](int g, const uint32_t (&r)[16]) {
             uint32_t mw = sel_row_stats ? causal16(g, nin) : 0u;
@@ -418,8 +413,8 @@ __global__ void __launch_bounds__(NTHR, 1) k_attn_dense_tile(const __grid_consta
               // NaN-free: kappa finite or -inf
               const int ba = (int)fminf(fmaxf(bf.x, 0.f), (float)(NBIN - 1));
               const int bb = (int)fminf(fmaxf(bf.y, 0.f), (float)(NBIN - 1));
-              if ((mw >> j) & 1u) atomicAdd(hrow + ba * (TQ / 2), inc);
-              if ((mw >> (j + 1)) & 1u) atomicAdd(hrow + bb * (TQ / 2), inc);
+              if ((mw >> j) & 1u) hrow[ba * TQ] += 1;
+              if ((mw >> (j + 1)) & 1u) hrow[bb * TQ] += 1;
             }
           });
         }

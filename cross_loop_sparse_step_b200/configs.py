@@ -10,7 +10,7 @@ width of loop r (0: stored unquantised).
 """
 import math
 
-C1 = dict(
+TINY_FP32 = dict(
     name="tiny-looped-block-fp32",
     n_tok=256, d_model=256, n_heads=4, head_dim=64, d_ffn=1024, n_layers=1, n_loops=4,
     dtype="f32", first_sparse=2,
@@ -21,11 +21,11 @@ C1 = dict(
 )
 
 # the same block with shrinking budgets, to exercise pruning of carried columns
-C1_SHRINK = dict(C1, name="tiny-looped-block-fp32-shrink",
-                 tok_frac={2: 0.5, 3: 0.25, 4: 0.125},
-                 col_k={2: 32, 3: 16, 4: 8})
+TINY_FP32_SHRINK = dict(TINY_FP32, name="tiny-looped-block-fp32-shrink",
+                        tok_frac={2: 0.5, 3: 0.25, 4: 0.125},
+                        col_k={2: 32, 3: 16, 4: 8})
 
-C2 = dict(
+PREFILL_4K = dict(
     name="ouro-1.4b-shape-prefill-4k",
     n_tok=4096, d_model=2048, n_heads=16, head_dim=128, d_ffn=5632, n_layers=24,
     n_loops=4, dtype="bf16", first_sparse=2,
@@ -35,7 +35,7 @@ C2 = dict(
     bias_frac=0.02, bias_value=4.0, synthetic_delta=True,
 )
 
-C3 = dict(
+PREFILL_32K = dict(
     name="ouro-2.6b-shape-prefill-32k",
     n_tok=32768, d_model=2048, n_heads=16, head_dim=128, d_ffn=5632, n_layers=48,
     n_loops=4, dtype="bf16", first_sparse=2,
@@ -64,15 +64,15 @@ def c4(n_loops, res_bits):
 # 64 sequences with 16K..32K cached tokens each; the generated token's loop r >= 2 step
 # per layer (its KV appended, sparse attention over 1024 carried columns plus the sink,
 # the block on the 64 new rows).
-C5 = dict(
+DECODE_B64 = dict(
     name="ouro-2.6b-shape-decode-b64",
     batch=64, ctx_min=16384, ctx_max=32768, d_model=2048, n_heads=16, head_dim=128,
     d_ffn=5632, n_layers=48, n_loops=4, dtype="bf16", col_k=1024, base_bits=8,
     res_bits=2, group=32, active_frac=0.15, bias_frac=0.02, bias_value=4.0, decode=True,
 )
 
-CONFIGS = {c["name"]: c for c in (C1, C1_SHRINK, C2, C3, c4(8, 2), c4(8, 4), c4(16, 2),
-                                   c4(16, 4), C5)}
+CONFIGS = {c["name"]: c for c in (TINY_FP32, TINY_FP32_SHRINK, PREFILL_4K, PREFILL_32K, c4(8, 2),
+                                   c4(8, 4), c4(16, 2), c4(16, 4), DECODE_B64)}
 
 
 def active_counts(cfg):

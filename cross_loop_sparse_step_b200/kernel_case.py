@@ -25,7 +25,7 @@ import torch
 
 from cross_loop_sparse_step_b200 import configs, fl, synth
 
-SHAPES = {"4k": configs.C2, "32k": configs.C3}
+SHAPES = {"4k": configs.PREFILL_4K, "32k": configs.PREFILL_32K}
 
 
 def make_store(cfg, act, g):

@@ -72,7 +72,7 @@ def _nested_sets(rs, n, counts, R):
 
 def test_32k_select_bit_exact():
     fl = _fl()
-    cfg = configs.C3
+    cfg = configs.PREFILL_32K
     N, d = cfg["n_tok"], cfg["d_model"]
     k = configs.active_counts(cfg)[2]
     g = synth.rng(31)
@@ -89,7 +89,7 @@ def test_32k_select_bit_exact():
 
 def test_32k_quant_bit_exact():
     fl = _fl()
-    cfg = configs.C3
+    cfg = configs.PREFILL_32K
     N, H, hd, g = cfg["n_tok"], cfg["n_heads"], cfg["head_dim"], cfg["group"]
     k2 = configs.active_counts(cfg)[2]
     rs = synth.rng(32)
@@ -116,7 +116,7 @@ def test_32k_dense_producer_sampled():
     queries (the kernel's grid is one CTA per query and head, so a subset is the same
     launch configuration per query)."""
     fl = _fl()
-    cfg = configs.C3
+    cfg = configs.PREFILL_32K
     N, H, hd, g, k = cfg["n_tok"], cfg["n_heads"], cfg["head_dim"], cfg["group"], 2048
     rs = synth.rng(33)
     ost = okv.LayerKV(N, H, hd, g, 8, {}, 1)
@@ -163,7 +163,7 @@ def test_32k_dense_producer_sampled():
 def test_sparse_step_full_size_sampled(name, R, loop, bits, k, kn, sample):
     fl = _fl()
     if name.startswith("32k"):
-        cfg = configs.C3
+        cfg = configs.PREFILL_32K
         counts = configs.active_counts(cfg)
         g = cfg["group"]
     else:

@@ -64,7 +64,7 @@ def _decode_hat(store, r, H, hd, g, N):
     return out
 
 
-@pytest.mark.parametrize("cfg", [configs.C1, configs.C1_SHRINK], ids=["c1", "c1-shrink"])
+@pytest.mark.parametrize("cfg", [configs.TINY_FP32, configs.TINY_FP32_SHRINK], ids=["c1", "c1-shrink"])
 def test_tiny_block_end_to_end(cfg):
     from cross_loop_sparse_step_b200 import fl
     N, d, H, hd, F, L, R = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn",
@@ -109,7 +109,7 @@ def test_tiny_block_end_to_end(cfg):
 
 
 def _c2_like(n_layers):
-    cfg = dict(configs.C2)
+    cfg = dict(configs.PREFILL_4K)
     cfg["n_layers"] = n_layers
     return cfg
 
@@ -167,7 +167,7 @@ def test_4k_shape_two_layers_two_loops_fp32():
 def test_4k_workload_24_layers_invariants():
     """The benchmark's launch configuration: 24 layers, loops 1..3 with the lazy updates."""
     from cross_loop_sparse_step_b200 import fl
-    cfg = dict(configs.C2)
+    cfg = dict(configs.PREFILL_4K)
     R = 3
     N, d, H, hd, F, L = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn",
                                           "n_layers"))

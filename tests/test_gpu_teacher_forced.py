@@ -266,7 +266,7 @@ def run_teacher_forced(cfg, R, n_tap=256, n_dense_check=32, seed=0):
 
 def test_4k_workload_all_layers_all_loops():
     """The benchmarked 4K workload: 24 layers, loops 1..4, every stage of every layer."""
-    rep = run_teacher_forced(dict(configs.C2), configs.C2["n_loops"])
+    rep = run_teacher_forced(dict(configs.PREFILL_4K), configs.PREFILL_4K["n_loops"])
     print("teacher-forced 4K:", rep)
     assert all(v > 0 for v in rep["checked"].values())
 
@@ -275,6 +275,6 @@ def test_32k_workload_all_layers_loops_1_2():
     """The 32K Ouro-2.6B-shape workload the benchmark times: all 48 layers, the dense loop 1
     (statistics for loop 2, k = 2048 of up to 32K columns) and the sparse loop 2 over the
     column-range tiles, on a sample of tokens."""
-    rep = run_teacher_forced(dict(configs.C3), 2, n_tap=64, n_dense_check=10)
+    rep = run_teacher_forced(dict(configs.PREFILL_32K), 2, n_tap=64, n_dense_check=10)
     print("teacher-forced 32K:", rep)
     assert all(v > 0 for v in rep["checked"].values())

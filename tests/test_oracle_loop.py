@@ -94,7 +94,7 @@ def test_dense_kv_bytes_match_pages():
             assert dense == int(rhs) * 2 ** 30
 
 
-@pytest.mark.parametrize("cfg,want", [(configs.C2, 6144.0), (configs.C3, 4608 + 0.45 * 1536)])
+@pytest.mark.parametrize("cfg,want", [(configs.PREFILL_4K, 6144.0), (configs.PREFILL_32K, 4608 + 0.45 * 1536)])
 def test_kv_bytes_closed_form_configs(cfg, want):
     n_act = configs.active_counts(cfg)
     got = loop.kv_bytes_per_token(cfg["n_tok"], cfg["d_model"], n_act, cfg["base_bits"],
@@ -105,7 +105,7 @@ def test_kv_bytes_closed_form_configs(cfg, want):
 
 
 def test_c1_runs_and_is_reproducible():
-    cfg = configs.C1
+    cfg = configs.TINY_FP32
     g = synth.rng(0)
     layers = synth.model_weights(g, cfg["n_layers"], cfg["d_model"], cfg["d_ffn"])
     h0 = synth.embeddings(g, cfg["n_tok"], cfg["d_model"])

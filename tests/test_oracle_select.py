@@ -49,9 +49,9 @@ def test_active_counts_agree():
             k = select.active_count(cfg["tok_frac"][r], cfg["n_tok"], prev)
             assert k == want[r], (cfg["name"], r)
             prev = k
-    assert configs.active_counts(configs.C2)[2] == 820
-    assert configs.active_counts(configs.C3)[2] == 4916
-    assert configs.active_counts(configs.C1)[2] == 64
+    assert configs.active_counts(configs.PREFILL_4K)[2] == 820
+    assert configs.active_counts(configs.PREFILL_32K)[2] == 4916
+    assert configs.active_counts(configs.TINY_FP32)[2] == 64
 
 
 def test_pareto_pair_concentrates_change():

@@ -4,28 +4,36 @@
 // the carried unselected contribution; §4.4: the selected K/V are brought into compact
 // on-chip buffers and QK^T / PV run on them).
 //
-// The queries of a tile carry different column sets. The CTA takes the union of the
-// tile's sets (a bitmap over the tokens, then ranks by prefix popcounts), walks the
-// union in chunks of 128 columns, and runs every chunk as a dense 128 x 128 tile on the
-// tensor cores with each query's membership as a mask:
-//   producer warps (two groups of four, one per pipeline stage) decode the chunk's K^
-//     and V^ rows - int8 base plus the residual chain of every loop that rewrote the
-//     column, fmaf(code, s, z) added in loop order, exactly the store's reconstruction -
-//     and write them as fp16 operand tiles in the 128-byte-swizzle layout, both as
-//     [column][element] rows: K^ is the K-major B operand of Q K^T, V^ the MN-major B
-//     operand of P V^;
-//   the MMA warp issues S = Q K^T into one of two TMEM score buffers, then, once the
-//     softmax has written P, O += P V^ into the TMEM output accumulator
-//     (tcgen05.mma kind::f16, M 128, N 128, fp32 accumulation);
-//   the softmax warps (thread = query row = TMEM lane) read their row of S, keep the
-//     columns their set names (the set is walked in step with the chunks), update an
-//     online maximum - the output is rescaled only when the maximum grows by more than
-//     2^8, so P stays below 256 in fp16 - and write P = 2^(s - max) as fp16; the row sum
-//     is taken over the fp16 values the MMA uses. At the end
-//     o = u + m * O / sum, with m the cached mass and u the unselected contribution.
-// Operand precision: q, K^, V^ and P enter the MMAs as fp16 (11 significant bits);
-// sums are binary32. Every wait is bounded; a wait that runs out records FL_ERR_TIMEOUT,
-// the CTA drains its MMAs, frees TMEM and returns.
+// The queries of a tile carry different column sets. The CTA walks chunks of 128 columns
+// and runs every chunk as a dense 128 x 128 tile on the tensor cores, each query's
+// membership applied as a mask. Three modes:
+//   CONTIG  chunks of the plain column range [0, t_max] of the tile - taken where the
+//           tile's union is nearly every column (a budget that is a sizeable part of the
+//           prompt); membership read from the bitmap of each query's set (16 bytes per
+//           query and chunk), masked causally;
+//   UNION   chunks of the union of the tile's sets (a bitmap over the tokens and prefix
+//           popcounts for ranks); the producers turn the union's words and each query's
+//           bitmap words over a chunk's span into its 128-bit mask;
+//   DECODE  the union, the producers decoding K^ and V^ from the quantised store (int8
+//           base plus the residual chain of every loop that rewrote the column, fmaf(code,
+//           s, z) added in loop order) - for calls of one tile, where nothing is shared.
+// In CONTIG and UNION the store has been staged once per call as fp16 rows (kv_stage.cu)
+// and the producers gather a chunk's K^ and V^ rows with cp.async, 16 lanes per 256-byte
+// row, into the 128-byte-swizzle K-major layout (K^ as [column][element], V^ the same and
+// read as an MN-major operand). Roles:
+//   producer warps (two groups of four, one per pipeline stage): the chunk's columns and
+//     their rows, the column biases, the masks (UNION);
+//   the MMA warp issues S = Q K^T into one of two TMEM score buffers and, once the softmax
+//     has written P, O += P V^ into the TMEM output accumulator (tcgen05.mma kind::f16,
+//     M 128, N 128, fp32 accumulation), each as soon as its barrier completes;
+//   the softmax warps (thread = query row = TMEM lane) take one pass per chunk against a
+//     running maximum, rescaling O only when it grows by more than 2^8 (P stays below 256
+//     in fp16), and write P = 2^(s - max) as fp16; the row sum is taken over the fp16
+//     values the MMA uses. At the end o = u + m * O / sum, with m the cached mass and u
+//     the unselected contribution.
+// Operand precision: q, K^, V^ and P enter the MMAs as fp16 (11 significant bits); sums
+// are binary32. Every wait is bounded; a wait that runs out records FL_ERR_TIMEOUT, the
+// CTA drains its MMAs, frees TMEM and returns.
 //
 // Taken for head_dim 128 over a quantised store (8-bit base, 2/4/8-bit residuals) when
 // the call writes no statistics (none requested, or in place with an unchanged budget).

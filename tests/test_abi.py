@@ -109,3 +109,43 @@ def test_host_validation_without_gpu():
     assert fl._append(ctypes.byref(kv), 2, p, p, 0, p, 1, 2 ** 31 - 1, None) == 2
     a = fl.AttnArgs()
     assert fl._attn(ctypes.byref(a), None) == 1
+
+
+def test_attention_workspace_sizes_without_gpu():
+    """The attention calls' workspace, sized on the host: a sparse call of many queries
+    stages the store as fp16 rows and its column sets as bitmaps; a call of few queries
+    streams its columns and needs none; a dense call that hands statistics on stages K^
+    twice (hi and lo) and V^. A call given less is rejected before any launch."""
+    from cross_loop_sparse_step_b200 import fl
+    N, H, hd = 32768, 16, 128
+    kv = fl.KvDesc()
+    kv.n_tok, kv.n_heads, kv.head_dim, kv.group, kv.base_bits, kv.n_loops = N, H, hd, 32, 8, 2
+    kv.res_bits[2] = 2
+    kv.slot = 16
+    kv.vnorm = 16
+    p = 16
+    staged = H * N * hd * 2                      # one fp16 [H][N][hd] array
+    words = (N + 127) // 128 * 4                 # bitmap words per (query, head)
+
+    a = fl.AttnArgs()
+    a.q, a.q_dt, a.q_tok, a.kv, a.loop, a.out, a.out_dt = p, 0, p, ctypes.pointer(kv), 2, p, 0
+    a.sel, a.mass, a.unsel, a.stat_rows, a.sel_stride = p, p, p, N, 2049
+    a.n_q = 4916
+    need = fl._attn_ws(ctypes.byref(a))
+    assert need == (2 * staged + 255) // 256 * 256 + H * a.n_q * words * 4
+    assert fl._attn(ctypes.byref(a), None) == 7          # no workspace: rejected
+    a.ws, a.ws_bytes = p, need - 1
+    assert fl._attn(ctypes.byref(a), None) == 7
+
+    a.ws, a.ws_bytes = None, 0
+    a.n_q = 32                                           # decode-sized: streamed, no workspace
+    assert fl._attn_ws(ctypes.byref(a)) == 0
+
+    d = fl.AttnArgs()
+    d.q, d.q_dt, d.q_tok, d.kv, d.loop, d.out, d.out_dt = p, 0, p, ctypes.pointer(kv), 1, p, 0
+    d.n_q, d.stat_rows, d.k_next, d.out_stride, d.stat_kind = N, N, 2048, 2049, 0
+    d.sel_out, d.mass_out, d.unsel_out = p, p, p
+    need_d = fl._attn_ws(ctypes.byref(d))
+    assert need_d >= 3 * staged + H * N * words * 4      # K^ hi, K^ lo, V^; bitmaps of S'
+    d.sel_out = d.mass_out = d.unsel_out = None          # no statistics: K^ and V^ only
+    assert fl._attn_ws(ctypes.byref(d)) == 2 * staged

@@ -258,9 +258,17 @@ typedef struct {
   int32_t out_stride;                  /* >= k_next + 1; rows as stat_rows */
   int32_t stat_kind;                   /* fl_stat_kind */
   void* out; fl_dtype out_dt;          /* device [n_q][H][hd] */
-  void* ws; size_t ws_bytes;
+  void* ws; size_t ws_bytes;          /* device workspace, see below */
 } fl_attn_args;
 
+/* Device workspace of a call (a fl_attn_args whose ws fields are ignored), 0 if none:
+ * for a sparse call of more than 128 queries (head_dim 128, no statistics written or in
+ * place with an unchanged budget) the store staged once as fp16 rows, K^ and V^
+ * [H][n_tok][hd], then the carried sets as column bitmaps [H][n_q][ceil(n_tok/128)*4]
+ * uint32; for a dense call the staged K^ and V^ (and K^ - fp16(K^) when it writes
+ * statistics) after the statistics producer's buffers. Calls of at most 32 sparse
+ * queries need none. fl_sparse_loop_attn rejects a call whose ws_bytes is smaller
+ * (FL_ERR_WORKSPACE, before any launch). The workspace serves one call at a time. */
 size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a);
 fl_status fl_sparse_loop_attn(const fl_attn_args* a, void* stream);
 

@@ -266,7 +266,7 @@ typedef struct {
  * place with an unchanged budget) the store staged once as fp16 rows, K^ and V^
  * [H][n_tok][hd], then the carried sets as column bitmaps [H][n_q][ceil(n_tok/128)*4]
  * uint32; for a dense call the staged K^ and V^ (and K^ - fp16(K^) when it writes
- * statistics) after the statistics producer's buffers. Calls of at most 32 sparse
+ * statistics) after the statistics producer's buffers. Sparse calls of at most 128
  * queries need none. fl_sparse_loop_attn rejects a call whose ws_bytes is smaller
  * (FL_ERR_WORKSPACE, before any launch). The workspace serves one call at a time. */
 size_t fl_sparse_loop_attn_workspace_bytes(const fl_attn_args* a);

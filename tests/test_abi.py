@@ -149,3 +149,29 @@ def test_attention_workspace_sizes_without_gpu():
     assert need_d >= 3 * staged + H * N * words * 4      # K^ hi, K^ lo, V^; bitmaps of S'
     d.sel_out = d.mass_out = d.unsel_out = None          # no statistics: K^ and V^ only
     assert fl._attn_ws(ctypes.byref(d)) == 2 * staged
+
+
+def test_loop_workspace_covers_the_attention_calls():
+    """fl_loop_step's workspace holds, besides the block's buffers, the largest attention
+    workspace of its schedule: at the 32K shape the dense loop 1 with statistics for loop
+    2 (staged K^ hi, K^ lo, V^ and the bitmaps of S'), more than a sparse loop's staged
+    K^, V^ and set bitmaps of its active rows."""
+    from cross_loop_sparse_step_b200 import configs, fl
+    cfg = configs.PREFILL_32K
+    N, d, H, hd, F = (cfg[k] for k in ("n_tok", "d_model", "n_heads", "head_dim", "d_ffn"))
+    m = fl.Model()
+    m.n_tok, m.d_model, m.n_heads, m.head_dim, m.d_ffn, m.n_layers, m.dt = N, d, H, hd, F, 1, 1
+    n_active = configs.active_counts(cfg)
+    col_k = {r: cfg["col_k"][r] for r in range(2, cfg["n_loops"] + 1)}
+    sched = fl.make_schedule(cfg["n_loops"], cfg["first_sparse"], n_active, col_k)
+    total = fl._loop_ws(ctypes.byref(m), ctypes.byref(sched))
+    staged = H * N * hd * 2
+    words = (N + 127) // 128 * 4
+    dense_min = 3 * staged + H * N * words * 4          # loop 1's staging and S' bitmaps
+    sparse = 2 * staged + H * n_active[2] * words * 4
+    assert total > dense_min > sparse
+    # a schedule without statistics: the largest call is a dense one over staged K^, V^
+    sched0 = fl.make_schedule(cfg["n_loops"], cfg["n_loops"] + 1, {r: N for r in range(1, 5)},
+                              {r: 0 for r in range(2, 5)})
+    total0 = fl._loop_ws(ctypes.byref(m), ctypes.byref(sched0))
+    assert total0 >= 2 * staged and total0 < total
